@@ -1,0 +1,152 @@
+"""Plant plausible mistakes in the CPU oracle and check that the pins catch each one.
+
+Every case patches one oracle function with a typical slip (transposed operand,
+dropped normalisation, wrong sign, wrong index or bit order, wrong tie rule,
+wrong constant) and asserts that at least one pin test from
+``test_oracle_pins`` fails.  Nothing here touches a GPU.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle.codebook as ocb
+import oracle.hadamard as oh
+import oracle.q4_0 as oq4
+import oracle.qjl as oqjl
+import oracle.rrq as orrq
+from tests import test_oracle_pins as pins
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_mutation_signs_after_transform(monkeypatch):
+    """Π = D·H/√d instead of H·D/√d."""
+    good = oh.rotation_matrix
+
+    def bad(seed, d):
+        h = oh.sylvester(d)
+        s = oh.rotation_signs(seed, d)
+        return s[:, None] * h / math.sqrt(d)
+
+    monkeypatch.setattr(oh, "rotation_matrix", bad)
+    monkeypatch.setattr(orrq, "rotation_matrix", bad)
+    assert _fails(pins.test_rotation_is_orthogonal_and_signs_first, 128)
+    monkeypatch.setattr(oh, "rotation_matrix", good)
+
+
+def test_mutation_missing_normalisation(monkeypatch):
+    def bad(seed, d):
+        return oh.sylvester(d) * oh.rotation_signs(seed, d)[None, :]
+
+    monkeypatch.setattr(oh, "rotation_matrix", bad)
+    monkeypatch.setattr(orrq, "rotation_matrix", bad)
+    assert _fails(pins.test_rotation_is_orthogonal_and_signs_first, 64)
+
+
+def test_mutation_decode_with_pi_instead_of_pi_transpose(monkeypatch):
+    good = orrq.rotate
+
+    def bad(x, seed, inverse=False):
+        return good(x, seed, inverse=False)
+
+    monkeypatch.setattr(orrq, "rotate", bad)
+    assert _fails(pins.test_round_trip_nmse_matches_lloyd_max_distortion, 4)
+
+
+def test_mutation_tie_rule(monkeypatch):
+    good = np.searchsorted
+
+    def bad_encode(x, bits, seed, levels=None):
+        enc = good_encode(x, bits, seed, levels)
+        tau = ocb.thresholds(ocb.lloyd_max(bits) if levels is None else levels)
+        enc.codes = good(tau, enc.u.ravel(), side="right").reshape(enc.codes.shape)
+        enc.packed = orrq.pack_codes(enc.codes, bits)
+        return enc
+
+    good_encode = orrq.encode
+    monkeypatch.setattr(orrq, "encode", bad_encode)
+    assert _fails(pins.test_zero_vector_and_exact_ties)
+
+
+def test_mutation_msb_first_packing(monkeypatch):
+    good = orrq.pack_codes
+
+    def bad(codes, bits):
+        codes = np.asarray(codes, dtype=np.int64)
+        n, d = codes.shape
+        planes = ((codes[:, :, None] >> np.arange(bits)[None, None, :]) & 1).astype(np.uint8)
+        return np.packbits(planes.reshape(n, d * bits), axis=1, bitorder="big")
+
+    monkeypatch.setattr(orrq, "pack_codes", bad)
+    assert _fails(pins.test_pack_matches_bitwise_reference, 4)
+    monkeypatch.setattr(orrq, "pack_codes", good)
+
+
+def test_mutation_centroid_sign(monkeypatch):
+    """Lloyd update with φ(τ_k) − φ(τ_{k−1}) (sign flipped) must miss the page values."""
+    ocb._lloyd_max.cache_clear()
+    good_phi = ocb._phi
+    monkeypatch.setattr(ocb, "_phi", lambda x: -good_phi(x))
+    try:
+        assert _fails(pins.test_codebook_page_values)
+    except (ValueError, ZeroDivisionError, OverflowError):
+        pass  # a diverging iteration is also caught
+    finally:
+        monkeypatch.setattr(ocb, "_phi", good_phi)
+        ocb._lloyd_max.cache_clear()
+
+
+def test_mutation_q4_0_nibble_order(monkeypatch):
+    good = oq4.encode
+
+    def bad(x, seed, rotate_first=True):
+        enc = good(x, seed, rotate_first)
+        b = enc.blocks.reshape(enc.blocks.shape[0], -1, 18).copy()
+        b[:, :, 2:] = ((b[:, :, 2:] & 0x0F) << 4) | (b[:, :, 2:] >> 4)
+        enc.blocks = b.reshape(enc.blocks.shape)
+        return enc
+
+    monkeypatch.setattr(oq4, "encode", bad)
+    assert _fails(pins.test_q4_0_hand_worked_blocks)
+
+
+def test_mutation_q4_0_unsigned_max(monkeypatch):
+    """Using +max|x| instead of the signed extreme for Δ."""
+    def bad(x, seed, rotate_first=True):
+        x = np.asarray(x, dtype=np.float64)
+        y = orrq.rotate(x, seed) if rotate_first else x
+        flipped = good(np.abs(y) * np.sign(y + 0.0) * 1.0, 0, rotate_first=False)
+        m = np.abs(y.reshape(y.shape[0], -1, 32)).max(axis=2)
+        delta = (m.astype(np.float32) / np.float32(-8.0))
+        b = flipped.blocks.reshape(y.shape[0], -1, 18).copy()
+        dh = delta.astype(np.float16).view(np.uint16)
+        b[:, :, 0] = dh & 0xFF
+        b[:, :, 1] = dh >> 8
+        flipped.blocks = b.reshape(flipped.blocks.shape)
+        return flipped
+
+    good = oq4.encode
+    monkeypatch.setattr(oq4, "encode", bad)
+    assert _fails(pins.test_q4_0_hand_worked_blocks)
+
+
+@pytest.mark.parametrize("factor", [1.0, math.pi / 2])
+def test_mutation_qjl_constant(monkeypatch, factor):
+    """Dropping √(π/2) (or squaring it) biases the estimator."""
+    good = oqjl.estimate_residual_dot
+
+    def bad(q_rot, s_matrix, packed_signs, rnorm):
+        return good(q_rot, s_matrix, packed_signs, rnorm) / math.sqrt(math.pi / 2) * factor
+
+    monkeypatch.setattr(oqjl, "estimate_residual_dot", bad)
+    assert _fails(pins.test_qjl_estimator_unbiased_monte_carlo)
