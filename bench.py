@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark: fp16 KV-cache vectors encoded + decoded per second on B200.
+
+Workload (one step): the fp16 K cache [32768 tokens × 8 KV heads × 128]
+(262,144 vectors; 2 % outlier channels ×15, log-normal per-token scale),
+encoded at 4 bits (randomized Hadamard rotation + N(0,1) Lloyd–Max codes +
+fp32 norm) and decoded back to fp16, through the C ABI (rrq_encode,
+rrq_decode).  Inputs are resident in HBM before timing starts; the 126 MB L2 is
+flushed (a 256 MiB write) before every timed kernel, and only the kernels are
+inside the CUDA-event pairs.  Multi-GPU (torchrun): every rank processes its
+own batch of the same size (weak scaling, no collective on the data path);
+the time is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (the plain fp64 restatement under
+``oracle/``) on a bounded sample of the same workload instead.
+
+Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV vectors/s encode+decode (d=128,b=4, fp16); achieved HBM GB/s vs peak"
+UNIT = "vectors/s"
+TOKENS, HEADS, D, BITS = 32768, 8, 128, 4
+N_VEC = TOKENS * HEADS
+BYTES_PER_VEC_ENC = D * 2 + D * BITS // 8 + 4   # read fp16, write codes + fp32 norm
+BYTES_PER_VEC_DEC = D * BITS // 8 + 4 + D * 2   # read codes + norm, write fp16
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["random_rotation_kv_b200/csrc/rrq_device.cuh",
+                  "random_rotation_kv_b200/csrc/quant_kernels.cuh",
+                  "random_rotation_kv_b200/csrc/rrq_params.h"]
+
+
+def workload_config(extra=None):
+    cfg = {"workload": "kv-cache K fp16 [32768 tokens x 8 kv heads x 128], 4-bit RHT + Lloyd-Max, "
+                       "encode+decode",
+           "vectors_per_gpu": N_VEC, "d": D, "bits": BITS, "io_dtype": "f16",
+           "rotation_seed": 42,
+           "l2": "flushed by a 256 MiB write before every timed kernel"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        entry = rec[kernel]
+        if entry.get("source_hash") != kernel_source_hash():
+            return None
+        return float(entry["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append((time.time(), ln.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        return self.lines
+
+    @staticmethod
+    def summarize(lines, t0, t1):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons, n = [], None, set(), 0
+        for t, ln in lines or []:
+            if not (t0 <= t <= t1 + 0.15):
+                continue
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            n += 1
+            for name, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": n}
+
+
+def gpu_id_for(torch, dev):
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        return str(dev)
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_step_time(x_sample: np.ndarray, reps: int = 1) -> float:
+    """Seconds for the oracle to encode + decode x_sample (fp16 [n, 128]), best of reps."""
+    from oracle import rrq as orc
+    best = float("inf")
+    for _ in range(reps):
+        t = time.perf_counter()
+        enc = orc.encode(x_sample.astype(np.float64), BITS, 42)
+        orc.decode(enc.packed, enc.norms, BITS, D, 42, out_dtype="f16")
+        best = min(best, time.perf_counter() - t)
+    return best
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(x_flat: np.ndarray, budget_s: float = 12.0):
+    """The oracle as it stands on a bounded sample of the workload."""
+    n0 = 8192
+    t0 = oracle_step_time(x_flat[:n0])
+    n = int(min(x_flat.shape[0], max(n0, n0 * budget_s / max(t0, 1e-3) / 2)))
+    t = oracle_step_time(x_flat[:n])
+    return {"value": n / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {n} of the {x_flat.shape[0]} workload vectors, encode+decode, "
+                      f"numpy fp64 (dense rotation matrix), {t:.2f} s wall"}
+
+
+# ------------------------------------------------------------ reference
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return  # rank 0 alone runs the CPU reference
+    from random_rotation_kv_b200 import workloads as W
+    w = W.kv()
+    x = w.flat()
+    # size each step's sample so that warm-up + timed steps take about
+    # --ref-budget seconds of CPU in total, whatever --steps is
+    rate = 2048 / oracle_step_time(x[:2048])
+    per_step = args.ref_budget * rate / (args.steps + args.warmup)
+    n_sample = int(min(args.ref_sample, max(128, per_step)))
+    for _ in range(args.warmup):
+        oracle_step_time(x[:n_sample])
+    times = [oracle_step_time(x[:n_sample]) for _ in range(args.steps)]
+    total = sum(times)
+    value = n_sample * args.steps / total
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config({"sample_vectors_per_step": n_sample}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"first {n_sample} workload vectors per step, encode+decode"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    from random_rotation_kv_b200 import binding as B
+    from random_rotation_kv_b200 import workloads as W
+
+    w = W.kv(seed=1002 + rank)  # each rank its own batch
+    x_host = w.flat()
+    x = torch.from_numpy(x_host).to(dev)
+    codes = torch.empty(N_VEC, D * BITS // 8, dtype=torch.uint8, device=dev)
+    norms = torch.empty(N_VEC, dtype=torch.float32, device=dev)
+    out = torch.empty(N_VEC, D, dtype=torch.float16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        flush.fill_(1)
+        if evs:
+            evs[0].record(stream)
+        B.rrq_encode(x, BITS, 42, codes=codes, norms=norms)
+        if evs:
+            evs[1].record(stream)
+        flush.fill_(2)
+        if evs:
+            evs[2].record(stream)
+        B.rrq_decode(codes, norms, D, BITS, 42, out_dtype=torch.float16, out=out)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    # keep the clocks in steady state before the timed region
+    t_end = time.time() + 0.5
+    while time.time() < t_end:
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(gpu_id_for(torch, dev)) if rank == 0 and not args.no_clocks else None
+    if sampler:
+        sampler.start()
+    barrier()
+    t0 = time.time()
+    for k in range(args.steps):
+        step(evs[k])
+    barrier()
+    t1 = time.time()
+    clocks = ClockSampler.summarize(sampler.stop(), t0, t1) if sampler else None
+    enc_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(enc_ms) + sum(dec_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * N_VEC * args.steps / (total_ms / 1e3)
+
+    # end to end through the public API: pinned host -> device -> encode -> decode -> host
+    x_pin = torch.from_numpy(x_host).pin_memory()
+    out_pin = torch.empty(N_VEC, D, dtype=torch.float16).pin_memory()
+    x_e2e = torch.empty_like(x)
+
+    def e2e_step():
+        x_e2e.copy_(x_pin, non_blocking=True)
+        B.rrq_encode(x_e2e, BITS, 42, codes=codes, norms=norms)
+        B.rrq_decode(codes, norms, D, BITS, 42, out_dtype=torch.float16, out=out)
+        out_pin.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * N_VEC * args.e2e_steps / (e2e_ms / 1e3)
+    assert torch.equal(out_pin, out.cpu())
+
+    if rank == 0:
+        peak, peak_kind = peaks()
+        enc_avg = sum(enc_ms) / len(enc_ms)
+        dec_avg = sum(dec_ms) / len(dec_ms)
+        dom, dom_ms, dom_bytes = (("encode", enc_avg, BYTES_PER_VEC_ENC) if enc_avg >= dec_avg
+                                  else ("decode", dec_avg, BYTES_PER_VEC_DEC))
+        achieved = dom_bytes * N_VEC / (dom_ms / 1e3) / 1e9
+        traffic = recorded_traffic(dom + "_kernel")
+        step_gbs = (BYTES_PER_VEC_ENC + BYTES_PER_VEC_DEC) * N_VEC / (ms_per_step / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": workload_config({"parallelism": f"dp{world} (independent batches)"}),
+            "roofline": {"bound": "hbm", "kernel": dom + "_kernel", "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_kind} copy bandwidth",
+                         "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dom_bytes * N_VEC},
+            "hbm": {"encode_us": 1e3 * enc_avg, "decode_us": 1e3 * dec_avg,
+                    "encode_gbs": BYTES_PER_VEC_ENC * N_VEC / (enc_avg / 1e3) / 1e9,
+                    "decode_gbs": BYTES_PER_VEC_DEC * N_VEC / (dec_avg / 1e3) / 1e9,
+                    "step_gbs": step_gbs, "step_frac_of_measured": step_gbs / peak,
+                    "step_frac_of_nominal_8tbs": step_gbs / NOMINAL_HBM_GBS},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": N_VEC * D * 2,
+                    "d2h_bytes_per_step": N_VEC * D * 2},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(x_host)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["rrq", "reference"], default="rrq")
+    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--ref-sample", type=int, default=16384,
+                    help="largest number of vectors per reference (oracle) step")
+    ap.add_argument("--ref-budget", type=float, default=90.0,
+                    help="seconds of CPU the whole reference run should take")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps, always
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

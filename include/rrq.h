@@ -1,0 +1,212 @@
+/*
+ * rrq.h — random-rotation vector quantisation for KV-cache and embedding vectors
+ * on NVIDIA B200 (sm_100a).  C ABI of librrq.so.
+ *
+ * The method ("Random-rotation quantization" page, brain.bigb.es, intro "the
+ * scheme", steps 1–3): rotate each vector by a random orthogonal Π, quantise
+ * every rotated coordinate independently with one fixed codebook computed once
+ * for the post-rotation marginal, and at decode time dequantise and apply Πᵀ.
+ * Π is the randomized Hadamard transform (section "Why rotation works";
+ * "TurboQuant and per-layer outlier-aware K" page, section "TurboQuant 2026":
+ * the FWHT):
+ *
+ *     Π = H·D/√d,  D = diag(s_0 .. s_{d-1}),  s_i = ±1,
+ *     H = Sylvester–Hadamard matrix of order d in natural order,
+ *     H_ij = (−1)^popcount(i & j).
+ *
+ * s_i = −1 exactly when bit 63 of SplitMix64 output number i is set, where
+ * output c of a generator seeded with `seed` is mix(seed + (c+1)·0x9E3779B97F4A7C15)
+ * (Steele, Lea & Flood 2014).  One D per call, shared by every vector.
+ *
+ * Common conventions
+ * ------------------
+ *  - Every data pointer is a DEVICE pointer owned by the caller, except where
+ *    an argument says "host".  The library allocates no device memory and
+ *    keeps no per-call state; it never synchronises the stream.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  Inputs and outputs must not alias.
+ *  - Vectors are rows of a dense row-major [n × d] array; a KV tensor
+ *    [tokens × heads × d] is n = tokens·heads rows, row t·heads + h.
+ *  - d is a power of two in [64, 512]; bits in 1..4; n ≥ 0 (n = 0 is a
+ *    no-op returning RRQ_OK).
+ *  - Array pointers must be 16-byte aligned (norm / scalar arrays: 4-byte).
+ *  - Element types: RRQ_F32 (float), RRQ_F16 (IEEE binary16), RRQ_BF16.
+ *  - Arguments are validated before any launch; an invalid call returns
+ *    RRQ_ERR_INVALID and touches no memory.  A failed launch returns
+ *    RRQ_ERR_CUDA.  Non-finite inputs give unspecified codes (no fault).
+ *  - fp32 / bf16 inputs need 1e-18 < ‖x‖₂ < 1e18 (the squared norm is
+ *    accumulated in fp32); fp16 inputs have no range restriction.
+ *
+ * Codebook (`codebook` arguments)
+ * -------------------------------
+ *  A HOST pointer to 2^bits strictly ascending finite floats, copied by value
+ *  at the call, or NULL for the Lloyd–Max codebook of N(0,1) ("Random-rotation
+ *  quantization" page, section "History", EDEN bullet: 1-bit ±√(2/π),
+ *  2-bit ±0.453, ±1.510).  Decision thresholds are the midpoints
+ *  τ_k = (c_k + c_{k+1})/2 (nearest-centroid cells; section "Three decoders,
+ *  one rotation", MSE decoder).  A codebook that is exactly symmetric
+ *  (c_k = −c_{L−1−k}) takes a faster path; any ascending codebook is accepted.
+ *
+ * Packed code format (RRQ_FORMAT_VERSION 1)
+ * -----------------------------------------
+ *  Per vector d·bits/8 bytes; coordinate i occupies bits [i·bits, (i+1)·bits)
+ *  of the byte string, least significant bit first (bits = 4: coordinate 2j
+ *  in the low nibble of byte j).  Code k means level c_k (code 0 = most
+ *  negative).  The per-vector scale is a separate fp32 array: ν = ‖x‖₂.
+ */
+#ifndef RRQ_H
+#define RRQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RRQ_FORMAT_VERSION 1
+
+/* status codes */
+#define RRQ_OK 0
+#define RRQ_ERR_INVALID 1     /* bad argument, detected before any launch       */
+#define RRQ_ERR_CUDA 2        /* a CUDA launch or runtime call failed           */
+#define RRQ_ERR_UNSUPPORTED 3 /* valid request this build does not implement    */
+
+/* element types */
+#define RRQ_F32 0
+#define RRQ_F16 1
+#define RRQ_BF16 2
+
+/* Packed-format version this library writes and reads. */
+int rrq_format_version(void);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* rrq_strerror(int status);
+
+/*
+ * rrq_codebook — the default codebook: ascending Lloyd–Max levels for N(0,1).
+ * "Random-rotation quantization" page, section "History", EDEN bullet.
+ * Computed on the host in double by Lloyd's iteration (centroid of each
+ * nearest-level cell under the normal density, thresholds at midpoints) and
+ * rounded to float; exactly symmetric.
+ *   bits    1..4
+ *   levels  HOST, float[2^bits], written in ascending order
+ * Returns RRQ_OK or RRQ_ERR_INVALID.  Thread-safe; no CUDA call.
+ */
+int rrq_codebook(int bits, float* levels);
+
+/*
+ * rrq_rotate — y = Πx (inverse = 0) or y = Πᵀx (inverse = 1), fp32 output.
+ * "Random-rotation quantization" page, scheme steps 1 and 3, and section
+ * "Why rotation works" (randomized Hadamard transform).
+ *   x      [n × d] of x_dtype
+ *   y      [n × d] float
+ * Errors: RRQ_ERR_INVALID (d, dtype, n, null or misaligned pointer),
+ * RRQ_ERR_CUDA.
+ */
+int rrq_rotate(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int inverse,
+               float* y, void* stream);
+
+/*
+ * rrq_encode — quantise n vectors.
+ * "Random-rotation quantization" page: scheme steps 1–2; "History", EDEN
+ * bullet (normalise to ≈N(0,1), Lloyd–Max codebook) and TurboQuant bullet
+ * (constant per-vector scale); "Three decoders, one rotation", MSE decoder.
+ * For each vector x:
+ *     ν = ‖x‖₂,  u = √d·Πx/ν  (u = 0 when ν = 0),
+ *     code_i = #{k : u_i > τ_k}   (a value on a threshold takes the lower code),
+ * codes are packed as described above and ν is stored as fp32.
+ *
+ * Optional QJL stage ("History", QJL and TurboQuant bullets: a 1-bit sign
+ * sketch of the residual makes inner products unbiased; "Bias vs
+ * unbiasedness"): when qjl_S is non-NULL, also
+ *     r = Πx − ŷ,  ŷ = (ν/√d)·c[code]  (the decoder's rotated-domain value),
+ *     qjl_bits bit i = [ (S·r)_i > 0 ],  qjl_rnorm = ‖r‖₂,
+ * with S the d×d matrix at qjl_S (bf16, row-major, see rrq_qjl_matrix).
+ * The product S·r runs on the tensor cores (tcgen05) with r split into three
+ * bf16 parts, so the signs are those of an fp32-accurate product.
+ *   x          [n × d] of x_dtype
+ *   codes      [n × d·bits/8] bytes (output)
+ *   norms      [n] float (output)
+ *   qjl_S      bf16 [d × d] or NULL (no QJL; then qjl_bits/qjl_rnorm ignored)
+ *   qjl_bits   [n × d/8] bytes (output, with qjl_S)
+ *   qjl_rnorm  [n] float (output, with qjl_S)
+ * Errors: RRQ_ERR_INVALID (bad d / bits / dtype / codebook, null or
+ * misaligned pointer), RRQ_ERR_UNSUPPORTED (QJL with d other than 128),
+ * RRQ_ERR_CUDA.
+ */
+int rrq_encode(const void* x, int x_dtype, int64_t n, int d, int bits, uint64_t seed,
+               const float* codebook, uint8_t* codes, float* norms,
+               const uint16_t* qjl_S, uint8_t* qjl_bits, float* qjl_rnorm, void* stream);
+
+/*
+ * rrq_decode — reconstruct n vectors from codes and norms.
+ * "Random-rotation quantization" page, scheme step 3 and "Three decoders,
+ * one rotation", MSE decoder:
+ *     ŷ_i = (ν/√d)·c[code_i],   x̂ = Πᵀŷ = (ν/d)·D·H·c[code],
+ * computed in fp32 and rounded to out_dtype (round to nearest even).
+ *   codes  [n × d·bits/8] bytes;  norms [n] float
+ *   out    [n × d] of out_dtype
+ * Errors: RRQ_ERR_INVALID, RRQ_ERR_CUDA.
+ */
+int rrq_decode(const uint8_t* codes, const float* norms, int64_t n, int d, int bits,
+               uint64_t seed, const float* codebook, void* out, int out_dtype, void* stream);
+
+/*
+ * rrq_qk_scores — decode-time attention scores against a quantised K cache,
+ * without decoding it.  "Random-rotation quantization" page, "Three decoders,
+ * one rotation", inner-product decoder: <q, x> is recovered from <Πq, code(Πx)>
+ * and a normalising scalar.  With q' = Πq (rotated once per call):
+ *     scores[h][t] = scale · (ν_{t,g}/√d) · Σ_i q'_{h,i} · c[code_{t,g,i}]
+ *                  = scale · <q_h, x̂_{t,g}>,    g = ⌊h·hkv/hq⌋ (GQA groups).
+ *   q       [hq × d] half (unrotated query heads)
+ *   codes   [T·hkv × d·bits/8] bytes, row t·hkv + g;  norms [T·hkv] float
+ *   scores  [hq × T] float (output)
+ * hq must be a multiple of hkv with hq/hkv in {1, 2, 4, 8}.
+ * Accuracy: products in fp16 pairs with fp32 partial sums; the error is far
+ * below 1e-3·‖q‖·‖x̂‖ for bits ≤ 4.
+ * Errors: RRQ_ERR_INVALID, RRQ_ERR_UNSUPPORTED (group size), RRQ_ERR_CUDA.
+ */
+int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norms, int64_t T,
+                  int hkv, int d, int bits, uint64_t seed, const float* codebook, float scale,
+                  float* scores, void* stream);
+
+/*
+ * rrq_q4_0_rot — "Attn-rot" (TurboQuant lite): rotate, then q4_0.
+ * "Attn-rot (TurboQuant lite) in llama.cpp" page: rotate K/V before an
+ * ordinary block format, q4_0 first of all.  With y = Πx (rotate = 1) or
+ * y = x (rotate = 0), per block of 32 consecutive coordinates:
+ *     m = the element of largest |y| (first on ties), Δ = m/−8 (fp32),
+ *     q_j = min(15, ⌊y_j/Δ + 8.5⌋)  (y_j·(1/Δ); 1/Δ := 0 when Δ = 0),
+ * stored as 18 bytes: fp16(Δ) little endian, then byte j = q_j | q_{j+16}<<4
+ * (the public llama.cpp q4_0 block, kept identical for interoperability).
+ *   x       [n × d] of x_dtype (d a multiple of 32 within [64, 512])
+ *   blocks  [n × d/32 × 18] bytes (output; 2-byte aligned suffices)
+ * Errors: RRQ_ERR_INVALID, RRQ_ERR_CUDA.
+ */
+int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate,
+                 void* blocks, void* stream);
+
+/*
+ * rrq_q4_0_rot_decode — inverse of rrq_q4_0_rot: ŷ_j = (q_j − 8)·fp16(Δ), then
+ * x̂ = Πᵀŷ when rotate = 1; fp32 arithmetic, rounded to out_dtype.
+ *   blocks  [n × d/32 × 18] bytes;  out [n × d] of out_dtype
+ */
+int rrq_q4_0_rot_decode(const void* blocks, int64_t n, int d, uint64_t seed, int rotate,
+                        void* out, int out_dtype, void* stream);
+
+/*
+ * rrq_qjl_matrix — the QJL projection S for a seed, on the HOST.
+ * Entry e = i·d + j: u1, u2 = top 53 bits of SplitMix64 outputs 2e, 2e+1 as
+ * uniforms in [0,1); z = sqrt(−2 ln(1 − u1))·cos(2π·u2) (Box–Muller);
+ * S[i][j] = bf16(z) (nearest even).  Written as bf16 bit patterns; the
+ * caller copies S to the device once and passes it to rrq_encode.
+ *   S  HOST, uint16_t[d × d]
+ * d a power of two in [64, 512].  Errors: RRQ_ERR_INVALID.
+ */
+int rrq_qjl_matrix(uint64_t seed, int d, uint16_t* S);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RRQ_H */

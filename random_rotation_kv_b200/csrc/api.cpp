@@ -1,0 +1,225 @@
+// api.cpp — the C ABI of librrq.so: argument validation, the default codebook,
+// per-call parameter blocks, and dispatch to the kernel launchers.
+//
+// Every entry point validates all arguments before touching the device and
+// returns RRQ_ERR_INVALID on the first violation; nothing is launched then.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "rrq.h"
+#include "rrq_params.h"
+
+namespace {
+
+constexpr double kInvSqrt2Pi = 0.39894228040143267794;
+
+bool d_ok(int d) { return d == 64 || d == 128 || d == 256 || d == 512; }
+bool bits_ok(int b) { return b >= 1 && b <= 4; }
+bool dtype_ok(int t) { return t == RRQ_F32 || t == RRQ_F16 || t == RRQ_BF16; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool arr_ok(const void* p, int64_t n, uintptr_t a) { return n == 0 || (p != nullptr && aligned(p, a)); }
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? RRQ_OK : RRQ_ERR_CUDA; }
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// ---------------------------------------------------------------- codebook
+// Lloyd–Max quantiser for N(0,1) ("Random-rotation quantization" page,
+// section "History", EDEN bullet).  Lloyd's alternation on the positive half
+// of a symmetric codebook: thresholds at midpoints of neighbouring levels
+// (0 between the two innermost), levels at the centroid of their cell,
+//   c = (φ(a) − φ(b)) / (Q(a) − Q(b)),  Q(x) = P(X > x) = erfc(x/√2)/2,
+// iterated until no level moves by more than 1e-15; the negative half is the
+// mirror image, so the codebook is exactly symmetric after rounding to float.
+double phi(double x) { return std::isinf(x) ? 0.0 : kInvSqrt2Pi * std::exp(-0.5 * x * x); }
+double upper_tail(double x) { return std::isinf(x) ? 0.0 : 0.5 * std::erfc(x / std::sqrt(2.0)); }
+
+struct DefaultCodebooks {
+  float levels[5][rrq::kMaxLevels];
+  DefaultCodebooks() {
+    std::memset(levels, 0, sizeof(levels));
+    for (int bits = 1; bits <= 4; ++bits) {
+      const int half = 1 << (bits - 1);
+      double c[8];
+      for (int j = 0; j < half; ++j) c[j] = 2.5 * (2 * j + 1) / (2.0 * half);
+      for (int it = 0; it < 200000; ++it) {
+        double moved = 0.0;
+        double nc[8];
+        for (int j = 0; j < half; ++j) {
+          const double a = j == 0 ? 0.0 : 0.5 * (c[j - 1] + c[j]);
+          const double b = j == half - 1 ? INFINITY : 0.5 * (c[j] + c[j + 1]);
+          nc[j] = (phi(a) - phi(b)) / (upper_tail(a) - upper_tail(b));
+          moved = std::fmax(moved, std::fabs(nc[j] - c[j]));
+        }
+        std::memcpy(c, nc, sizeof(double) * half);
+        if (moved < 1e-15) break;
+      }
+      const int L = 2 * half;
+      for (int j = 0; j < half; ++j) {
+        levels[bits][half + j] = static_cast<float>(c[j]);
+        levels[bits][half - 1 - j] = -static_cast<float>(c[j]);
+      }
+      (void)L;
+    }
+  }
+};
+
+const DefaultCodebooks& default_codebooks() {
+  static const DefaultCodebooks cb;  // built once, thread-safe initialisation
+  return cb;
+}
+
+// Fill the per-call parameter block; returns RRQ_ERR_INVALID for a bad codebook.
+int make_params(int bits, const float* codebook, uint64_t seed, int d, rrq::QuantParams* p) {
+  std::memset(p, 0, sizeof(*p));
+  const int L = 1 << bits;
+  const float* c = codebook ? codebook : default_codebooks().levels[bits];
+  for (int k = 0; k < L; ++k) {
+    if (!std::isfinite(c[k])) return RRQ_ERR_INVALID;
+    if (k > 0 && !(c[k] > c[k - 1])) return RRQ_ERR_INVALID;
+    p->levels[k] = c[k];
+  }
+  for (int k = 0; k + 1 < L; ++k)
+    p->thr[k] = static_cast<float>((static_cast<double>(c[k]) + static_cast<double>(c[k + 1])) * 0.5);
+  int sym = 1;
+  for (int k = 0; k < L; ++k) sym &= (c[k] == -c[L - 1 - k]) ? 1 : 0;
+  p->sym = sym;
+  p->bits = bits;
+  p->seed = seed;
+  p->inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  p->inv_d = 1.0f / static_cast<float>(d);
+  return RRQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rrq_format_version(void) { return RRQ_FORMAT_VERSION; }
+
+const char* rrq_strerror(int status) {
+  switch (status) {
+    case RRQ_OK: return "ok";
+    case RRQ_ERR_INVALID: return "invalid argument (checked before launch; nothing was run)";
+    case RRQ_ERR_CUDA: return "CUDA launch or runtime error";
+    case RRQ_ERR_UNSUPPORTED: return "valid request that this build does not implement";
+  }
+  return "unknown status";
+}
+
+int rrq_codebook(int bits, float* levels) {
+  if (!bits_ok(bits) || levels == nullptr) return RRQ_ERR_INVALID;
+  std::memcpy(levels, default_codebooks().levels[bits], sizeof(float) * (1u << bits));
+  return RRQ_OK;
+}
+
+int rrq_rotate(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int inverse, float* y,
+               void* stream) {
+  if (n < 0 || !d_ok(d) || !dtype_ok(x_dtype) || (inverse != 0 && inverse != 1))
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 16) || !arr_ok(y, n, 16)) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  return status_of(rrq::launch_rotate(x, x_dtype, n, d, seed, inverse, inv_sqrt_d, y,
+                                      as_stream(stream)));
+}
+
+int rrq_encode(const void* x, int x_dtype, int64_t n, int d, int bits, uint64_t seed,
+               const float* codebook, uint8_t* codes, float* norms, const uint16_t* qjl_S,
+               uint8_t* qjl_bits, float* qjl_rnorm, void* stream) {
+  if (n < 0 || !d_ok(d) || !bits_ok(bits) || !dtype_ok(x_dtype)) return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 16) || !arr_ok(codes, n, 16) || !arr_ok(norms, n, 4)) return RRQ_ERR_INVALID;
+  if (qjl_S != nullptr) {
+    if (!aligned(qjl_S, 16) || !arr_ok(qjl_bits, n, 16) || !arr_ok(qjl_rnorm, n, 4))
+      return RRQ_ERR_INVALID;
+  }
+  rrq::QuantParams p;
+  if (make_params(bits, codebook, seed, d, &p) != RRQ_OK) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  if (qjl_S != nullptr) {
+    if (d != 128) return RRQ_ERR_UNSUPPORTED;
+    return status_of(rrq::launch_encode_qjl(x, x_dtype, n, d, p, qjl_S, codes, norms, qjl_bits,
+                                            qjl_rnorm, as_stream(stream)));
+  }
+  return status_of(rrq::launch_encode(x, x_dtype, n, d, p, codes, norms, as_stream(stream)));
+}
+
+int rrq_decode(const uint8_t* codes, const float* norms, int64_t n, int d, int bits, uint64_t seed,
+               const float* codebook, void* out, int out_dtype, void* stream) {
+  if (n < 0 || !d_ok(d) || !bits_ok(bits) || !dtype_ok(out_dtype)) return RRQ_ERR_INVALID;
+  if (!arr_ok(codes, n, 16) || !arr_ok(norms, n, 4) || !arr_ok(out, n, 16)) return RRQ_ERR_INVALID;
+  rrq::QuantParams p;
+  if (make_params(bits, codebook, seed, d, &p) != RRQ_OK) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  return status_of(rrq::launch_decode(codes, norms, n, d, p, out, out_dtype, as_stream(stream)));
+}
+
+int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norms, int64_t T,
+                  int hkv, int d, int bits, uint64_t seed, const float* codebook, float scale,
+                  float* scores, void* stream) {
+  if (T < 0 || !d_ok(d) || !bits_ok(bits) || hq < 1 || hkv < 1 || hq % hkv != 0 ||
+      !std::isfinite(scale))
+    return RRQ_ERR_INVALID;
+  if (q == nullptr || !aligned(q, 16)) return RRQ_ERR_INVALID;
+  if (!arr_ok(codes, T, 16) || !arr_ok(norms, T, 4) || !arr_ok(scores, T, 16))
+    return RRQ_ERR_INVALID;
+  const int group = hq / hkv;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return RRQ_ERR_UNSUPPORTED;
+  rrq::QuantParams p;
+  if (make_params(bits, codebook, seed, d, &p) != RRQ_OK) return RRQ_ERR_INVALID;
+  if (T == 0) return RRQ_OK;
+  return status_of(rrq::launch_qk_scores(q, hq, codes, norms, T, hkv, d, p, scale, scores,
+                                         as_stream(stream)));
+}
+
+int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate,
+                 void* blocks, void* stream) {
+  if (n < 0 || !d_ok(d) || !dtype_ok(x_dtype) || (rotate != 0 && rotate != 1))
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 16) || !arr_ok(blocks, n, 2)) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  return status_of(rrq::launch_q4_0(x, x_dtype, n, d, seed, rotate, inv_sqrt_d, blocks,
+                                    as_stream(stream)));
+}
+
+int rrq_q4_0_rot_decode(const void* blocks, int64_t n, int d, uint64_t seed, int rotate, void* out,
+                        int out_dtype, void* stream) {
+  if (n < 0 || !d_ok(d) || !dtype_ok(out_dtype) || (rotate != 0 && rotate != 1))
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(blocks, n, 2) || !arr_ok(out, n, 16)) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  return status_of(rrq::launch_q4_0_decode(blocks, n, d, seed, rotate, inv_sqrt_d, out, out_dtype,
+                                           as_stream(stream)));
+}
+
+// QJL projection on the host: Box–Muller from two SplitMix64 outputs per entry,
+// rounded to bf16 (nearest even) directly from double.
+int rrq_qjl_matrix(uint64_t seed, int d, uint16_t* S) {
+  if (!d_ok(d) || S == nullptr) return RRQ_ERR_INVALID;
+  auto out = [seed](uint64_t c) {
+    uint64_t z = seed + (c + 1ull) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  };
+  const double two_pi = 6.283185307179586476925286766559;
+  const int64_t total = int64_t(d) * d;
+  for (int64_t e = 0; e < total; ++e) {
+    const double u1 = double(out(2 * uint64_t(e)) >> 11) * (1.0 / 9007199254740992.0);
+    const double u2 = double(out(2 * uint64_t(e) + 1) >> 11) * (1.0 / 9007199254740992.0);
+    const double z = std::sqrt(-2.0 * std::log(1.0 - u1)) * std::cos(two_pi * u2);
+    // round to bf16: keep 8 significant bits, ties to even (exact in double)
+    int ex = 0;
+    const double m = std::frexp(z, &ex);  // z = m·2^ex, 0.5 ≤ |m| < 1
+    const double r = std::nearbyint(std::ldexp(m, 8));
+    const float f = static_cast<float>(std::ldexp(r, ex - 8));  // exact in float
+    uint32_t bits;
+    std::memcpy(&bits, &f, 4);
+    S[e] = static_cast<uint16_t>(bits >> 16);
+  }
+  return RRQ_OK;
+}
+
+}  // extern "C"

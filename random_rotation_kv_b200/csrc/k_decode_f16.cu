@@ -1,0 +1,7 @@
+// Instantiates the f16-output decode kernels (split per element type to build in parallel).
+#include "quant_kernels.cuh"
+
+namespace rrq {
+template cudaError_t decode_typed<__half>(const uint8_t*, const float*, int64_t, int,
+                                        const QuantParams&, __half*, cudaStream_t);
+}  // namespace rrq

@@ -1,0 +1,120 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+validates arguments before any launch, and its host-side helpers (codebook,
+QJL matrix) agree with the oracle.  No kernel is launched here."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import codebook as ocb
+from oracle import rng as orng
+from random_rotation_kv_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rrq.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rrq_\w+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = B.lib()
+    declared = _declared_symbols()
+    assert len(declared) >= 10
+    for name in declared:
+        assert hasattr(lib, name), name
+    # the binding declares exactly the header's entry points
+    assert sorted(B.SIGNATURES) == declared
+
+
+def test_format_version_and_strerror():
+    assert B.rrq_format_version() == 1
+    for st in range(4):
+        assert len(B.strerror(st)) > 0
+    assert B.strerror(99) == "unknown status"
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_default_codebook_matches_oracle(bits):
+    c = B.rrq_codebook(bits).astype(np.float64)
+    o = ocb.lloyd_max(bits)
+    assert np.all(np.abs(c - o) <= 2 ** -23 * np.abs(o))  # float rounding of the same levels
+    assert np.array_equal(c, -c[::-1])
+
+
+def test_codebook_rejects_bad_bits():
+    lib = B.lib()
+    buf = (ctypes.c_float * 32)()
+    for bits in (0, 5, -1):
+        assert lib.rrq_codebook(bits, ctypes.cast(buf, ctypes.c_void_p)) == B.RRQ_ERR_INVALID
+    assert lib.rrq_codebook(2, None) == B.RRQ_ERR_INVALID
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_qjl_matrix_bit_exact_vs_oracle(d):
+    lib = B.lib()
+    host = np.zeros(d * d, dtype=np.uint16)
+    assert lib.rrq_qjl_matrix(4242, d, ctypes.c_void_p(host.ctypes.data)) == B.RRQ_OK
+    want = orng.bf16_bits(orng.qjl_gaussian(4242, d)).ravel()
+    assert np.array_equal(host, want)
+    assert lib.rrq_qjl_matrix(1, 100, ctypes.c_void_p(host.ctypes.data)) == B.RRQ_ERR_INVALID
+
+
+# Fake, never-dereferenced device addresses: every call below must be rejected
+# by validation before any CUDA call.
+P = ctypes.c_void_p(0x10000)
+P_MIS = ctypes.c_void_p(0x10002)
+
+
+def test_encode_validation_before_launch():
+    lib = B.lib()
+    enc = lib.rrq_encode
+    ok = dict(x=P, dt=B.RRQ_F16, n=8, d=128, bits=4)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return enc(a["x"], a["dt"], a["n"], a["d"], a["bits"], 42, kw.get("cb"), P, P,
+                   kw.get("S"), kw.get("qb"), kw.get("qn"), None)
+
+    assert call(d=100) == B.RRQ_ERR_INVALID
+    assert call(d=32) == B.RRQ_ERR_INVALID
+    assert call(d=1024) == B.RRQ_ERR_INVALID
+    assert call(bits=0) == B.RRQ_ERR_INVALID
+    assert call(bits=5) == B.RRQ_ERR_INVALID
+    assert call(dt=7) == B.RRQ_ERR_INVALID
+    assert call(n=-1) == B.RRQ_ERR_INVALID
+    assert call(x=ctypes.c_void_p(None)) == B.RRQ_ERR_INVALID
+    assert call(x=P_MIS) == B.RRQ_ERR_INVALID
+    bad_cb = (ctypes.c_float * 16)(*([0.0] * 16))  # not strictly ascending
+    assert call(cb=ctypes.cast(bad_cb, ctypes.c_void_p)) == B.RRQ_ERR_INVALID
+    nan_cb = (ctypes.c_float * 16)(*([float("nan")] + list(range(15))))
+    assert call(cb=ctypes.cast(nan_cb, ctypes.c_void_p)) == B.RRQ_ERR_INVALID
+    # QJL outputs must be given with S
+    assert call(S=P, qb=None, qn=P) == B.RRQ_ERR_INVALID
+    # n = 0 with valid arguments is a no-op that touches nothing
+    assert call(n=0, x=ctypes.c_void_p(None)) == B.RRQ_OK
+
+
+def test_other_entry_points_validate():
+    lib = B.lib()
+    assert lib.rrq_decode(P, P, 4, 100, 4, 0, None, P, B.RRQ_F16, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_decode(P, P, 4, 128, 4, 0, None, P, 9, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_decode(P, P_MIS, 4, 128, 4, 0, None, P, B.RRQ_F16, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_rotate(P, B.RRQ_F16, 4, 128, 0, 2, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_rotate(P_MIS, B.RRQ_F16, 4, 128, 0, 0, P, None) == B.RRQ_ERR_INVALID
+    # scores: hq not a multiple of hkv, unsupported group, non-finite scale
+    assert lib.rrq_qk_scores(P, 30, P, P, 16, 8, 128, 4, 0, None, 1.0, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_qk_scores(P, 48, P, P, 16, 3, 128, 4, 0, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
+    assert lib.rrq_qk_scores(P, 32, P, P, 16, 8, 128, 4, 0, None, float("inf"), P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_qk_scores(P, 32, P, P, 0, 8, 128, 4, 0, None, 1.0, P, None) == B.RRQ_OK
+    assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 96, 0, 1, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 128, 0, 3, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_q4_0_rot_decode(P, 4, 128, 0, 1, P, 5, None) == B.RRQ_ERR_INVALID
