@@ -280,7 +280,7 @@ def run_gpu(args):
     for _ in range(args.warmup):
         step()
     # keep the clocks in steady state before the timed region
-    t_end = time.time() + 0.5
+    t_end = time.time() + args.settle_s
     while time.time() < t_end:
         step()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -380,6 +380,8 @@ def main():
                     help="largest number of vectors per reference (oracle) step")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of CPU the whole reference run should take")
+    ap.add_argument("--settle-s", type=float, default=0.5,
+                    help="seconds of untimed steps before timing, so clocks reach steady state")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     args = ap.parse_args()

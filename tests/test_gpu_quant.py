@@ -101,7 +101,7 @@ def test_kv_workload_encode_decode_parity():
     enc, codes, norms = check_encode(x, "f16", 4, what="kv")
     out = B.rrq_decode(torch.from_numpy(enc.packed).to(DEV), torch.from_numpy(enc.norms).to(DEV),
                        128, 4, 42, out_dtype=torch.float16)
-    ref = orc.decode(enc.packed, enc.norms, 4, 128, 42, "f16")
+    ref = orc.decode(enc.packed, enc.norms, 4, 128, 42, out_dtype="f16")
     P.assert_reconstruction_close(host_f64(out), ref, np.linalg.norm(x.astype(np.float64), axis=1))
 
 
@@ -183,7 +183,7 @@ def test_full_size_kv_sampled_parity():
     gc = P.unpack_codes(codes[rows].cpu().numpy(), 4, 128)
     P.assert_codes_match(gc, enc.codes, enc.u, tau, "full kv")
     P.assert_norms_close(norms[rows].cpu().numpy(), enc.norm64, 128, "full kv")
-    ref = orc.decode(codes[rows].cpu().numpy(), norms[rows].cpu().numpy(), 4, 128, 42, "f16")
+    ref = orc.decode(codes[rows].cpu().numpy(), norms[rows].cpu().numpy(), 4, 128, 42, out_dtype="f16")
     P.assert_reconstruction_close(host_f64(out[rows]), ref, np.linalg.norm(xs, axis=1), "full kv")
     # whole-array property: round-trip NMSE of the rotated scheme ≤ the Gaussian D_4 (+5 %)
     xf = xd.float()
