@@ -38,8 +38,8 @@ from __future__ import annotations
 import numpy as np
 
 from .codebook import lloyd_max, thresholds
-from .hadamard import rotation_matrix
-from .rng import bf16_round
+from .hadamard import rotation_matrix, sylvester
+from .rng import bf16_round, rotation_signs
 
 
 def as_f64(x) -> np.ndarray:
@@ -114,11 +114,17 @@ def encode(x, bits: int, seed: int, levels=None) -> Encoded:
     n, d = x.shape
     c = default_levels(bits) if levels is None else np.asarray(levels, dtype=np.float64)
     tau = thresholds(c)
-    y = rotate(x, seed)
+    # √d·Πx = H·(D·x) exactly (Π = H·D/√d); with the ±1 matrix H the fp64
+    # products are exact and the sums of fp16/bf16 inputs are exact too, so a
+    # coordinate that lies exactly on a threshold (e.g. u = 0) is decided by the
+    # tie rule above rather than by rounding noise.
+    hd = sylvester(d) * rotation_signs(seed, d)[None, :]
+    y_sqrt_d = x @ hd.T
+    y = y_sqrt_d / np.sqrt(d)
     nu = np.sqrt(np.sum(x * x, axis=1))
     u = np.zeros_like(y)
     nzr = nu > 0
-    u[nzr] = np.sqrt(d) * y[nzr] / nu[nzr, None]
+    u[nzr] = y_sqrt_d[nzr] / nu[nzr, None]
     # code = number of thresholds strictly below u
     codes = np.searchsorted(tau, u.ravel(), side="left").reshape(n, d).astype(np.int64)
     return Encoded(codes, pack_codes(codes, bits), nu.astype(np.float32), nu, y, u)
