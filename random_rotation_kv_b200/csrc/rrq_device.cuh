@@ -116,94 +116,6 @@ template <int D, int G> struct Layout {
   __host__ __device__ static constexpr int chunk(int s, int h) { return s * G + h; }
 };
 
-// Load chunk-by-chunk (optionally XOR-ing the sign masks of D first) into v.
-// `row` points at the vector's first element; `valid` false yields zeros.
-template <typename T, int D, int G, bool FLIP>
-__device__ __forceinline__ void load_vector(const T* __restrict__ row, bool valid, int h,
-                                            const uint32_t* smask, float (&v)[D / G]) {
-  using L = Layout<D, G>;
-#pragma unroll
-  for (int s = 0; s < L::S; ++s) {
-    const int q = L::chunk(s, h);
-    if constexpr (Elem<T>::kBytes == 2) {
-      uint4 raw = valid ? ld_stream(row + q * 8) : make_uint4(0, 0, 0, 0);
-      if constexpr (FLIP) raw = xor4(raw, reinterpret_cast<const uint4*>(smask)[q]);
-      const float2 a = unpack2<T>(raw.x), b = unpack2<T>(raw.y);
-      const float2 c = unpack2<T>(raw.z), d = unpack2<T>(raw.w);
-      v[s * 8 + 0] = a.x; v[s * 8 + 1] = a.y; v[s * 8 + 2] = b.x; v[s * 8 + 3] = b.y;
-      v[s * 8 + 4] = c.x; v[s * 8 + 5] = c.y; v[s * 8 + 6] = d.x; v[s * 8 + 7] = d.y;
-    } else {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint4 raw = valid ? ld_stream(row + q * 8 + half * 4) : make_uint4(0, 0, 0, 0);
-        if constexpr (FLIP) raw = xor4(raw, reinterpret_cast<const uint4*>(smask)[q * 2 + half]);
-        v[s * 8 + half * 4 + 0] = __uint_as_float(raw.x);
-        v[s * 8 + half * 4 + 1] = __uint_as_float(raw.y);
-        v[s * 8 + half * 4 + 2] = __uint_as_float(raw.z);
-        v[s * 8 + half * 4 + 3] = __uint_as_float(raw.w);
-      }
-    }
-  }
-}
-
-// Store v (times `scale`) chunk-by-chunk as T, optionally XOR-ing sign masks.
-template <typename T, int D, int G, bool FLIP>
-__device__ __forceinline__ void store_vector(T* __restrict__ row, bool valid, int h,
-                                             const uint32_t* smask, const float (&v)[D / G],
-                                             float scale) {
-  using L = Layout<D, G>;
-#pragma unroll
-  for (int s = 0; s < L::S; ++s) {
-    const int q = L::chunk(s, h);
-    if constexpr (Elem<T>::kBytes == 2) {
-      uint4 w;
-      w.x = pack2<T>(v[s * 8 + 0] * scale, v[s * 8 + 1] * scale);
-      w.y = pack2<T>(v[s * 8 + 2] * scale, v[s * 8 + 3] * scale);
-      w.z = pack2<T>(v[s * 8 + 4] * scale, v[s * 8 + 5] * scale);
-      w.w = pack2<T>(v[s * 8 + 6] * scale, v[s * 8 + 7] * scale);
-      if constexpr (FLIP) w = xor4(w, reinterpret_cast<const uint4*>(smask)[q]);
-      if (valid) st_stream(row + q * 8, w);
-    } else {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint4 w;
-        w.x = __float_as_uint(v[s * 8 + half * 4 + 0] * scale);
-        w.y = __float_as_uint(v[s * 8 + half * 4 + 1] * scale);
-        w.z = __float_as_uint(v[s * 8 + half * 4 + 2] * scale);
-        w.w = __float_as_uint(v[s * 8 + half * 4 + 3] * scale);
-        if constexpr (FLIP) w = xor4(w, reinterpret_cast<const uint4*>(smask)[q * 2 + half]);
-        if (valid) st_stream(row + q * 8 + half * 4, w);
-      }
-    }
-  }
-}
-
-// Unnormalised Walsh–Hadamard transform of the group's D values.
-template <int D, int G>
-__device__ __forceinline__ void fwht(float (&v)[D / G], int h) {
-  constexpr int C = D / G;
-#pragma unroll
-  for (int m = 1; m < C; m <<= 1) {
-#pragma unroll
-    for (int r = 0; r < C; ++r) {
-      if ((r & m) == 0) {
-        const float a = v[r], b = v[r | m];
-        v[r] = a + b;
-        v[r | m] = a - b;
-      }
-    }
-  }
-#pragma unroll
-  for (int m = 1; m < G; m <<= 1) {
-    const float sgn = (h & m) ? -1.f : 1.f;
-#pragma unroll
-    for (int r = 0; r < C; ++r) {
-      const float t = __shfl_xor_sync(kFull, v[r], m);
-      v[r] = fmaf(v[r], sgn, t);  // lower lane: v + t; upper lane: t − v
-    }
-  }
-}
-
 // Sum over the G lanes of a group.
 template <int G>
 __device__ __forceinline__ float group_sum(float x) {
@@ -211,6 +123,84 @@ __device__ __forceinline__ float group_sum(float x) {
   for (int m = 1; m < G; m <<= 1) x += __shfl_xor_sync(kFull, x, m);
   return x;
 }
+
+// ---------------------------------------------------------- packed fp32 pairs
+// sm_100 issues two fp32 additions / multiplies per instruction (f32x2).  All
+// of these round each component once, exactly like the scalar operation.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a − b (b·(−1) is exact)
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// Unnormalised Walsh–Hadamard transform on packed pairs: w[k] holds values
+// r = 2k and 2k+1 of the lane (same coordinate map as fwht above).  Bit 0 of r
+// is a butterfly inside each pair; the other local bits pair whole registers.
+template <int D, int G>
+__device__ __forceinline__ void fwht2(float2 (&w)[D / G / 2], int h) {
+  constexpr int P = D / G / 2;
+#pragma unroll
+  for (int k = 0; k < P; ++k) {
+    const float a = w[k].x, b = w[k].y;
+    w[k] = make_float2(a + b, a - b);
+  }
+#pragma unroll
+  for (int mm = 1; mm < P; mm <<= 1) {
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      if ((k & mm) == 0) {
+        const float2 a = w[k], b = w[k | mm];
+        w[k] = add2(a, b);
+        w[k | mm] = sub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < G; m <<= 1) {
+    const float sg = (h & m) ? -1.f : 1.f;
+    const float2 sgn = make_float2(sg, sg);
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      const float2 t = make_float2(__shfl_xor_sync(kFull, w[k].x, m), __shfl_xor_sync(kFull, w[k].y, m));
+      w[k] = fma2(w[k], sgn, t);  // lower lane: w + t; upper lane: t − w
+    }
+  }
+}
+
+// One chunk (8 elements) of raw input words -> 4 packed pairs, sign masks applied.
+template <typename T, bool FLIP>
+__device__ __forceinline__ void chunk_to_pairs(const uint4* raw, const uint4* mask, float2* w) {
+  if constexpr (Elem<T>::kBytes == 2) {
+    uint4 r = raw[0];
+    if constexpr (FLIP) r = xor4(r, mask[0]);
+    w[0] = unpack2<T>(r.x); w[1] = unpack2<T>(r.y); w[2] = unpack2<T>(r.z); w[3] = unpack2<T>(r.w);
+  } else {
+    uint4 r0 = raw[0], r1 = raw[1];
+    if constexpr (FLIP) { r0 = xor4(r0, mask[0]); r1 = xor4(r1, mask[1]); }
+    w[0] = make_float2(__uint_as_float(r0.x), __uint_as_float(r0.y));
+    w[1] = make_float2(__uint_as_float(r0.z), __uint_as_float(r0.w));
+    w[2] = make_float2(__uint_as_float(r1.x), __uint_as_float(r1.y));
+    w[3] = make_float2(__uint_as_float(r1.z), __uint_as_float(r1.w));
+  }
+}
+
+// Raw 16-byte words of one vector owned by a lane (S chunks; 2 words per chunk for fp32).
+template <typename T, int D, int G> struct RawVec {
+  static constexpr int kWordsPerChunk = Elem<T>::kBytes == 2 ? 1 : 2;
+  static constexpr int N = Layout<D, G>::S * kWordsPerChunk;
+  uint4 r[N];
+  __device__ __forceinline__ void load(const T* __restrict__ row, bool valid, int h) {
+#pragma unroll
+    for (int s = 0; s < Layout<D, G>::S; ++s) {
+      const int q = Layout<D, G>::chunk(s, h);
+#pragma unroll
+      for (int c = 0; c < kWordsPerChunk; ++c)
+        r[s * kWordsPerChunk + c] =
+            valid ? ld_stream(row + q * 8 + c * 4) : make_uint4(0, 0, 0, 0);
+    }
+  }
+};
 
 // Lanes per vector for a head dimension: 2 up to d = 128, then 64 values a lane.
 template <int D> struct GroupOf { static constexpr int value = D <= 128 ? 2 : D / 64; };
