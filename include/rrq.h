@@ -29,7 +29,9 @@
  *    [tokens × heads × d] is n = tokens·heads rows, row t·heads + h.
  *  - d is a power of two in [64, 512]; bits in 1..4; n ≥ 0 (n = 0 is a
  *    no-op returning RRQ_OK).
- *  - Array pointers must be 16-byte aligned (norm / scalar arrays: 4-byte).
+ *  - Vector and code arrays must be 32-byte aligned (the kernels move whole
+ *    32-byte sectors); norm arrays 4-byte; other alignments are stated per
+ *    entry point.
  *  - Element types: RRQ_F32 (float), RRQ_F16 (IEEE binary16), RRQ_BF16.
  *  - Arguments are validated before any launch; an invalid call returns
  *    RRQ_ERR_INVALID and touches no memory.  A failed launch returns

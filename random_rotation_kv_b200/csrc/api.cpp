@@ -117,7 +117,7 @@ int rrq_rotate(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int 
                void* stream) {
   if (n < 0 || !d_ok(d) || !dtype_ok(x_dtype) || (inverse != 0 && inverse != 1))
     return RRQ_ERR_INVALID;
-  if (!arr_ok(x, n, 16) || !arr_ok(y, n, 16)) return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 32) || !arr_ok(y, n, 32)) return RRQ_ERR_INVALID;
   if (n == 0) return RRQ_OK;
   const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   return status_of(rrq::launch_rotate(x, x_dtype, n, d, seed, inverse, inv_sqrt_d, y,
@@ -128,7 +128,7 @@ int rrq_encode(const void* x, int x_dtype, int64_t n, int d, int bits, uint64_t 
                const float* codebook, uint8_t* codes, float* norms, const uint16_t* qjl_S,
                uint8_t* qjl_bits, float* qjl_rnorm, void* stream) {
   if (n < 0 || !d_ok(d) || !bits_ok(bits) || !dtype_ok(x_dtype)) return RRQ_ERR_INVALID;
-  if (!arr_ok(x, n, 16) || !arr_ok(codes, n, 16) || !arr_ok(norms, n, 4)) return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 32) || !arr_ok(codes, n, 32) || !arr_ok(norms, n, 4)) return RRQ_ERR_INVALID;
   if (qjl_S != nullptr) {
     if (!aligned(qjl_S, 16) || !arr_ok(qjl_bits, n, 16) || !arr_ok(qjl_rnorm, n, 4))
       return RRQ_ERR_INVALID;
@@ -147,7 +147,7 @@ int rrq_encode(const void* x, int x_dtype, int64_t n, int d, int bits, uint64_t 
 int rrq_decode(const uint8_t* codes, const float* norms, int64_t n, int d, int bits, uint64_t seed,
                const float* codebook, void* out, int out_dtype, void* stream) {
   if (n < 0 || !d_ok(d) || !bits_ok(bits) || !dtype_ok(out_dtype)) return RRQ_ERR_INVALID;
-  if (!arr_ok(codes, n, 16) || !arr_ok(norms, n, 4) || !arr_ok(out, n, 16)) return RRQ_ERR_INVALID;
+  if (!arr_ok(codes, n, 32) || !arr_ok(norms, n, 4) || !arr_ok(out, n, 32)) return RRQ_ERR_INVALID;
   rrq::QuantParams p;
   if (make_params(bits, codebook, seed, d, &p) != RRQ_OK) return RRQ_ERR_INVALID;
   if (n == 0) return RRQ_OK;

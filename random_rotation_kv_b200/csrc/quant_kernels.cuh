@@ -8,29 +8,38 @@
 //   "Three decoders, one rotation", MSE decoder: nearest of 2^b centroids.
 //
 // Per vector (one group of G lanes, see rrq_device.cuh):
-//   encode: 16 B loads (issued one grid-stride iteration ahead) → XOR rotation
-//           signs on the raw elements → ν² = Σx² (fp32 pairs, group shuffle
-//           sum) → unnormalised FWHT y' = H·D·x = √d·Πx → code_i = #{k : y'_i >
-//           ν·τ_k}, the same decision as u_i = y'_i/ν > τ_k with the scale
-//           folded into the thresholds once per vector → b-bit packing.
-//   decode: codes (loaded one iteration ahead) → levels c[code] → FWHT →
-//           × ν/d → round to the output type → XOR rotation signs → 16 B stores.
+//   encode: 32 B loads (issued one grid-stride iteration ahead) → XOR rotation
+//           signs on the raw elements → ν² = Σx² (packed fp32, group shuffle
+//           sum) → unnormalised FWHT y' = H·D·x = √d·Πx → code_i =
+//           #{k : y'_i > ν·τ_k}, the same decision as u_i = y'_i/ν > τ_k with
+//           the scale folded into the thresholds once per vector → packing.
+//   decode: codes (loaded one iteration ahead) → levels c[code] from shared
+//           memory → FWHT → × ν/d → round to the output type → XOR rotation
+//           signs → 32 B stores.
 //   rotate: y = Πx (signs, FWHT, × 1/√d) or y = Πᵀx (FWHT, × 1/√d, signs).
-// Instruction economy matters more than anything else here: the kernels are
-// issue-bound before they are HBM-bound, so arithmetic runs on packed fp32
-// pairs and the codebook search is a branch-free binary search.
+//
+// The kernels are issue-bound before they are HBM-bound, so the code search
+// is split between the two arithmetic pipes: half of the coordinates take a
+// branch-free compare/select binary search (integer/logic pipe), the other
+// half an equivalent search built from saturating FMAs (FMA pipe).
 #pragma once
 
 #include "rrq_device.cuh"
 
 namespace rrq {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kMinBlocks = 3;  // resident blocks per SM the register budget must allow
+
+// Values per lane: 64 for the encoder (the raw input of the next iteration is
+// held in registers too), 128 for the decoder (so a d ≤ 128 vector is one
+// lane and the transform needs no shuffles).
+template <int D> struct EncC { static constexpr int value = D < 64 ? D : 64; };
+template <int D> struct DecC { static constexpr int value = D < 128 ? D : 128; };
 
 // ------------------------------------------------------------- code search
 // Number of thresholds t[0..2^K−2] (ascending) strictly below a, by a K-level
-// branch-free binary search: the predicate of each level picks the next
-// threshold with a select, so a 16-level codebook costs 3 compares.
+// branch-free binary search: each level's predicate selects the next threshold.
 template <int K>
 __device__ __forceinline__ uint32_t count_below(float a, const float (&t)[(1 << K) > 1 ? (1 << K) - 1 : 1]) {
   if constexpr (K == 0) {
@@ -52,19 +61,18 @@ __device__ __forceinline__ uint32_t count_below(float a, const float (&t)[(1 << 
   }
 }
 
-// Code of one rotated value y' for an exactly symmetric codebook with L levels:
-// T[j] = ν·τ_{L/2+j} (the positive thresholds; τ_{L/2−1} = 0).
+// Code of one rotated value y' for an exactly symmetric codebook with 2^B
+// levels; T[j] = ν·τ_{L/2+j} (the positive thresholds; τ_{L/2−1} = 0):
 //   y' > 0:  code = L/2 + #{j : |y'| > T_j}
 //   y' ≤ 0:  code = L/2 − 1 − #{j : |y'| > T_j}
-// The second line takes ties |y'| = T_j to the upper code where the exact rule
-// (strict u > τ) takes the lower one; such values lie on a threshold, inside the
-// band where codes are allowed to differ.  y' = ±0 gives L/2 − 1 exactly.
+// The second line takes a tie |y'| = T_j to the upper code where the exact
+// rule (strict u > τ) takes the lower one; such a value lies on a threshold,
+// inside the band where codes may differ.  y' = ±0 gives L/2 − 1 exactly.
 // With m' = (L/2 − 1) − m = m ^ (L/2 − 1): code = pos ? m' ^ (L − 1) : m'.
 template <int B>
 __device__ __forceinline__ uint32_t code_sym(float y, const float (&T)[(1 << (B - 1)) > 1 ? (1 << (B - 1)) - 1 : 1]) {
   constexpr uint32_t L = 1u << B;
-  const uint32_t m = count_below<B - 1>(fabsf(y), T);
-  const uint32_t mm = m ^ (L / 2 - 1);
+  const uint32_t mm = count_below<B - 1>(fabsf(y), T) ^ (L / 2 - 1);
   return y > 0.f ? (mm ^ (L - 1)) : mm;
 }
 
@@ -77,96 +85,196 @@ __device__ __forceinline__ uint32_t code_generic(float y, const float (&tg)[L - 
   return m;
 }
 
-// Chunk q of a packed row: 8 codes of B bits = B bytes at byte offset q·B,
-// little endian (code e at bits [e·B, (e+1)·B)).
-template <int B>
-__device__ __forceinline__ void store_chunk(uint8_t* __restrict__ row, int q, uint32_t w) {
-  if constexpr (B == 4) {
-    reinterpret_cast<uint32_t*>(row)[q] = w;
-  } else if constexpr (B == 2) {
-    reinterpret_cast<uint16_t*>(row)[q] = uint16_t(w);
-  } else if constexpr (B == 1) {
-    row[q] = uint8_t(w);
-  } else {
-    row[3 * q + 0] = uint8_t(w);
-    row[3 * q + 1] = uint8_t(w >> 8);
-    row[3 * q + 2] = uint8_t(w >> 16);
-  }
-}
+// The same 4-bit symmetric search on the FMA pipe.  With big = 2^k chosen so
+// that ulp(T_0)·big = 1, every scaled threshold tb_j = T_j·big is an integer
+// and a·big is an integer whenever a ≥ T_0, so sat(a·big − tb) is exactly 1
+// when a > T and exactly 0 otherwise (a < T_0 gives a negative argument).
+// Thresholds of later levels are picked by arithmetic on the 0/1 results
+// (integer-valued, hence exact to within an ulp of the scaled threshold —
+// far inside the boundary band).
+struct Sym4 {
+  float t[7];   // T_j, for the compare/select path
+  float big;    // power of two, ulp(T_0)·big = 1
+  float tb[7];  // T_j·big
+  float d51, c1, c2, c3;
 
-template <int B>
-__device__ __forceinline__ uint32_t load_chunk(const uint8_t* __restrict__ row, int q) {
-  if constexpr (B == 4) {
-    return __ldcs(reinterpret_cast<const uint32_t*>(row) + q);
-  } else if constexpr (B == 2) {
-    return __ldcs(reinterpret_cast<const uint16_t*>(row) + q);
-  } else if constexpr (B == 1) {
-    return __ldcs(row + q);
-  } else {
-    return uint32_t(__ldcs(row + 3 * q)) | (uint32_t(__ldcs(row + 3 * q + 1)) << 8) |
-           (uint32_t(__ldcs(row + 3 * q + 2)) << 16);
-  }
-}
-
-// Packed pairs of one lane -> stored row (times `scale`), optional sign XOR.
-template <typename T, int D, int G, bool FLIP>
-__device__ __forceinline__ void store_pairs(T* __restrict__ row, bool valid, int h,
-                                            const uint32_t* smask, const float2 (&w)[D / G / 2],
-                                            float scale) {
-  using Lay = Layout<D, G>;
-  const float2 s2 = make_float2(scale, scale);
+  __device__ __forceinline__ void init(float ns, const QuantParams& p) {
 #pragma unroll
-  for (int s = 0; s < Lay::S; ++s) {
-    const int q = Lay::chunk(s, h);
-    const float2 a = mul2(w[s * 4 + 0], s2), b = mul2(w[s * 4 + 1], s2);
-    const float2 c = mul2(w[s * 4 + 2], s2), d = mul2(w[s * 4 + 3], s2);
-    if constexpr (Elem<T>::kBytes == 2) {
-      uint4 o = make_uint4(pack2<T>(a.x, a.y), pack2<T>(b.x, b.y), pack2<T>(c.x, c.y),
-                           pack2<T>(d.x, d.y));
-      if constexpr (FLIP) o = xor4(o, reinterpret_cast<const uint4*>(smask)[q]);
-      if (valid) st_stream(row + q * 8, o);
+    for (int j = 0; j < 7; ++j) t[j] = ns * p.thr[8 + j];
+    const uint32_t be = (__float_as_uint(t[0]) >> 23) & 0xffu;
+    const int bb = min(254, max(1, 277 - int(be)));
+    big = __uint_as_float(uint32_t(bb) << 23);
+#pragma unroll
+    for (int j = 0; j < 7; ++j) tb[j] = t[j] * big;
+    d51 = tb[5] - tb[1];
+    c1 = tb[2] - tb[0];
+    c2 = tb[4] - tb[0];
+    c3 = (tb[6] - tb[4]) - c1;
+  }
+
+  // code as an exact small integer in a float
+  __device__ __forceinline__ float code_fma(float y) const {
+    const float a = fabsf(y);
+    const float p2 = __saturatef(fmaf(a, big, -tb[3]));
+    const float tb1 = fmaf(p2, d51, tb[1]);
+    const float p1 = __saturatef(fmaf(a, big, -tb1));
+    const float tb0 = fmaf(p1, fmaf(p2, c3, c1), fmaf(p2, c2, tb[0]));
+    const float p0 = __saturatef(fmaf(a, big, -tb0));
+    const float m = fmaf(p2, 4.f, fmaf(p1, 2.f, p0));
+    const float ps = y > 0.f ? 1.f : 0.f;
+    return fmaf(ps, fmaf(m, 2.f, 1.f), 7.f - m);  // pos: 8 + m, else 7 − m
+  }
+};
+
+// 16 codes of one sector (4 bits each) -> two words; coordinates 0..3 and
+// 8..11 take the compare/select path, 4..7 and 12..15 the FMA path.
+__device__ __forceinline__ uint2 sector_codes4(const float2* w, const Sym4& k) {
+  uint32_t out[2];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const float2* v = w + 4 * half;
+    const uint32_t lo = code_sym<4>(v[0].x, k.t) | (code_sym<4>(v[0].y, k.t) << 4) |
+                        (code_sym<4>(v[1].x, k.t) << 8) | (code_sym<4>(v[1].y, k.t) << 12);
+    float f = k.code_fma(v[3].y);
+    f = fmaf(f, 16.f, k.code_fma(v[3].x));
+    f = fmaf(f, 16.f, k.code_fma(v[2].y));
+    f = fmaf(f, 16.f, k.code_fma(v[2].x));  // exact integer < 2^16
+    const uint32_t hi = __float_as_uint(f + 8388608.f);  // low 16 bits = f
+    out[half] = __byte_perm(lo, hi, 0x5410);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+// Number of positive thresholds of a symmetric codebook at B bits (≥ 1 slot).
+template <int B> constexpr int npos() { return (1 << (B - 1)) > 1 ? (1 << (B - 1)) - 1 : 1; }
+
+// 16 codes of one sector at B bits (B·16 bits, little endian) on the
+// compare/select path.
+template <int B, bool SYM>
+__device__ __forceinline__ uint64_t sector_codes(const float2* w, const float (&tp)[npos<B>()],
+                                                 const float (&tg)[(1 << B) - 1]) {
+  uint64_t acc = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t c0, c1;
+    if constexpr (SYM) {
+      c0 = code_sym<B>(w[j].x, tp);
+      c1 = code_sym<B>(w[j].y, tp);
     } else {
-      uint4 o0 = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
-                            __float_as_uint(b.y));
-      uint4 o1 = make_uint4(__float_as_uint(c.x), __float_as_uint(c.y), __float_as_uint(d.x),
-                            __float_as_uint(d.y));
-      if constexpr (FLIP) {
-        o0 = xor4(o0, reinterpret_cast<const uint4*>(smask)[q * 2]);
-        o1 = xor4(o1, reinterpret_cast<const uint4*>(smask)[q * 2 + 1]);
-      }
+      c0 = code_generic<1 << B>(w[j].x, tg);
+      c1 = code_generic<1 << B>(w[j].y, tg);
+    }
+    acc |= uint64_t(c0 | (c1 << B)) << (2 * j * B);
+  }
+  return acc;
+}
+
+// ------------------------------------------------------- packed code rows
+// A lane's code bits: for G = 1 the whole row (contiguous); otherwise only the
+// lane's sectors, each 2B bytes at byte offset q·2B of the row.
+template <int NB>  // NB = bytes
+__device__ __forceinline__ void store_bytes(uint8_t* __restrict__ p, const uint32_t* words) {
+  if constexpr (NB % 32 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 32; ++i) {
+      W8 v;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v.w[j] = words[i * 8 + j];
+      st256(p + 32 * i, v);
+    }
+  } else if constexpr (NB % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 16; ++i)
+      reinterpret_cast<uint4*>(p)[i] =
+          make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]);
+  } else {
+    static_assert(NB % 8 == 0, "code rows are a multiple of 8 bytes");
+#pragma unroll
+    for (int i = 0; i < NB / 8; ++i)
+      reinterpret_cast<uint2*>(p)[i] = make_uint2(words[2 * i], words[2 * i + 1]);
+  }
+}
+
+template <int NB>
+__device__ __forceinline__ void load_bytes(const uint8_t* __restrict__ p, bool valid, uint32_t* words) {
+  if constexpr (NB % 32 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 32; ++i) {
+      W8 v;
       if (valid) {
-        st_stream(row + q * 8, o0);
-        st_stream(row + q * 8 + 4, o1);
+        v = ld256(p + 32 * i);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v.w[j] = 0u;
       }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) words[i * 8 + j] = v.w[j];
+    }
+  } else if constexpr (NB % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 16; ++i) {
+      const uint4 v = valid ? __ldcs(reinterpret_cast<const uint4*>(p) + i) : make_uint4(0, 0, 0, 0);
+      words[4 * i] = v.x; words[4 * i + 1] = v.y; words[4 * i + 2] = v.z; words[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < NB / 8; ++i) {
+      const uint2 v = valid ? __ldcs(reinterpret_cast<const uint2*>(p) + i) : make_uint2(0, 0);
+      words[2 * i] = v.x; words[2 * i + 1] = v.y;
     }
   }
 }
 
-// Raw words -> packed pairs, with optional sign XOR.
-template <typename T, int D, int G, bool FLIP>
-__device__ __forceinline__ void raw_to_pairs(const RawVec<T, D, G>& raw, int h,
-                                             const uint32_t* smask, float2 (&w)[D / G / 2]) {
-  using Lay = Layout<D, G>;
-  constexpr int WPC = RawVec<T, D, G>::kWordsPerChunk;
-#pragma unroll
-  for (int s = 0; s < Lay::S; ++s) {
-    const int q = Lay::chunk(s, h);
-    chunk_to_pairs<T, FLIP>(&raw.r[s * WPC], reinterpret_cast<const uint4*>(smask) + q * WPC,
-                            &w[s * 4]);
+// Bits [pos, pos+nb) of a little-endian word array (nb ≤ 8; pos and nb are
+// constants after unrolling, so the array stays in registers).
+__device__ __forceinline__ uint32_t get_bits(const uint32_t* words, int pos, int nb) {
+  const int wi = pos >> 5, off = pos & 31;
+  uint32_t v = words[wi] >> off;
+  if (off + nb > 32) v |= words[wi + 1] << (32 - off);
+  return v & ((1u << nb) - 1u);
+}
+
+// One sector (2B bytes) of a row at byte offset q·2B (G > 1 layouts).
+template <int B>
+__device__ __forceinline__ void store_sector_codes(uint8_t* __restrict__ row, int q, uint64_t v) {
+  if constexpr (B == 4) {
+    reinterpret_cast<uint2*>(row)[q] = make_uint2(uint32_t(v), uint32_t(v >> 32));
+  } else if constexpr (B == 2) {
+    reinterpret_cast<uint32_t*>(row)[q] = uint32_t(v);
+  } else if constexpr (B == 1) {
+    reinterpret_cast<uint16_t*>(row)[q] = uint16_t(v);
+  } else {
+    uint16_t* p = reinterpret_cast<uint16_t*>(row) + 3 * q;
+    p[0] = uint16_t(v); p[1] = uint16_t(v >> 16); p[2] = uint16_t(v >> 32);
+  }
+}
+
+template <int B>
+__device__ __forceinline__ uint64_t load_sector_codes(const uint8_t* __restrict__ row, int q) {
+  if constexpr (B == 4) {
+    const uint2 v = __ldcs(reinterpret_cast<const uint2*>(row) + q);
+    return uint64_t(v.x) | (uint64_t(v.y) << 32);
+  } else if constexpr (B == 2) {
+    return __ldcs(reinterpret_cast<const uint32_t*>(row) + q);
+  } else if constexpr (B == 1) {
+    return __ldcs(reinterpret_cast<const uint16_t*>(row) + q);
+  } else {
+    const uint16_t* p = reinterpret_cast<const uint16_t*>(row) + 3 * q;
+    return uint64_t(__ldcs(p)) | (uint64_t(__ldcs(p + 1)) << 16) | (uint64_t(__ldcs(p + 2)) << 32);
   }
 }
 
 // ------------------------------------------------------------------ encode
 template <typename T, int D, int B, bool SYM>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
               float* __restrict__ norms, const QuantParams p) {
-  constexpr int G = GroupOf<D>::value;
-  using Lay = Layout<D, G>;
-  constexpr int P = Lay::C / 2, S = Lay::S, VPW = Lay::VPW;
+  constexpr int C = EncC<D>::value;
+  using Lay = Layout<D, C>;
+  constexpr int G = Lay::G, P = Lay::P, SEC = Lay::SEC, VPW = Lay::VPW;
   constexpr int L = 1 << B;
   constexpr int CB = D * B / 8;  // code bytes per vector
-  __shared__ __align__(16) uint32_t smask[SignMask<T>::template words<D>()];
+  __shared__ __align__(16) uint32_t smask[mask_words<T, D>()];
   build_sign_mask<T, D>(smask, p.seed);
   __syncthreads();
 
@@ -175,51 +283,66 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
   const int64_t stride = ((int64_t(gridDim.x) * blockDim.x) >> 5) * VPW;
 
   int64_t vec = gwarp * VPW + vsub;
-  RawVec<T, D, G> nxt;
+  RawVec<T, D, C> nxt;
   nxt.load(x + vec * D, vec < n, h);
   for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
     const bool valid = vec < n;
     float2 w[P];
-    raw_to_pairs<T, D, G, true>(nxt, h, smask, w);
+    raw_to_pairs<T, D, C, true>(nxt, h, smask, w);
     nxt.load(x + (vec + stride) * D, vec + stride < n, h);  // next iteration, in flight now
 
     float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < P; ++k) ss2 = fma2(w[k], w[k], ss2);
     const float nu = sqrtf(group_sum<G>(ss2.x + ss2.y));
-    fwht2<D, G>(w, h);
+    fwht2<D, C>(w, h);
     const float ns = nu > 0.f ? nu : 1.f;  // ν = 0: y' = 0, u = 0 against the plain thresholds
     uint8_t* crow = codes + vec * CB;
-    if constexpr (SYM) {
-      float tp[L / 2 > 1 ? L / 2 - 1 : 1];
+
+    uint64_t sec[SEC];
+    if constexpr (SYM && B == 4) {
+      Sym4 k4;
+      k4.init(ns, p);
 #pragma unroll
-      for (int j = 0; j < L / 2 - 1; ++j) tp[j] = ns * p.thr[L / 2 + j];
-#pragma unroll
-      for (int s = 0; s < S; ++s) {
-        uint32_t cw = 0;
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const float2 y = w[s * 4 + e / 2];
-          cw |= code_sym<B>(y.x, tp) << (e * B);
-          cw |= code_sym<B>(y.y, tp) << ((e + 1) * B);
-        }
-        if (valid) store_chunk<B>(crow, Lay::chunk(s, h), cw);
+      for (int s = 0; s < SEC; ++s) {
+        const uint2 v = sector_codes4(&w[s * 8], k4);
+        sec[s] = uint64_t(v.x) | (uint64_t(v.y) << 32);
       }
     } else {
-      float tg[L - 1];
+      float tp[npos<B>()] = {};
+      float tg[L - 1] = {};
+      if constexpr (SYM) {
 #pragma unroll
-      for (int k = 0; k < L - 1; ++k) tg[k] = ns * p.thr[k];
+        for (int j = 0; j < L / 2 - 1; ++j) tp[j] = ns * p.thr[L / 2 + j];
+      } else {
 #pragma unroll
-      for (int s = 0; s < S; ++s) {
-        uint32_t cw = 0;
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const float2 y = w[s * 4 + e / 2];
-          cw |= code_generic<L>(y.x, tg) << (e * B);
-          cw |= code_generic<L>(y.y, tg) << ((e + 1) * B);
-        }
-        if (valid) store_chunk<B>(crow, Lay::chunk(s, h), cw);
+        for (int k = 0; k < L - 1; ++k) tg[k] = ns * p.thr[k];
       }
+#pragma unroll
+      for (int s = 0; s < SEC; ++s) sec[s] = sector_codes<B, SYM>(&w[s * 8], tp, tg);
+    }
+    if constexpr (G == 1) {
+      uint32_t words[CB / 4];
+#pragma unroll
+      for (int i = 0; i < CB / 4; ++i) words[i] = 0u;
+#pragma unroll
+      for (int s = 0; s < SEC; ++s) {
+        // sector s at bit s·16B
+        if constexpr (B == 4) { words[2 * s] = uint32_t(sec[s]); words[2 * s + 1] = uint32_t(sec[s] >> 32); }
+        else if constexpr (B == 2) { words[s] = uint32_t(sec[s]); }
+        else if constexpr (B == 1) { words[s / 2] |= uint32_t(sec[s]) << (16 * (s & 1)); }
+        else {  // B == 3: 48 bits at bit 48·s
+          const int pos = 48 * s, wi = pos / 32, off = pos % 32;
+          words[wi] |= uint32_t(sec[s] << off);
+          words[wi + 1] |= uint32_t(sec[s] >> (32 - off));
+          if (off > 16) words[wi + 2] |= uint32_t(sec[s] >> (64 - off));
+        }
+      }
+      if (valid) store_bytes<CB>(crow, words);
+    } else {
+#pragma unroll
+      for (int s = 0; s < SEC; ++s)
+        if (valid) store_sector_codes<B>(crow, Lay::sector(s, h), sec[s]);
     }
     if (valid && h == 0) norms[vec] = nu;
   }
@@ -227,15 +350,16 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
 
 // ------------------------------------------------------------------ decode
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms, int64_t n,
               T* __restrict__ out, const QuantParams p) {
-  constexpr int G = GroupOf<D>::value;
-  using Lay = Layout<D, G>;
-  constexpr int P = Lay::C / 2, S = Lay::S, VPW = Lay::VPW;
+  constexpr int C = DecC<D>::value;
+  using Lay = Layout<D, C>;
+  constexpr int G = Lay::G, P = Lay::P, SEC = Lay::SEC, VPW = Lay::VPW;
   constexpr int L = 1 << B;
   constexpr int CB = D * B / 8;
-  __shared__ __align__(16) uint32_t smask[SignMask<T>::template words<D>()];
+  constexpr int NW = (G == 1) ? CB / 4 : SEC * 2;  // code words held per lane
+  __shared__ __align__(16) uint32_t smask[mask_words<T, D>()];
   __shared__ float slev[L];
   build_sign_mask<T, D>(smask, p.seed);
   if (threadIdx.x < L) slev[threadIdx.x] = p.levels[threadIdx.x];
@@ -246,48 +370,63 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   const int64_t stride = ((int64_t(gridDim.x) * blockDim.x) >> 5) * VPW;
 
   int64_t vec = gwarp * VPW + vsub;
-  uint32_t cw_next[S];
+  uint32_t nw[NW];
   float nu_next = 0.f;
   auto fetch = [&](int64_t v) {
     const bool ok = v < n;
     const uint8_t* crow = codes + v * CB;
+    if constexpr (G == 1) {
+      load_bytes<CB>(crow, ok, nw);
+    } else {
 #pragma unroll
-    for (int s = 0; s < S; ++s) cw_next[s] = ok ? load_chunk<B>(crow, Lay::chunk(s, h)) : 0u;
+      for (int s = 0; s < SEC; ++s) {
+        const uint64_t c = ok ? load_sector_codes<B>(crow, Lay::sector(s, h)) : 0ull;
+        nw[2 * s] = uint32_t(c);
+        nw[2 * s + 1] = uint32_t(c >> 32);
+      }
+    }
     nu_next = ok ? __ldcs(norms + v) : 0.f;
   };
   fetch(vec);
   for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
     const bool valid = vec < n;
-    uint32_t cw[S];
+    uint32_t cw[NW];
 #pragma unroll
-    for (int s = 0; s < S; ++s) cw[s] = cw_next[s];
+    for (int i = 0; i < NW; ++i) cw[i] = nw[i];
     const float nu = nu_next;
     fetch(vec + stride);  // next iteration, in flight now
 
     float2 w[P];
 #pragma unroll
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SEC; ++s) {
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        w[s * 4 + e / 2] = make_float2(slev[(cw[s] >> (e * B)) & (L - 1)],
-                                       slev[(cw[s] >> ((e + 1) * B)) & (L - 1)]);
+      for (int e = 0; e < 16; e += 2) {
+        uint32_t c0, c1;
+        if constexpr (G == 1) {
+          c0 = get_bits(cw, (s * 16 + e) * B, B);
+          c1 = get_bits(cw, (s * 16 + e + 1) * B, B);
+        } else {
+          c0 = get_bits(cw + 2 * s, e * B, B);
+          c1 = get_bits(cw + 2 * s, (e + 1) * B, B);
+        }
+        w[s * 8 + e / 2] = make_float2(slev[c0], slev[c1]);
       }
     }
-    fwht2<D, G>(w, h);
-    store_pairs<T, D, G, true>(out + vec * D, valid, h, smask, w, nu * p.inv_d);
+    fwht2<D, C>(w, h);
+    store_pairs<T, D, C, true>(out + vec * D, valid, h, smask, w, nu * p.inv_d);
   }
 }
 
 // ------------------------------------------------------------------ rotate
 template <typename T, int D, bool INV>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 rotate_kernel(const T* __restrict__ x, int64_t n, float* __restrict__ y, uint64_t seed,
               float inv_sqrt_d) {
-  constexpr int G = GroupOf<D>::value;
-  using Lay = Layout<D, G>;
-  constexpr int P = Lay::C / 2, VPW = Lay::VPW;
-  __shared__ __align__(16) uint32_t smask_in[SignMask<T>::template words<D>()];
-  __shared__ __align__(16) uint32_t smask_out[SignMask<float>::template words<D>()];
+  constexpr int C = EncC<D>::value;
+  using Lay = Layout<D, C>;
+  constexpr int G = Lay::G, P = Lay::P, VPW = Lay::VPW;
+  __shared__ __align__(16) uint32_t smask_in[mask_words<T, D>()];
+  __shared__ __align__(16) uint32_t smask_out[mask_words<float, D>()];
   if constexpr (!INV) build_sign_mask<T, D>(smask_in, seed);
   else build_sign_mask<float, D>(smask_out, seed);
   __syncthreads();
@@ -296,25 +435,27 @@ rotate_kernel(const T* __restrict__ x, int64_t n, float* __restrict__ y, uint64_
   const int64_t gwarp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t stride = ((int64_t(gridDim.x) * blockDim.x) >> 5) * VPW;
   int64_t vec = gwarp * VPW + vsub;
-  RawVec<T, D, G> nxt;
+  RawVec<T, D, C> nxt;
   nxt.load(x + vec * D, vec < n, h);
   for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
     const bool valid = vec < n;
     float2 w[P];
-    raw_to_pairs<T, D, G, !INV>(nxt, h, smask_in, w);
+    raw_to_pairs<T, D, C, !INV>(nxt, h, smask_in, w);
     nxt.load(x + (vec + stride) * D, vec + stride < n, h);
-    fwht2<D, G>(w, h);
-    store_pairs<float, D, G, INV>(y + vec * D, valid, h, smask_out, w, inv_sqrt_d);
+    fwht2<D, C>(w, h);
+    store_pairs<float, D, C, INV>(y + vec * D, valid, h, smask_out, w, inv_sqrt_d);
   }
 }
 
 // ---------------------------------------------------------------- launchers
-constexpr int vectors_per_block(int d) { return (kThreads / 32) * (32 / (d <= 128 ? 2 : d / 64)); }
+template <int C_>
+constexpr int vectors_per_block(int d) { return (kThreads / 32) * (32 / (d / (d < C_ ? d : C_))); }
 
 template <typename T, int D, int B>
 cudaError_t encode_db(const T* x, int64_t n, const QuantParams& p, uint8_t* codes, float* norms,
                       cudaStream_t stream) {
-  const int64_t work = (n + vectors_per_block(D) - 1) / vectors_per_block(D);
+  constexpr int vpb = vectors_per_block<EncC<D>::value>(D);
+  const int64_t work = (n + vpb - 1) / vpb;
   if (p.sym) {
     auto k = encode_kernel<T, D, B, true>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
@@ -354,7 +495,8 @@ cudaError_t encode_typed(const T* x, int64_t n, int d, const QuantParams& p, uin
 template <typename T, int D, int B>
 cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const QuantParams& p,
                       T* out, cudaStream_t stream) {
-  const int64_t work = (n + vectors_per_block(D) - 1) / vectors_per_block(D);
+  constexpr int vpb = vectors_per_block<DecC<D>::value>(D);
+  const int64_t work = (n + vpb - 1) / vpb;
   auto k = decode_kernel<T, D, B>;
   const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
   k<<<grid, kThreads, 0, stream>>>(codes, norms, n, out, p);
@@ -388,7 +530,8 @@ cudaError_t decode_typed(const uint8_t* codes, const float* norms, int64_t n, in
 template <typename T, int D>
 cudaError_t rotate_d(const T* x, int64_t n, uint64_t seed, int inverse, float inv_sqrt_d, float* y,
                      cudaStream_t stream) {
-  const int64_t work = (n + vectors_per_block(D) - 1) / vectors_per_block(D);
+  constexpr int vpb = vectors_per_block<EncC<D>::value>(D);
+  const int64_t work = (n + vpb - 1) / vpb;
   if (inverse) {
     auto k = rotate_kernel<T, D, true>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);

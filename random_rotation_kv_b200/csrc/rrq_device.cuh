@@ -1,17 +1,20 @@
 // rrq_device.cuh — device building blocks shared by the rrq kernels (sm_100a).
 //
-// Lane layout.  A vector of D coordinates is owned by a group of G consecutive
-// lanes of a warp (32/G vectors per warp).  The vector is cut into chunks of 8
-// consecutive coordinates (16 bytes of fp16/bf16); chunk q lives in lane
-// h = q mod G, slot s = q / G, so one 16-byte load instruction of the warp
-// reads G·16 contiguous bytes of every vector it touches (fully used
-// sectors).  Lane h therefore holds C = D/G values v[r], r = s·8 + e, for
-// coordinate i = (s·G + h)·8 + e.  In the bits of i: bits 0..2 are e (local),
-// bits 3..3+log2(G)−1 are the lane bits h, the rest are s (local).
+// Lane layout.  A vector of D coordinates is owned by a group of G = D/C
+// consecutive lanes of a warp, each lane holding C coordinates (C ≤ 128, a
+// per-kernel choice; 32/G vectors per warp).  The vector is cut into sectors
+// of 16 consecutive coordinates (32 bytes of fp16/bf16, one DRAM sector);
+// sector q lives in lane h = q mod G, slot s = q / G.  Each lane moves whole
+// sectors with 256-bit loads and stores (sm_100 `ld/st.global.v8.b32`), and
+// for G > 1 the G lanes of a vector read G adjacent sectors in one
+// instruction.  Lane h holds values v[r], r = s·16 + e, of coordinate
+// i = (s·G + h)·16 + e: bits 0..3 of i are e (local), bits 4..4+log2(G)−1 are
+// the lane bits h, the remaining bits are s (local).
 //
 // Walsh–Hadamard transform.  The unnormalised transform y = H·v with
 // H_ij = (−1)^popcount(i&j) factors into one butterfly (a, b) → (a+b, a−b)
-// per bit of i, in any order.  Local bits are butterflies between registers;
+// per bit of i, in any order.  Local bits are butterflies between registers
+// (on packed fp32 pairs: sm_100 issues two fp32 additions per instruction);
 // lane bits are one __shfl_xor_sync per value, the lower lane adding and the
 // upper lane subtracting.  ("Random-rotation quantization" page, section "Why
 // rotation works": the randomized Hadamard transform, O(d log d).)
@@ -44,46 +47,48 @@ __host__ __device__ __forceinline__ uint32_t sign_bit(uint64_t seed, int i) {
 
 // ------------------------------------------------------------ element types
 template <typename T> struct Elem;
-template <> struct Elem<float> {
-  static constexpr int kDtype = RRQ_F32;
-  static constexpr int kBytes = 4;
-};
-template <> struct Elem<__half> {
-  static constexpr int kDtype = RRQ_F16;
-  static constexpr int kBytes = 2;
-};
-template <> struct Elem<__nv_bfloat16> {
-  static constexpr int kDtype = RRQ_BF16;
-  static constexpr int kBytes = 2;
-};
+template <> struct Elem<float> { static constexpr int kBytes = 4; };
+template <> struct Elem<__half> { static constexpr int kBytes = 2; };
+template <> struct Elem<__nv_bfloat16> { static constexpr int kBytes = 2; };
 
-// Sign-flip masks in shared memory, one 32-bit XOR word per pair of 16-bit
-// elements (sign bits 15 and 31) or per fp32 element (bit 31).
-template <typename T> struct SignMask {
-  static constexpr int kWordsPerChunk = (Elem<T>::kBytes == 2) ? 4 : 8;
-  template <int D> static constexpr int words() { return D / 8 * kWordsPerChunk; }
-};
+// 32-bit words per 16-coordinate sector of T.
+template <typename T> constexpr int sector_words() { return 16 * Elem<T>::kBytes / 4; }
+
+// Sign-flip masks in shared memory: one XOR word per element word of a sector
+// (sign bits 15 and 31 for a pair of 16-bit elements, bit 31 for fp32).
+template <typename T, int D> constexpr int mask_words() { return D / 16 * sector_words<T>(); }
 
 template <typename T, int D>
 __device__ __forceinline__ void build_sign_mask(uint32_t* smask, uint64_t seed) {
   if constexpr (Elem<T>::kBytes == 2) {
-    for (int k = threadIdx.x; k < D / 2; k += blockDim.x) {
+    for (int k = threadIdx.x; k < D / 2; k += blockDim.x)
       smask[k] = (sign_bit(seed, 2 * k) << 15) | (sign_bit(seed, 2 * k + 1) << 31);
-    }
   } else {
     for (int i = threadIdx.x; i < D; i += blockDim.x) smask[i] = sign_bit(seed, i) << 31;
   }
 }
 
-// ----------------------------------------------------- 16-byte memory helpers
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  return __ldcs(reinterpret_cast<const uint4*>(p));
+// -------------------------------------------------------- 256-bit accesses
+struct alignas(32) W8 {
+  uint32_t w[8];
+};
+
+// Streaming 32-byte load (read once: no L1 allocation).
+__device__ __forceinline__ W8 ld256(const void* p) {
+  W8 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
+                 "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
+               : "l"(p));
+  return r;
 }
-__device__ __forceinline__ void st_stream(void* p, uint4 v) {
-  __stcs(reinterpret_cast<uint4*>(p), v);
-}
-__device__ __forceinline__ uint4 xor4(uint4 a, uint4 b) {
-  return make_uint4(a.x ^ b.x, a.y ^ b.y, a.z ^ b.z, a.w ^ b.w);
+
+// Streaming 32-byte store (evict-first).
+__device__ __forceinline__ void st256(void* p, const W8& v) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+               "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+               "r"(v.w[7])
+               : "memory");
 }
 
 // 2 packed 16-bit elements -> 2 floats (exact)
@@ -97,49 +102,130 @@ template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t w)
 }
 
 // 2 floats -> 2 packed 16-bit elements, round to nearest even
-template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
-template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
+template <typename T> __device__ __forceinline__ uint32_t pack2(float2 v);
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float2 v) {
+  __half2 h = __float22half2_rn(v);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float2 v) {
+  __nv_bfloat162 h = __float22bfloat162_rn(v);
   return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// ---------------------------------------------------------------- lane layout
-template <int D, int G> struct Layout {
-  static_assert(D % (8 * G) == 0, "D must be a multiple of 8*G");
-  static constexpr int C = D / G;     // values per lane
-  static constexpr int S = C / 8;     // chunks per lane
-  static constexpr int VPW = 32 / G;  // vectors per warp
-  __host__ __device__ static constexpr int chunk(int s, int h) { return s * G + h; }
-};
-
-// Sum over the G lanes of a group.
-template <int G>
-__device__ __forceinline__ float group_sum(float x) {
-#pragma unroll
-  for (int m = 1; m < G; m <<= 1) x += __shfl_xor_sync(kFull, x, m);
-  return x;
 }
 
 // ---------------------------------------------------------- packed fp32 pairs
-// sm_100 issues two fp32 additions / multiplies per instruction (f32x2).  All
-// of these round each component once, exactly like the scalar operation.
+// Each component is rounded once, exactly like the scalar operation.
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a − b (b·(−1) is exact)
+  const unsigned long long ua = *reinterpret_cast<const unsigned long long*>(&a);
+  const unsigned long long ub = *reinterpret_cast<const unsigned long long*>(&b);
+  unsigned long long ur;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(ur) : "l"(ua), "l"(ub));
+  return *reinterpret_cast<float2*>(&ur);
 }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// ---------------------------------------------------------------- lane layout
+template <int D, int C> struct Layout {
+  static_assert(C % 16 == 0 && D % C == 0, "C must be a multiple of 16 dividing D");
+  static constexpr int G = D / C;       // lanes per vector
+  static constexpr int SEC = C / 16;    // sectors per lane
+  static constexpr int P = C / 2;       // packed pairs per lane
+  static constexpr int VPW = 32 / G;    // vectors per warp
+  __host__ __device__ static constexpr int sector(int s, int h) { return s * G + h; }
+};
+
+// One sector of raw words -> 8 packed pairs, with optional sign XOR from smem.
+template <typename T, bool FLIP>
+__device__ __forceinline__ void sector_to_pairs(const uint32_t* raw, const uint32_t* mask,
+                                                float2* w) {
+  if constexpr (Elem<T>::kBytes == 2) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = unpack2<T>(FLIP ? raw[j] ^ mask[j] : raw[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      w[j] = make_float2(__uint_as_float(FLIP ? raw[2 * j] ^ mask[2 * j] : raw[2 * j]),
+                         __uint_as_float(FLIP ? raw[2 * j + 1] ^ mask[2 * j + 1] : raw[2 * j + 1]));
+  }
+}
+
+// The lane's raw input words of one vector.
+template <typename T, int D, int C> struct RawVec {
+  static constexpr int SW = sector_words<T>();  // 8 (16-bit) or 16 (fp32)
+  static constexpr int N = Layout<D, C>::SEC * SW;
+  uint32_t r[N];
+  __device__ __forceinline__ void load(const T* __restrict__ row, bool valid, int h) {
+#pragma unroll
+    for (int s = 0; s < Layout<D, C>::SEC; ++s) {
+      const T* src = row + Layout<D, C>::sector(s, h) * 16;
+#pragma unroll
+      for (int c = 0; c < SW / 8; ++c) {
+        W8 v;
+        if (valid) {
+          v = ld256(src + c * (32 / Elem<T>::kBytes));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v.w[j] = 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[s * SW + c * 8 + j] = v.w[j];
+      }
+    }
+  }
+};
+
+template <typename T, int D, int C, bool FLIP>
+__device__ __forceinline__ void raw_to_pairs(const RawVec<T, D, C>& raw, int h,
+                                             const uint32_t* smask, float2 (&w)[C / 2]) {
+  using Lay = Layout<D, C>;
+  constexpr int SW = sector_words<T>();
+#pragma unroll
+  for (int s = 0; s < Lay::SEC; ++s)
+    sector_to_pairs<T, FLIP>(&raw.r[s * SW], smask + Lay::sector(s, h) * SW, &w[s * 8]);
+}
+
+// Packed pairs of one lane -> stored row (times `scale`), optional sign XOR.
+template <typename T, int D, int C, bool FLIP>
+__device__ __forceinline__ void store_pairs(T* __restrict__ row, bool valid, int h,
+                                            const uint32_t* smask, const float2 (&w)[C / 2],
+                                            float scale) {
+  using Lay = Layout<D, C>;
+  constexpr int SW = sector_words<T>();
+  const float2 s2 = make_float2(scale, scale);
+#pragma unroll
+  for (int s = 0; s < Lay::SEC; ++s) {
+    const int q = Lay::sector(s, h);
+    const uint32_t* m = smask + q * SW;
+#pragma unroll
+    for (int c = 0; c < SW / 8; ++c) {
+      W8 o;
+      if constexpr (Elem<T>::kBytes == 2) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t p = pack2<T>(mul2(w[s * 8 + j], s2));
+          o.w[j] = FLIP ? p ^ m[j] : p;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 v = mul2(w[s * 8 + c * 4 + j], s2);
+          o.w[2 * j] = FLIP ? __float_as_uint(v.x) ^ m[c * 8 + 2 * j] : __float_as_uint(v.x);
+          o.w[2 * j + 1] =
+              FLIP ? __float_as_uint(v.y) ^ m[c * 8 + 2 * j + 1] : __float_as_uint(v.y);
+        }
+      }
+      if (valid) st256(row + q * 16 + c * (32 / Elem<T>::kBytes), o);
+    }
+  }
+}
+
 // Unnormalised Walsh–Hadamard transform on packed pairs: w[k] holds values
-// r = 2k and 2k+1 of the lane (same coordinate map as fwht above).  Bit 0 of r
-// is a butterfly inside each pair; the other local bits pair whole registers.
-template <int D, int G>
-__device__ __forceinline__ void fwht2(float2 (&w)[D / G / 2], int h) {
-  constexpr int P = D / G / 2;
+// r = 2k and 2k+1 of the lane.  Bit 0 of r is a butterfly inside each pair;
+// the other local bits pair whole registers; lane bits use shuffles.
+template <int D, int C>
+__device__ __forceinline__ void fwht2(float2 (&w)[C / 2], int h) {
+  constexpr int P = C / 2, G = D / C;
 #pragma unroll
   for (int k = 0; k < P; ++k) {
     const float a = w[k].x, b = w[k].y;
@@ -162,47 +248,19 @@ __device__ __forceinline__ void fwht2(float2 (&w)[D / G / 2], int h) {
     const float2 sgn = make_float2(sg, sg);
 #pragma unroll
     for (int k = 0; k < P; ++k) {
-      const float2 t = make_float2(__shfl_xor_sync(kFull, w[k].x, m), __shfl_xor_sync(kFull, w[k].y, m));
+      const float2 t =
+          make_float2(__shfl_xor_sync(kFull, w[k].x, m), __shfl_xor_sync(kFull, w[k].y, m));
       w[k] = fma2(w[k], sgn, t);  // lower lane: w + t; upper lane: t − w
     }
   }
 }
 
-// One chunk (8 elements) of raw input words -> 4 packed pairs, sign masks applied.
-template <typename T, bool FLIP>
-__device__ __forceinline__ void chunk_to_pairs(const uint4* raw, const uint4* mask, float2* w) {
-  if constexpr (Elem<T>::kBytes == 2) {
-    uint4 r = raw[0];
-    if constexpr (FLIP) r = xor4(r, mask[0]);
-    w[0] = unpack2<T>(r.x); w[1] = unpack2<T>(r.y); w[2] = unpack2<T>(r.z); w[3] = unpack2<T>(r.w);
-  } else {
-    uint4 r0 = raw[0], r1 = raw[1];
-    if constexpr (FLIP) { r0 = xor4(r0, mask[0]); r1 = xor4(r1, mask[1]); }
-    w[0] = make_float2(__uint_as_float(r0.x), __uint_as_float(r0.y));
-    w[1] = make_float2(__uint_as_float(r0.z), __uint_as_float(r0.w));
-    w[2] = make_float2(__uint_as_float(r1.x), __uint_as_float(r1.y));
-    w[3] = make_float2(__uint_as_float(r1.z), __uint_as_float(r1.w));
-  }
+// Sum over the G lanes of a group.
+template <int G>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int m = 1; m < G; m <<= 1) x += __shfl_xor_sync(kFull, x, m);
+  return x;
 }
-
-// Raw 16-byte words of one vector owned by a lane (S chunks; 2 words per chunk for fp32).
-template <typename T, int D, int G> struct RawVec {
-  static constexpr int kWordsPerChunk = Elem<T>::kBytes == 2 ? 1 : 2;
-  static constexpr int N = Layout<D, G>::S * kWordsPerChunk;
-  uint4 r[N];
-  __device__ __forceinline__ void load(const T* __restrict__ row, bool valid, int h) {
-#pragma unroll
-    for (int s = 0; s < Layout<D, G>::S; ++s) {
-      const int q = Layout<D, G>::chunk(s, h);
-#pragma unroll
-      for (int c = 0; c < kWordsPerChunk; ++c)
-        r[s * kWordsPerChunk + c] =
-            valid ? ld_stream(row + q * 8 + c * 4) : make_uint4(0, 0, 0, 0);
-    }
-  }
-};
-
-// Lanes per vector for a head dimension: 2 up to d = 128, then 64 values a lane.
-template <int D> struct GroupOf { static constexpr int value = D <= 128 ? 2 : D / 64; };
 
 }  // namespace rrq
