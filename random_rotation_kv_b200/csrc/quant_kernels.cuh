@@ -349,6 +349,58 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
 }
 
 // ------------------------------------------------------------------ decode
+// Shared-memory ring that keeps each lane's codes and norm NS−1 grid-stride
+// iterations ahead (one lane per vector, d ≤ 128).  Every lane copies and
+// later reads only its own slots, so no warp synchronisation is needed; the
+// slot layout [stage][unit][lane] makes both the cp.async writes and the
+// reads of a warp touch consecutive words (no bank conflicts).
+template <int CB, int NS>
+struct CodeRing {
+  static constexpr int UNIT = (CB % 16 == 0) ? 16 : 8;  // bytes per copy
+  static constexpr int UPV = CB / UNIT;                  // units per vector
+  static constexpr int BYTES = NS * 32 * (CB + 4);       // per warp
+  uint8_t* base;  // this warp's ring
+
+  __device__ __forceinline__ uint8_t* unit(int stage, int u, int lane) const {
+    return base + ((stage * UPV + u) * 32 + lane) * UNIT;
+  }
+  __device__ __forceinline__ float* norm(int stage, int lane) const {
+    return reinterpret_cast<float*>(base + NS * 32 * CB) + stage * 32 + lane;
+  }
+  // Copy vector v's codes and norm into `stage` (zeros when v ≥ n).
+  __device__ __forceinline__ void issue(int stage, int lane, const uint8_t* codes,
+                                        const float* norms, int64_t v, int64_t n) const {
+    const bool ok = v < n;
+    const uint8_t* src = codes + (ok ? v : 0) * CB;
+#pragma unroll
+    for (int u = 0; u < UPV; ++u) {
+      if constexpr (UNIT == 16) cp_async16(smem_addr(unit(stage, u, lane)), src + u * 16, ok ? 16 : 0);
+      else cp_async8(smem_addr(unit(stage, u, lane)), src + u * 8, ok ? 8 : 0);
+    }
+    cp_async4(smem_addr(norm(stage, lane)), norms + (ok ? v : 0), ok ? 4 : 0);
+  }
+  __device__ __forceinline__ void read(int stage, int lane, uint32_t* words, float& nu) const {
+#pragma unroll
+    for (int u = 0; u < UPV; ++u) {
+      if constexpr (UNIT == 16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(unit(stage, u, lane));
+        words[4 * u] = v.x; words[4 * u + 1] = v.y; words[4 * u + 2] = v.z; words[4 * u + 3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(unit(stage, u, lane));
+        words[2 * u] = v.x; words[2 * u + 1] = v.y;
+      }
+    }
+    nu = *norm(stage, lane);
+  }
+};
+
+constexpr int kDecodeStages = 4;
+
+template <int D, int B>
+constexpr size_t decode_smem_bytes() {
+  return DecC<D>::value == D ? size_t(kThreads / 32) * CodeRing<D * B / 8, kDecodeStages>::BYTES : 0;
+}
+
 template <typename T, int D, int B>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
 decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms, int64_t n,
@@ -359,8 +411,10 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   constexpr int L = 1 << B;
   constexpr int CB = D * B / 8;
   constexpr int NW = (G == 1) ? CB / 4 : SEC * 2;  // code words held per lane
+  constexpr int NS = kDecodeStages;
   __shared__ __align__(16) uint32_t smask[mask_words<T, D>()];
   __shared__ float slev[L];
+  extern __shared__ __align__(16) uint8_t ring_mem[];
   build_sign_mask<T, D>(smask, p.seed);
   if (threadIdx.x < L) slev[threadIdx.x] = p.levels[threadIdx.x];
   __syncthreads();
@@ -368,34 +422,9 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   const int64_t gwarp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t stride = ((int64_t(gridDim.x) * blockDim.x) >> 5) * VPW;
-
   int64_t vec = gwarp * VPW + vsub;
-  uint32_t nw[NW];
-  float nu_next = 0.f;
-  auto fetch = [&](int64_t v) {
-    const bool ok = v < n;
-    const uint8_t* crow = codes + v * CB;
-    if constexpr (G == 1) {
-      load_bytes<CB>(crow, ok, nw);
-    } else {
-#pragma unroll
-      for (int s = 0; s < SEC; ++s) {
-        const uint64_t c = ok ? load_sector_codes<B>(crow, Lay::sector(s, h)) : 0ull;
-        nw[2 * s] = uint32_t(c);
-        nw[2 * s + 1] = uint32_t(c >> 32);
-      }
-    }
-    nu_next = ok ? __ldcs(norms + v) : 0.f;
-  };
-  fetch(vec);
-  for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
-    const bool valid = vec < n;
-    uint32_t cw[NW];
-#pragma unroll
-    for (int i = 0; i < NW; ++i) cw[i] = nw[i];
-    const float nu = nu_next;
-    fetch(vec + stride);  // next iteration, in flight now
 
+  auto body = [&](const uint32_t* cw, float nu, int64_t v) {
     float2 w[P];
 #pragma unroll
     for (int s = 0; s < SEC; ++s) {
@@ -413,7 +442,44 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
       }
     }
     fwht2<D, C>(w, h);
-    store_pairs<T, D, C, true>(out + vec * D, valid, h, smask, w, nu * p.inv_d);
+    store_pairs<T, D, C, true>(out + v * D, v < n, h, smask, w, nu * p.inv_d);
+  };
+
+  if constexpr (G == 1) {
+    const CodeRing<CB, NS> ring{ring_mem + (threadIdx.x >> 5) * CodeRing<CB, NS>::BYTES};
+#pragma unroll
+    for (int k = 0; k < NS - 1; ++k) {
+      ring.issue(k, lane, codes, norms, vec + k * stride, n);
+      cp_async_commit();
+    }
+    int stage = 0;
+    for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
+      cp_async_wait<NS - 2>();
+      uint32_t cw[NW];
+      float nu;
+      ring.read(stage, lane, cw, nu);
+      // refill the slot read in the previous iteration with iteration +NS−1
+      ring.issue((stage + NS - 1) % NS, lane, codes, norms, vec + (NS - 1) * stride, n);
+      cp_async_commit();
+      stage = (stage + 1) % NS;
+      body(cw, nu, vec);
+    }
+    cp_async_wait<0>();
+  } else {
+    // d > 128: several lanes per vector; codes read straight from global memory
+    for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
+      const bool ok = vec < n;
+      uint32_t cw[NW];
+      const uint8_t* crow = codes + (ok ? vec : 0) * CB;
+#pragma unroll
+      for (int s = 0; s < SEC; ++s) {
+        const uint64_t c = ok ? load_sector_codes<B>(crow, Lay::sector(s, h)) : 0ull;
+        cw[2 * s] = uint32_t(c);
+        cw[2 * s + 1] = uint32_t(c >> 32);
+      }
+      const float nu = ok ? __ldcs(norms + vec) : 0.f;
+      body(cw, nu, vec);
+    }
   }
 }
 
@@ -498,8 +564,9 @@ cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const
   constexpr int vpb = vectors_per_block<DecC<D>::value>(D);
   const int64_t work = (n + vpb - 1) / vpb;
   auto k = decode_kernel<T, D, B>;
-  const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
-  k<<<grid, kThreads, 0, stream>>>(codes, norms, n, out, p);
+  constexpr size_t smem = decode_smem_bytes<D, B>();
+  const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, smem, work);
+  k<<<grid, kThreads, smem, stream>>>(codes, norms, n, out, p);
   return cudaGetLastError();
 }
 
