@@ -396,9 +396,19 @@ struct CodeRing {
 
 constexpr int kDecodeStages = 4;
 
-template <int D, int B>
+// 4-bit codes and 16-bit outputs: look up a byte (two codes) at once.  Entry
+// e = lo | hi << 4 holds (c_lo + c_hi, c_lo − c_hi) as fp16 — the first
+// butterfly of the transform already applied.  The fp16 rounding (2^-12
+// relative) sits far below the 16-bit output's own rounding.  The table is
+// replicated per lane (word e·32 + lane), so every lane reads its own bank.
+template <typename T, int B>
+constexpr bool use_pair_table() { return B == 4 && Elem<T>::kBytes == 2; }
+constexpr int kPairTableWords = 256 * 32;
+
+template <typename T, int D, int B>
 constexpr size_t decode_smem_bytes() {
-  return DecC<D>::value == D ? size_t(kThreads / 32) * CodeRing<D * B / 8, kDecodeStages>::BYTES : 0;
+  return (DecC<D>::value == D ? size_t(kThreads / 32) * CodeRing<D * B / 8, kDecodeStages>::BYTES : 0) +
+         (use_pair_table<T, B>() ? kPairTableWords * 4 : 0);
 }
 
 template <typename T, int D, int B>
@@ -412,11 +422,22 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   constexpr int CB = D * B / 8;
   constexpr int NW = (G == 1) ? CB / 4 : SEC * 2;  // code words held per lane
   constexpr int NS = kDecodeStages;
+  constexpr bool PAIR = use_pair_table<T, B>();
   __shared__ __align__(16) uint32_t smask[mask_words<T, D>()];
   __shared__ float slev[L];
-  extern __shared__ __align__(16) uint8_t ring_mem[];
+  extern __shared__ __align__(16) uint8_t dyn_smem[];
+  uint32_t* ptab = reinterpret_cast<uint32_t*>(dyn_smem);  // pair table (PAIR only)
+  uint8_t* ring_mem = dyn_smem + (PAIR ? kPairTableWords * 4 : 0);
   build_sign_mask<T, D>(smask, p.seed);
   if (threadIdx.x < L) slev[threadIdx.x] = p.levels[threadIdx.x];
+  if constexpr (PAIR) {
+    for (int i = threadIdx.x; i < kPairTableWords; i += blockDim.x) {
+      const int e = i >> 5;
+      const float lo = p.levels[e & 15], hi = p.levels[e >> 4];
+      const __half2 v = __floats2half2_rn(lo + hi, lo - hi);
+      ptab[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  }
   __syncthreads();
 
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
@@ -424,24 +445,33 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   const int64_t stride = ((int64_t(gridDim.x) * blockDim.x) >> 5) * VPW;
   int64_t vec = gwarp * VPW + vsub;
 
+  const uint32_t* lane_tab = ptab + lane;
   auto body = [&](const uint32_t* cw, float nu, int64_t v) {
     float2 w[P];
 #pragma unroll
     for (int s = 0; s < SEC; ++s) {
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
-        uint32_t c0, c1;
-        if constexpr (G == 1) {
-          c0 = get_bits(cw, (s * 16 + e) * B, B);
-          c1 = get_bits(cw, (s * 16 + e + 1) * B, B);
+        if constexpr (PAIR) {
+          // byte (s·16 + e)/2 of the lane's code words: codes of values e, e+1
+          const int bytepos = G == 1 ? (s * 16 + e) * 4 : 64 * s + e * 4;
+          const uint32_t byte = get_bits(cw, bytepos, 8);
+          const uint32_t pv = lane_tab[byte << 5];
+          w[s * 8 + e / 2] = __half22float2(*reinterpret_cast<const __half2*>(&pv));
         } else {
-          c0 = get_bits(cw + 2 * s, e * B, B);
-          c1 = get_bits(cw + 2 * s, (e + 1) * B, B);
+          uint32_t c0, c1;
+          if constexpr (G == 1) {
+            c0 = get_bits(cw, (s * 16 + e) * B, B);
+            c1 = get_bits(cw, (s * 16 + e + 1) * B, B);
+          } else {
+            c0 = get_bits(cw + 2 * s, e * B, B);
+            c1 = get_bits(cw + 2 * s, (e + 1) * B, B);
+          }
+          w[s * 8 + e / 2] = make_float2(slev[c0], slev[c1]);
         }
-        w[s * 8 + e / 2] = make_float2(slev[c0], slev[c1]);
       }
     }
-    fwht2<D, C>(w, h);
+    fwht2<D, C, PAIR>(w, h);
     store_pairs<T, D, C, true>(out + v * D, v < n, h, smask, w, nu * p.inv_d);
   };
 
@@ -564,7 +594,12 @@ cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const
   constexpr int vpb = vectors_per_block<DecC<D>::value>(D);
   const int64_t work = (n + vpb - 1) / vpb;
   auto k = decode_kernel<T, D, B>;
-  constexpr size_t smem = decode_smem_bytes<D, B>();
+  constexpr size_t smem = decode_smem_bytes<T, D, B>();
+  if constexpr (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
   const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, smem, work);
   k<<<grid, kThreads, smem, stream>>>(codes, norms, n, out, p);
   return cudaGetLastError();

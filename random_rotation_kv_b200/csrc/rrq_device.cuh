@@ -247,13 +247,16 @@ __device__ __forceinline__ void store_pairs(T* __restrict__ row, bool valid, int
 // Unnormalised Walsh–Hadamard transform on packed pairs: w[k] holds values
 // r = 2k and 2k+1 of the lane.  Bit 0 of r is a butterfly inside each pair;
 // the other local bits pair whole registers; lane bits use shuffles.
-template <int D, int C>
+// PAIRED = true: the butterfly inside each pair was already applied.
+template <int D, int C, bool PAIRED = false>
 __device__ __forceinline__ void fwht2(float2 (&w)[C / 2], int h) {
   constexpr int P = C / 2, G = D / C;
+  if constexpr (!PAIRED) {
 #pragma unroll
-  for (int k = 0; k < P; ++k) {
-    const float a = w[k].x, b = w[k].y;
-    w[k] = make_float2(a + b, a - b);
+    for (int k = 0; k < P; ++k) {
+      const float a = w[k].x, b = w[k].y;
+      w[k] = make_float2(a + b, a - b);
+    }
   }
 #pragma unroll
   for (int mm = 1; mm < P; mm <<= 1) {
