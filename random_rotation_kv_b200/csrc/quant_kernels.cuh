@@ -24,6 +24,8 @@
 // half an equivalent search built from saturating FMAs (FMA pipe).
 #pragma once
 
+#include <type_traits>
+
 #include "rrq_device.cuh"
 
 namespace rrq {
@@ -349,67 +351,44 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
 }
 
 // ------------------------------------------------------------------ decode
-// Shared-memory ring that keeps each lane's codes and norm NS−1 grid-stride
-// iterations ahead (one lane per vector, d ≤ 128).  Every lane copies and
-// later reads only its own slots, so no warp synchronisation is needed; the
-// slot layout [stage][unit][lane] makes both the cp.async writes and the
-// reads of a warp touch consecutive words (no bank conflicts).
-template <int CB, int NS>
-struct CodeRing {
-  static constexpr int UNIT = (CB % 16 == 0) ? 16 : 8;  // bytes per copy
-  static constexpr int UPV = CB / UNIT;                  // units per vector
-  static constexpr int BYTES = NS * 32 * (CB + 4);       // per warp
-  uint8_t* base;  // this warp's ring
+// d ≤ 128: one lane per vector, batches of 32 consecutive vectors per warp.
+// Global traffic moves in whole lines while the arithmetic stays per lane:
+//  * codes and norms of batch k+NS−1 are copied (cp.async, 8 vectors = 512
+//    contiguous bytes per instruction) into a per-warp ring of padded rows
+//    (80 B for d·b/8 = 64: conflict-free 128-bit reads by the owning lane);
+//  * each lane writes its reconstructed row into a padded shared tile
+//    (row stride ≡ 16 mod 128 B: conflict-free) and issues a bulk (TMA) copy
+//    of that row to global memory.
+// d > 128: several lanes per vector (shuffle stages); codes read straight
+// from global memory, 32-byte stores.
+constexpr int kDecodeStages = 3;
 
-  __device__ __forceinline__ uint8_t* unit(int stage, int u, int lane) const {
-    return base + ((stage * UPV + u) * 32 + lane) * UNIT;
-  }
-  __device__ __forceinline__ float* norm(int stage, int lane) const {
-    return reinterpret_cast<float*>(base + NS * 32 * CB) + stage * 32 + lane;
-  }
-  // Copy vector v's codes and norm into `stage` (zeros when v ≥ n).
-  __device__ __forceinline__ void issue(int stage, int lane, const uint8_t* codes,
-                                        const float* norms, int64_t v, int64_t n) const {
-    const bool ok = v < n;
-    const uint8_t* src = codes + (ok ? v : 0) * CB;
-#pragma unroll
-    for (int u = 0; u < UPV; ++u) {
-      if constexpr (UNIT == 16) cp_async16(smem_addr(unit(stage, u, lane)), src + u * 16, ok ? 16 : 0);
-      else cp_async8(smem_addr(unit(stage, u, lane)), src + u * 8, ok ? 8 : 0);
-    }
-    cp_async4(smem_addr(norm(stage, lane)), norms + (ok ? v : 0), ok ? 4 : 0);
-  }
-  __device__ __forceinline__ void read(int stage, int lane, uint32_t* words, float& nu) const {
-#pragma unroll
-    for (int u = 0; u < UPV; ++u) {
-      if constexpr (UNIT == 16) {
-        const uint4 v = *reinterpret_cast<const uint4*>(unit(stage, u, lane));
-        words[4 * u] = v.x; words[4 * u + 1] = v.y; words[4 * u + 2] = v.z; words[4 * u + 3] = v.w;
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(unit(stage, u, lane));
-        words[2 * u] = v.x; words[2 * u + 1] = v.y;
-      }
-    }
-    nu = *norm(stage, lane);
-  }
-};
-
-constexpr int kDecodeStages = 4;
-
-// 4-bit codes and 16-bit outputs: look up a byte (two codes) at once.  Entry
-// e = lo | hi << 4 holds (c_lo + c_hi, c_lo − c_hi) as fp16 — the first
+// 4-bit codes and fp16 outputs: look up a byte (two codes) at once.  Entry
+// e = lo | hi << 4 holds (c_lo + c_hi, c_lo − c_hi) in fp16 — the first
 // butterfly of the transform already applied.  The fp16 rounding (2^-12
-// relative) sits far below the 16-bit output's own rounding.  The table is
-// replicated per lane (word e·32 + lane), so every lane reads its own bank.
+// relative) is below the fp16 output's own rounding; bf16 and fp32 outputs use
+// exact fp32 levels.  The table is replicated per lane (word e·32 + lane), so
+// every lane reads its own bank.
 template <typename T, int B>
-constexpr bool use_pair_table() { return B == 4 && Elem<T>::kBytes == 2; }
+constexpr bool use_pair_table() { return B == 4 && std::is_same<T, __half>::value; }
 constexpr int kPairTableWords = 256 * 32;
 
-template <typename T, int D, int B>
-constexpr size_t decode_smem_bytes() {
-  return (DecC<D>::value == D ? size_t(kThreads / 32) * CodeRing<D * B / 8, kDecodeStages>::BYTES : 0) +
-         (use_pair_table<T, B>() ? kPairTableWords * 4 : 0);
-}
+template <typename T, int D, int B> struct DecodeSmem {
+  static constexpr int CB = D * B / 8;
+  static constexpr int CBP = (CB + 15) / 16 * 16;       // codes, padded
+  static constexpr int RR = CBP + 16;                    // ring row: codes | norm | pad
+  static constexpr int UNIT = (CB % 16 == 0) ? 16 : 8;  // cp.async unit
+  static constexpr int UPV = CB / UNIT;
+  static constexpr int ROW = D * Elem<T>::kBytes;        // output row bytes
+  static constexpr int TROW = ROW + 16;                  // padded tile row
+  static constexpr int RING = kDecodeStages * 32 * RR;
+  static constexpr int WARP = RING + 32 * TROW;          // per warp
+  static constexpr bool ONE_LANE = DecC<D>::value == D;
+  static constexpr size_t total() {
+    return (ONE_LANE ? size_t(kThreads / 32) * WARP : 0) +
+           (use_pair_table<T, B>() ? size_t(kPairTableWords) * 4 : 0);
+  }
+};
 
 template <typename T, int D, int B>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
@@ -417,9 +396,10 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
               T* __restrict__ out, const QuantParams p) {
   constexpr int C = DecC<D>::value;
   using Lay = Layout<D, C>;
+  using SM = DecodeSmem<T, D, B>;
   constexpr int G = Lay::G, P = Lay::P, SEC = Lay::SEC, VPW = Lay::VPW;
   constexpr int L = 1 << B;
-  constexpr int CB = D * B / 8;
+  constexpr int CB = SM::CB;
   constexpr int NW = (G == 1) ? CB / 4 : SEC * 2;  // code words held per lane
   constexpr int NS = kDecodeStages;
   constexpr bool PAIR = use_pair_table<T, B>();
@@ -427,7 +407,7 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   __shared__ float slev[L];
   extern __shared__ __align__(16) uint8_t dyn_smem[];
   uint32_t* ptab = reinterpret_cast<uint32_t*>(dyn_smem);  // pair table (PAIR only)
-  uint8_t* ring_mem = dyn_smem + (PAIR ? kPairTableWords * 4 : 0);
+  uint8_t* warp_mem = dyn_smem + (PAIR ? kPairTableWords * 4 : 0) + (threadIdx.x >> 5) * SM::WARP;
   build_sign_mask<T, D>(smask, p.seed);
   if (threadIdx.x < L) slev[threadIdx.x] = p.levels[threadIdx.x];
   if constexpr (PAIR) {
@@ -443,20 +423,17 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   const int64_t gwarp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t stride = ((int64_t(gridDim.x) * blockDim.x) >> 5) * VPW;
-  int64_t vec = gwarp * VPW + vsub;
-
   const uint32_t* lane_tab = ptab + lane;
-  auto body = [&](const uint32_t* cw, float nu, int64_t v) {
-    float2 w[P];
+
+  // codes -> levels (in pairs) -> transform; w holds the lane's values
+  auto expand = [&](const uint32_t* cw, float2 (&w)[P]) {
 #pragma unroll
     for (int s = 0; s < SEC; ++s) {
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
         if constexpr (PAIR) {
-          // byte (s·16 + e)/2 of the lane's code words: codes of values e, e+1
           const int bytepos = G == 1 ? (s * 16 + e) * 4 : 64 * s + e * 4;
-          const uint32_t byte = get_bits(cw, bytepos, 8);
-          const uint32_t pv = lane_tab[byte << 5];
+          const uint32_t pv = lane_tab[get_bits(cw, bytepos, 8) << 5];
           w[s * 8 + e / 2] = __half22float2(*reinterpret_cast<const __half2*>(&pv));
         } else {
           uint32_t c0, c1;
@@ -472,31 +449,67 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
       }
     }
     fwht2<D, C, PAIR>(w, h);
-    store_pairs<T, D, C, true>(out + v * D, v < n, h, smask, w, nu * p.inv_d);
   };
 
   if constexpr (G == 1) {
-    const CodeRing<CB, NS> ring{ring_mem + (threadIdx.x >> 5) * CodeRing<CB, NS>::BYTES};
+    uint8_t* ring = warp_mem;
+    uint8_t* tile_row = warp_mem + SM::RING + lane * SM::TROW;
+    // warp-cooperative copy of batch `bvec` (32 vectors from bvec) into stage
+    auto issue = [&](int stage, int64_t bvec) {
+      uint8_t* st = ring + stage * 32 * SM::RR;
+#pragma unroll
+      for (int i = 0; i < SM::UPV; ++i) {
+        const int t = lane + 32 * i;  // unit t of the batch
+        const int v = t / SM::UPV, u = t % SM::UPV;
+        const bool ok = bvec + v < n;
+        const uint8_t* src = codes + (ok ? (bvec + v) * CB + u * SM::UNIT : 0);
+        const uint32_t dst = smem_addr(st + v * SM::RR + u * SM::UNIT);
+        if constexpr (SM::UNIT == 16) cp_async16(dst, src, ok ? 16 : 0);
+        else cp_async8(dst, src, ok ? 8 : 0);
+      }
+      const bool ok = bvec + lane < n;
+      cp_async4(smem_addr(st + lane * SM::RR + SM::CBP), norms + (ok ? bvec + lane : 0), ok ? 4 : 0);
+    };
+    const int64_t wbase = gwarp * 32;
 #pragma unroll
     for (int k = 0; k < NS - 1; ++k) {
-      ring.issue(k, lane, codes, norms, vec + k * stride, n);
+      issue(k, wbase + k * stride);
       cp_async_commit();
     }
     int stage = 0;
-    for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
+    for (int64_t base = wbase; base < n; base += stride) {
       cp_async_wait<NS - 2>();
+      __syncwarp();
+      const uint8_t* row = ring + stage * 32 * SM::RR + lane * SM::RR;
       uint32_t cw[NW];
-      float nu;
-      ring.read(stage, lane, cw, nu);
-      // refill the slot read in the previous iteration with iteration +NS−1
-      ring.issue((stage + NS - 1) % NS, lane, codes, norms, vec + (NS - 1) * stride, n);
+#pragma unroll
+      for (int i = 0; i < CB / 4; i += (SM::UNIT / 4)) {
+        if constexpr (SM::UNIT == 16) {
+          const uint4 v = *reinterpret_cast<const uint4*>(row + 4 * i);
+          cw[i] = v.x; cw[i + 1] = v.y; cw[i + 2] = v.z; cw[i + 3] = v.w;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(row + 4 * i);
+          cw[i] = v.x; cw[i + 1] = v.y;
+        }
+      }
+      const float nu = *reinterpret_cast<const float*>(row + SM::CBP);
+      __syncwarp();  // every lane has read this stage before it is refilled
+      issue((stage + NS - 1) % NS, base + (NS - 1) * stride);
       cp_async_commit();
       stage = (stage + 1) % NS;
-      body(cw, nu, vec);
+
+      float2 w[P];
+      expand(cw, w);
+      const int64_t vec = base + lane;
+      bulk_wait_read_all();  // the previous bulk store has read this lane's tile row
+      store_pairs_smem<T, D>(tile_row, smask, w, nu * p.inv_d);
+      fence_proxy_async_smem();
+      if (vec < n) bulk_store(out + vec * D, smem_addr(tile_row), SM::ROW);
     }
     cp_async_wait<0>();
+    bulk_wait_all();
   } else {
-    // d > 128: several lanes per vector; codes read straight from global memory
+    int64_t vec = gwarp * VPW + vsub;
     for (int64_t base = gwarp * VPW; base < n; base += stride, vec += stride) {
       const bool ok = vec < n;
       uint32_t cw[NW];
@@ -508,7 +521,9 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
         cw[2 * s + 1] = uint32_t(c >> 32);
       }
       const float nu = ok ? __ldcs(norms + vec) : 0.f;
-      body(cw, nu, vec);
+      float2 w[P];
+      expand(cw, w);
+      store_pairs<T, D, C, true>(out + vec * D, ok, h, smask, w, nu * p.inv_d);
     }
   }
 }
@@ -594,7 +609,7 @@ cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const
   constexpr int vpb = vectors_per_block<DecC<D>::value>(D);
   const int64_t work = (n + vpb - 1) / vpb;
   auto k = decode_kernel<T, D, B>;
-  constexpr size_t smem = decode_smem_bytes<T, D, B>();
+  constexpr size_t smem = DecodeSmem<T, D, B>::total();
   if constexpr (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

@@ -115,6 +115,22 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Bulk (TMA) copy of a shared-memory range to global memory; the issuing
+// thread later waits for the source to be read before reusing it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
+               "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // 2 packed 16-bit elements -> 2 floats (exact)
 template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t w);
 template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t w) {
@@ -240,6 +256,35 @@ __device__ __forceinline__ void store_pairs(T* __restrict__ row, bool valid, int
         }
       }
       if (valid) st256(row + q * 16 + c * (32 / Elem<T>::kBytes), o);
+    }
+  }
+}
+
+// One lane's whole row (G = 1) times `scale`, sign XOR applied, into shared
+// memory at `dst` (16-byte stores, 16-byte aligned).
+template <typename T, int D>
+__device__ __forceinline__ void store_pairs_smem(uint8_t* dst, const uint32_t* smask,
+                                                 const float2 (&w)[D / 2], float scale) {
+  const float2 s2 = make_float2(scale, scale);
+  if constexpr (Elem<T>::kBytes == 2) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {  // chunk c: values 8c .. 8c+7
+      const uint4 m = reinterpret_cast<const uint4*>(smask)[c];
+      uint4 o;
+      o.x = pack2<T>(mul2(w[4 * c + 0], s2)) ^ m.x;
+      o.y = pack2<T>(mul2(w[4 * c + 1], s2)) ^ m.y;
+      o.z = pack2<T>(mul2(w[4 * c + 2], s2)) ^ m.z;
+      o.w = pack2<T>(mul2(w[4 * c + 3], s2)) ^ m.w;
+      reinterpret_cast<uint4*>(dst)[c] = o;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {  // chunk c: values 4c .. 4c+3
+      const uint4 m = reinterpret_cast<const uint4*>(smask)[c];
+      const float2 a = mul2(w[2 * c], s2), b = mul2(w[2 * c + 1], s2);
+      reinterpret_cast<uint4*>(dst)[c] =
+          make_uint4(__float_as_uint(a.x) ^ m.x, __float_as_uint(a.y) ^ m.y,
+                     __float_as_uint(b.x) ^ m.z, __float_as_uint(b.y) ^ m.w);
     }
   }
 }
