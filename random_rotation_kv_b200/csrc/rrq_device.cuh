@@ -156,11 +156,7 @@ template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float2 v) {
 // Each component is rounded once, exactly like the scalar operation.
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  const unsigned long long ua = *reinterpret_cast<const unsigned long long*>(&a);
-  const unsigned long long ub = *reinterpret_cast<const unsigned long long*>(&b);
-  unsigned long long ur;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(ur) : "l"(ua), "l"(ub));
-  return *reinterpret_cast<float2*>(&ur);
+  return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a − b: b·(−1) is exact
 }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
