@@ -384,14 +384,18 @@ template <typename T, int D, int B> struct DecodeSmem {
   static constexpr int RING = kDecodeStages * 32 * RR;
   static constexpr int WARP = RING + 32 * TROW;          // per warp
   static constexpr bool ONE_LANE = DecC<D>::value == D;
-  static constexpr size_t total() {
-    return (ONE_LANE ? size_t(kThreads / 32) * WARP : 0) +
-           (use_pair_table<T, B>() ? size_t(kPairTableWords) * 4 : 0);
-  }
+  static constexpr int TABLE = use_pair_table<T, B>() ? kPairTableWords * 4 : 0;
+  // One block per SM holding as many warps as shared memory allows (≤ 12,
+  // which the 168-register budget also allows); the warps share one table.
+  static constexpr int kMaxBlockSmem = 227 * 1024;
+  static constexpr int WARPS_BY_SMEM = ONE_LANE ? (kMaxBlockSmem - TABLE) / WARP : 12;
+  static constexpr int WARPS = WARPS_BY_SMEM < 12 ? WARPS_BY_SMEM : 12;
+  static constexpr int THREADS = WARPS * 32;
+  static constexpr size_t total() { return (ONE_LANE ? size_t(WARPS) * WARP : 0) + TABLE; }
 };
 
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(kThreads, kMinBlocks)
+__global__ void __launch_bounds__(DecodeSmem<T, D, B>::THREADS, 1)
 decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms, int64_t n,
               T* __restrict__ out, const QuantParams p) {
   constexpr int C = DecC<D>::value;
@@ -606,7 +610,8 @@ cudaError_t encode_typed(const T* x, int64_t n, int d, const QuantParams& p, uin
 template <typename T, int D, int B>
 cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const QuantParams& p,
                       T* out, cudaStream_t stream) {
-  constexpr int vpb = vectors_per_block<DecC<D>::value>(D);
+  using SM = DecodeSmem<T, D, B>;
+  constexpr int vpb = SM::WARPS * (32 / (D / DecC<D>::value));
   const int64_t work = (n + vpb - 1) / vpb;
   auto k = decode_kernel<T, D, B>;
   constexpr size_t smem = DecodeSmem<T, D, B>::total();
@@ -615,8 +620,8 @@ cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
   }
-  const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, smem, work);
-  k<<<grid, kThreads, smem, stream>>>(codes, norms, n, out, p);
+  const int grid = grid_for(reinterpret_cast<const void*>(k), SM::THREADS, smem, work);
+  k<<<grid, SM::THREADS, smem, stream>>>(codes, norms, n, out, p);
   return cudaGetLastError();
 }
 
