@@ -165,6 +165,7 @@ int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norm
     return RRQ_ERR_INVALID;
   const int group = hq / hkv;
   if (group != 1 && group != 2 && group != 4 && group != 8) return RRQ_ERR_UNSUPPORTED;
+  if (!rrq::qk_scores_supported(d, bits, hq, hkv)) return RRQ_ERR_UNSUPPORTED;
   rrq::QuantParams p;
   if (make_params(bits, codebook, seed, d, &p) != RRQ_OK) return RRQ_ERR_INVALID;
   if (T == 0) return RRQ_OK;

@@ -2,10 +2,6 @@
 #include "rrq_params.h"
 
 namespace rrq {
-cudaError_t launch_qk_scores(const void*, int, const uint8_t*, const float*, int64_t, int, int,
-                             const QuantParams&, float, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
-}
 cudaError_t launch_q4_0(const void*, int, int64_t, int, uint64_t, int, float, void*, cudaStream_t) {
   return cudaErrorNotSupported;
 }

@@ -227,15 +227,6 @@ __device__ __forceinline__ void load_bytes(const uint8_t* __restrict__ p, bool v
   }
 }
 
-// Bits [pos, pos+nb) of a little-endian word array (nb ≤ 8; pos and nb are
-// constants after unrolling, so the array stays in registers).
-__device__ __forceinline__ uint32_t get_bits(const uint32_t* words, int pos, int nb) {
-  const int wi = pos >> 5, off = pos & 31;
-  uint32_t v = words[wi] >> off;
-  if (off + nb > 32) v |= words[wi + 1] << (32 - off);
-  return v & ((1u << nb) - 1u);
-}
-
 // One sector (2B bytes) of a row at byte offset q·2B (G > 1 layouts).
 template <int B>
 __device__ __forceinline__ void store_sector_codes(uint8_t* __restrict__ row, int q, uint64_t v) {

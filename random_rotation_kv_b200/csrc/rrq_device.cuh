@@ -323,6 +323,15 @@ __device__ __forceinline__ void fwht2(float2 (&w)[C / 2], int h) {
   }
 }
 
+// Bits [pos, pos+nb) of a little-endian word array (nb ≤ 8; pos and nb are
+// constants after unrolling, so the array stays in registers).
+__device__ __forceinline__ uint32_t get_bits(const uint32_t* words, int pos, int nb) {
+  const int wi = pos >> 5, off = pos & 31;
+  uint32_t v = words[wi] >> off;
+  if (off + nb > 32) v |= words[wi + 1] << (32 - off);
+  return v & ((1u << nb) - 1u);
+}
+
 // Sum over the G lanes of a group.
 template <int G>
 __device__ __forceinline__ float group_sum(float x) {

@@ -35,6 +35,9 @@ cudaError_t launch_decode(const uint8_t* codes, const float* norms, int64_t n, i
 cudaError_t launch_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norms,
                              int64_t T, int hkv, int d, const QuantParams& p, float scale,
                              float* scores, cudaStream_t stream);
+// Whether rrq_qk_scores supports (d, bits, hq, hkv): hkv a power of two and
+// the kernel's shared-memory footprint within one CTA's limit.
+bool qk_scores_supported(int d, int bits, int hq, int hkv);
 cudaError_t launch_q4_0(const void* x, int dtype, int64_t n, int d, uint64_t seed, int rotate,
                         float inv_sqrt_d, void* blocks, cudaStream_t stream);
 cudaError_t launch_q4_0_decode(const void* blocks, int64_t n, int d, uint64_t seed, int rotate,
