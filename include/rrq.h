@@ -182,7 +182,7 @@ int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norm
  * stored as 18 bytes: fp16(Δ) little endian, then byte j = q_j | q_{j+16}<<4
  * (the public llama.cpp q4_0 block, kept identical for interoperability).
  *   x       [n × d] of x_dtype (d a multiple of 32 within [64, 512])
- *   blocks  [n × d/32 × 18] bytes (output; 2-byte aligned suffices)
+ *   blocks  [n × d/32 × 18] bytes (output; 16-byte aligned)
  * Errors: RRQ_ERR_INVALID, RRQ_ERR_CUDA.
  */
 int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate,

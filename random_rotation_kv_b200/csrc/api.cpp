@@ -177,7 +177,7 @@ int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, in
                  void* blocks, void* stream) {
   if (n < 0 || !d_ok(d) || !dtype_ok(x_dtype) || (rotate != 0 && rotate != 1))
     return RRQ_ERR_INVALID;
-  if (!arr_ok(x, n, 16) || !arr_ok(blocks, n, 2)) return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 32) || !arr_ok(blocks, n, 16)) return RRQ_ERR_INVALID;
   if (n == 0) return RRQ_OK;
   const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   return status_of(rrq::launch_q4_0(x, x_dtype, n, d, seed, rotate, inv_sqrt_d, blocks,
@@ -188,7 +188,7 @@ int rrq_q4_0_rot_decode(const void* blocks, int64_t n, int d, uint64_t seed, int
                         int out_dtype, void* stream) {
   if (n < 0 || !d_ok(d) || !dtype_ok(out_dtype) || (rotate != 0 && rotate != 1))
     return RRQ_ERR_INVALID;
-  if (!arr_ok(blocks, n, 2) || !arr_ok(out, n, 16)) return RRQ_ERR_INVALID;
+  if (!arr_ok(blocks, n, 16) || !arr_ok(out, n, 32)) return RRQ_ERR_INVALID;
   if (n == 0) return RRQ_OK;
   const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   return status_of(rrq::launch_q4_0_decode(blocks, n, d, seed, rotate, inv_sqrt_d, out, out_dtype,
