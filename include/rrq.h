@@ -178,7 +178,7 @@ int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norm
  * ordinary block format, q4_0 first of all.  With y = Πx (rotate = 1) or
  * y = x (rotate = 0), per block of 32 consecutive coordinates:
  *     m = the element of largest |y| (first on ties), Δ = m/−8 (fp32),
- *     q_j = min(15, ⌊y_j/Δ + 8.5⌋)  (y_j·(1/Δ); 1/Δ := 0 when Δ = 0),
+ *     q_j = min(15, ⌊fp32(fp32(y_j·inv) + 8.5)⌋),  inv = fp32(1/Δ) (0 when Δ = 0),
  * stored as 18 bytes: fp16(Δ) little endian, then byte j = q_j | q_{j+16}<<4
  * (the public llama.cpp q4_0 block, kept identical for interoperability).
  *   x       [n × d] of x_dtype (d a multiple of 32 within [64, 512])

@@ -11,9 +11,12 @@ The page names q4_0 but does not define it.  The reading used (the public
 llama.cpp/GGML q4_0 block, kept identical for interoperability):
 
 * blocks of 32 consecutive (rotated) coordinates;
+* the decisions are taken in fp32, the precision of the format's reference
+  arithmetic (the pages fix none): y is rounded to fp32 first;
 * m = the block element of largest magnitude, with its sign (first index on
-  ties); Δ = fp32(m) / −8; inv = 1/Δ (0 when Δ = 0);
-* q_j = min(15, ⌊y_j·inv + 8.5⌋) (the argument is ≥ 0.5 since |y_j·inv| ≤ 8);
+  ties); Δ = m / −8 (exact); inv = fp32(1/Δ) (0 when Δ = 0);
+* q_j = min(15, ⌊fp32(fp32(y_j·inv) + 8.5)⌋) (the argument is ≥ 0.5 since
+  |y_j·inv| ≤ 8);
 * stored: fp16(Δ) (2 bytes, little endian) then 16 bytes; byte j holds q_j in
   its low nibble and q_{j+16} in its high nibble — 18 bytes per block;
 * decode: (q_j − 8)·fp16(Δ), then Πᵀ when the vector was rotated.
@@ -50,16 +53,17 @@ def encode(x, seed: int, rotate_first: bool = True) -> Q4Encoded:
     y = rotate(x, seed) if rotate_first else x.copy()
     nb = d // BLOCK
     yb = y.reshape(n, nb, BLOCK)
-    idx = np.argmax(np.abs(yb), axis=2)  # first index on ties
-    m = np.take_along_axis(yb, idx[:, :, None], axis=2)[:, :, 0]
-    delta = (m.astype(np.float32) / np.float32(-8.0)).astype(np.float32)
-    d64 = delta.astype(np.float64)
-    inv = np.zeros_like(d64)
-    nz = d64 != 0
-    inv[nz] = 1.0 / d64[nz]
-    ratio = yb * inv[:, :, None] + 8.5
-    q = np.minimum(15, np.floor(ratio)).astype(np.int64)
-    q = np.maximum(q, 0)
+    y32 = yb.astype(np.float32)
+    idx = np.argmax(np.abs(y32), axis=2)  # first index on ties
+    m = np.take_along_axis(y32, idx[:, :, None], axis=2)[:, :, 0]
+    delta = (m / np.float32(-8.0)).astype(np.float32)
+    inv = np.zeros_like(delta)
+    nz = delta != 0
+    inv[nz] = np.float32(1.0) / delta[nz]
+    r32 = (y32 * inv[:, :, None]).astype(np.float32) + np.float32(8.5)
+    q = np.minimum(15, np.maximum(0, np.floor(r32))).astype(np.int64)
+    # the same quantity in fp64, for measuring distances to code boundaries
+    ratio = yb * inv[:, :, None].astype(np.float64) + 8.5
     # serialise: fp16 delta, then nibbles (j low, j+16 high)
     blocks = np.zeros((n, nb, BLOCK_BYTES), dtype=np.uint8)
     dh = delta.astype(np.float16).view(np.uint16)

@@ -6,7 +6,7 @@
 // defining it; the public llama.cpp q4_0 block is used, kept identical for
 // interoperability:
 //   m = block element of largest |y| (first on ties), Δ = m/−8 (fp32),
-//   q_j = min(15, ⌊y_j·(1/Δ) + 8.5⌋) (1/Δ := 0 when Δ = 0),
+//   q_j = min(15, ⌊fp32(fp32(y_j·inv) + 8.5)⌋), inv = fp32(1/Δ) (0 when Δ = 0),
 //   18 bytes: fp16(Δ) little endian, then byte j = q_j | q_{j+16} << 4;
 //   decode: (q_j − 8)·fp16(Δ).
 // With rotation y = Πx = H·D·x/√d, decode applies Πᵀ = D·H/√d.
@@ -61,8 +61,10 @@ __device__ __forceinline__ uint2 sector_codes_q4(const float2* w, float inv) {
   uint32_t out[2] = {0u, 0u};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const int q0 = min(15, max(0, int(floorf(fmaf(w[k].x, inv, 8.5f)))));
-    const int q1 = min(15, max(0, int(floorf(fmaf(w[k].y, inv, 8.5f)))));
+    // fp32 y·inv, then + 8.5, each rounded (no fused multiply-add), as the
+    // format's reference arithmetic
+    const int q0 = min(15, max(0, int(floorf(__fadd_rn(__fmul_rn(w[k].x, inv), 8.5f)))));
+    const int q1 = min(15, max(0, int(floorf(__fadd_rn(__fmul_rn(w[k].y, inv), 8.5f)))));
     out[k / 4] |= (uint32_t(q0) << (8 * (k % 4))) | (uint32_t(q1) << (8 * (k % 4) + 4));
   }
   return make_uint2(out[0], out[1]);
