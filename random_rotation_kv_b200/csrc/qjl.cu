@@ -1,0 +1,393 @@
+// qjl.cu — MSE encode fused with the QJL 1-bit sketch of the residual, with
+// the d×d projection on the 5th-generation tensor cores (tcgen05).
+//
+// "Random-rotation quantization" page, "History": QJL — a DRIVE-style one-bit
+// construction for attention keys made unbiased through residuals;
+// TurboQuant — a (b−1)-bit biased MSE quantiser followed by an unbiased 1-bit
+// one.  "Bias vs unbiasedness": the residual chain removes the MSE shrinkage.
+// For each vector:
+//     r = Πx − ŷ (rotated domain, ŷ = (ν/√d)·c[code]),  ρ = ‖r‖₂,
+//     v = S·r (S: d×d, bf16-valued Gaussian),  bit_i = [v_i > 0].
+//
+// Tile of 128 vectors per CTA iteration (one thread per vector, d = 128):
+//  1. the input tile arrives by cp.async in padded shared rows (prefetched one
+//     tile ahead);
+//  2. each thread runs the MSE encoder on its vector (codes and ν to global
+//     memory), forms r in fp32 and splits it exactly into three bf16 parts
+//     r = r_hi + r_mid + r_lo (8 significant bits each: together the 24 of
+//     fp32), written into three A operand tiles [128 × 128] (K-major, no
+//     swizzle: 8×16-byte core matrices);
+//  3. one thread issues 3 × 8 tcgen05.mma (M = 128, N = 128, K = 16,
+//     bf16 × bf16 → fp32) against S (B operand, resident for the whole
+//     kernel), accumulating V = R·Sᵀ in tensor memory; products are exact and
+//     only the fp32 accumulation rounds;
+//  4. tcgen05.commit arrives on an mbarrier; each warp reads its 32 TMEM lanes
+//     (one lane = one vector's 128 outputs) and packs the signs.
+// Every wait is bounded; on a timeout the tile's residual norms are set to
+// NaN, the CTA drains its copies, frees its tensor memory and returns.
+#include "quant_kernels.cuh"
+
+namespace rrq {
+namespace {
+
+constexpr int kQjlD = 128;
+constexpr int kQjlTile = 128;
+constexpr int kQjlThreads = 128;
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kWaitLimit = 1u << 24;  // try_wait polls before giving up
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, no swizzle (canonical layout of
+// 8-row × 16-byte core matrices; lbo = distance between core matrices along K,
+// sbo = distance between 8-row groups).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;  // descriptor version for sm_100
+  return d;                // base offset 0, layout type 0 (no swizzle)
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
+// N = 128 (bits 17..22 = N/8), M = 128 (bits 24..28 = M/16).
+constexpr uint32_t kIdescBf16M128N128 =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((128u / 8) << 17) | ((128u / 16) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdescBf16M128N128), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Byte offset of element (row, k) in a [128 × 128] bf16 K-major core-matrix tile.
+constexpr uint32_t kLbo = 128;   // next 8 k
+constexpr uint32_t kSbo = 2048;  // next 8 rows
+__device__ __forceinline__ uint32_t cm_offset(int row, int kb) {  // kb = k/8, 16-byte chunk
+  return uint32_t(row >> 3) * kSbo + uint32_t(kb) * kLbo + uint32_t(row & 7) * 16;
+}
+
+template <typename T>
+struct QjlSmem {
+  static constexpr int ROWB = kQjlD * Elem<T>::kBytes;       // input row bytes
+  static constexpr int ROWP = ROWB + 16;                      // padded
+  static constexpr int STAGES = Elem<T>::kBytes == 2 ? 2 : 1;
+  static constexpr int OPER = kQjlTile * kQjlD * 2;          // one bf16 operand tile (32 KB)
+  static constexpr int S_OFF = 0;
+  static constexpr int A_OFF = S_OFF + OPER;                  // 3 parts
+  static constexpr int IN_OFF = A_OFF + 3 * OPER;
+  static constexpr int IN_BYTES = STAGES * kQjlTile * ROWP;
+  static constexpr int TOTAL = IN_OFF + IN_BYTES;
+};
+
+struct QjlArgs {
+  const void* x;
+  int64_t n;
+  const uint16_t* S;  // bf16 bits [128][128]
+  uint8_t* codes;
+  float* norms;
+  uint8_t* qbits;
+  float* rnorm;
+  QuantParams p;
+};
+
+template <typename T, int B, bool SYM>
+__global__ void __launch_bounds__(kQjlThreads, 1) qjl_encode_kernel(const QjlArgs a) {
+  using Sm = QjlSmem<T>;
+  constexpr int D = kQjlD, P = D / 2, SEC = D / 16, L = 1 << B, CB = D * B / 8;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ __align__(16) uint32_t smask[mask_words<T, D>()];
+  __shared__ float slev[L];
+  __shared__ __align__(8) uint64_t mbar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int tile_ok;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const QuantParams& p = a.p;
+  const T* x = static_cast<const T*>(a.x);
+  build_sign_mask<T, D>(smask, p.seed);
+  if (tid < L) slev[tid] = p.levels[tid];
+  // S -> B operand tile (core-matrix layout), 16-byte chunks
+  for (int c = tid; c < kQjlD * 16; c += kQjlThreads) {
+    const int row = c >> 4, kb = c & 15;
+    const uint4 v = *reinterpret_cast<const uint4*>(a.S + row * kQjlD + kb * 8);
+    *reinterpret_cast<uint4*>(smem + Sm::S_OFF + cm_offset(row, kb)) = v;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) mbar_init(&mbar, 1);
+  fence_proxy_async_smem();  // S tile and barrier visible to the async proxy
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  const int64_t ntiles = (a.n + kQjlTile - 1) / kQjlTile;
+  // input tile t -> stage: 128 rows, 16-byte units, coalesced, padded rows
+  auto issue = [&](int stage, int64_t t) {
+    uint8_t* st = smem + Sm::IN_OFF + stage * kQjlTile * Sm::ROWP;
+    constexpr int UPR = Sm::ROWB / 16;  // units per row
+    for (int u = tid; u < kQjlTile * UPR; u += kQjlThreads) {
+      const int row = u / UPR, c = u % UPR;
+      const int64_t v = t * kQjlTile + row;
+      const bool ok = t < ntiles && v < a.n;
+      const uint8_t* src = static_cast<const uint8_t*>(a.x) + (ok ? v * Sm::ROWB + c * 16 : 0);
+      cp_async16(smem_addr(st + row * Sm::ROWP + c * 16), src, ok ? 16 : 0);
+    }
+  };
+  int64_t t = blockIdx.x;
+  if constexpr (Sm::STAGES == 2) issue(0, t);
+  cp_async_commit();
+  uint32_t phase = 0;
+  bool failed = false;
+  for (int it = 0; t < ntiles; ++it, t += gridDim.x) {
+    const int stage = Sm::STAGES == 2 ? (it & 1) : 0;
+    if constexpr (Sm::STAGES == 2) {
+      issue(stage ^ 1, t + gridDim.x);  // next tile, in flight now
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      issue(0, t);
+      cp_async_commit();
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+
+    // ---- MSE encode of vector `vec` by this thread
+    const int64_t vec = t * kQjlTile + tid;
+    const bool valid = vec < a.n;
+    const uint8_t* row = smem + Sm::IN_OFF + stage * kQjlTile * Sm::ROWP + tid * Sm::ROWP;
+    float2 w[P];
+#pragma unroll
+    for (int s = 0; s < SEC; ++s) {
+      uint32_t raw[sector_words<T>()];
+#pragma unroll
+      for (int c = 0; c < sector_words<T>() / 4; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + s * 16 * Elem<T>::kBytes + c * 16);
+        raw[4 * c] = v.x; raw[4 * c + 1] = v.y; raw[4 * c + 2] = v.z; raw[4 * c + 3] = v.w;
+      }
+      sector_to_pairs<T, true>(raw, smask + s * sector_words<T>(), &w[s * 8]);
+    }
+    float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < P; ++k) ss2 = fma2(w[k], w[k], ss2);
+    const float nu = sqrtf(ss2.x + ss2.y);
+    fwht2<D, D>(w, 0);
+    const float ns = nu > 0.f ? nu : 1.f;
+    uint64_t sec[SEC];
+    {
+      float tp[npos<B>()] = {};
+      float tg[L - 1] = {};
+      if constexpr (SYM) {
+#pragma unroll
+        for (int j = 0; j < L / 2 - 1; ++j) tp[j] = ns * p.thr[L / 2 + j];
+      } else {
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) tg[k] = ns * p.thr[k];
+      }
+#pragma unroll
+      for (int s = 0; s < SEC; ++s) sec[s] = sector_codes<B, SYM>(&w[s * 8], tp, tg);
+    }
+    {
+      uint32_t words[CB / 4];
+#pragma unroll
+      for (int i = 0; i < CB / 4; ++i) words[i] = 0u;
+#pragma unroll
+      for (int s = 0; s < SEC; ++s) {  // sector s at bit s·16B
+        const int pos = s * 16 * B, wi = pos / 32, off = pos % 32;
+        words[wi] |= uint32_t(sec[s] << off);
+        if (off + 16 * B > 32) words[wi + 1] |= uint32_t(sec[s] >> (32 - off));
+        if (off + 16 * B > 64) words[wi + 2] |= uint32_t(sec[s] >> (64 - off));
+      }
+      if (valid) {
+        store_bytes<CB>(a.codes + vec * CB, words);
+        a.norms[vec] = nu;
+      }
+    }
+
+    // ---- residual r = (y' − ν·c[code])/√d, split into three bf16 parts
+    float rr = 0.f;
+#pragma unroll
+    for (int s = 0; s < SEC; ++s) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // 8 values = one 16-byte chunk per part
+        uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = half * 8 + 2 * j;  // value index within the sector
+          const uint32_t c0 = uint32_t(sec[s] >> (e * B)) & (L - 1);
+          const uint32_t c1 = uint32_t(sec[s] >> ((e + 1) * B)) & (L - 1);
+          const float2 y = w[s * 8 + half * 4 + j];
+          float r0 = (y.x - nu * slev[c0]) * p.inv_sqrt_d;
+          float r1 = (y.y - nu * slev[c1]) * p.inv_sqrt_d;
+          if (!valid) { r0 = 0.f; r1 = 0.f; }
+          rr = fmaf(r0, r0, fmaf(r1, r1, rr));
+          const __nv_bfloat162 h = __floats2bfloat162_rn(r0, r1);
+          const float2 hf = __bfloat1622float2(h);
+          const float m0 = r0 - hf.x, m1 = r1 - hf.y;  // exact
+          const __nv_bfloat162 md = __floats2bfloat162_rn(m0, m1);
+          const float2 mf = __bfloat1622float2(md);
+          const __nv_bfloat162 l = __floats2bfloat162_rn(m0 - mf.x, m1 - mf.y);  // exact
+          hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+          mid[j] = *reinterpret_cast<const uint32_t*>(&md);
+          lo[j] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        const uint32_t off = cm_offset(tid, s * 2 + half);
+        *reinterpret_cast<uint4*>(smem + Sm::A_OFF + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(smem + Sm::A_OFF + Sm::OPER + off) =
+            make_uint4(mid[0], mid[1], mid[2], mid[3]);
+        *reinterpret_cast<uint4*>(smem + Sm::A_OFF + 2 * Sm::OPER + off) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    const float rho = sqrtf(rr);
+
+    // ---- V = R·Sᵀ on the tensor cores
+    fence_proxy_async_smem();  // A tiles visible to the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t s_base = smem_addr(smem + Sm::S_OFF);
+      uint32_t acc = 0;
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        const uint32_t a_base = smem_addr(smem + Sm::A_OFF + part * Sm::OPER);
+#pragma unroll
+        for (int ks = 0; ks < kQjlD / 16; ++ks) {
+          mma_bf16(tmem, smem_desc(a_base + ks * 2 * kLbo, kLbo, kSbo),
+                   smem_desc(s_base + ks * 2 * kLbo, kLbo, kSbo), acc);
+          acc = 1;
+        }
+      }
+      mma_commit(&mbar);
+      bool ok = false;
+      for (uint32_t i = 0; i < kWaitLimit && !ok; ++i) ok = mbar_try_wait(&mbar, phase);
+      tile_ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    phase ^= 1u;
+    if (!tile_ok) {
+      if (valid) a.rnorm[vec] = __int_as_float(0x7fc00000);  // NaN marks the failure
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+
+    // ---- signs: warp w reads TMEM lanes 32w..32w+31 (this thread's vector)
+    uint32_t bits[4];
+#pragma unroll
+    for (int cchunk = 0; cchunk < 4; ++cchunk) {
+      uint32_t v[32];
+      tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(cchunk * 32), v);
+      tmem_ld_wait();
+      uint32_t b = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) b |= (__uint_as_float(v[j]) > 0.f ? 1u : 0u) << j;
+      bits[cchunk] = b;
+    }
+    if (valid) {
+      reinterpret_cast<uint4*>(a.qbits + vec * (kQjlD / 8))[0] = make_uint4(bits[0], bits[1], bits[2], bits[3]);
+      a.rnorm[vec] = rho;
+    }
+    tc_fence_before();
+    __syncthreads();  // TMEM read and A tiles free before the next tile
+  }
+  cp_async_wait<0>();
+  tc_fence_before();
+  __syncthreads();
+  (void)failed;
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+template <typename T, int B>
+cudaError_t launch_qjl_tb(const QjlArgs& a, cudaStream_t stream) {
+  auto k = a.p.sym ? qjl_encode_kernel<T, B, true> : qjl_encode_kernel<T, B, false>;
+  constexpr int smem = QjlSmem<T>::TOTAL;
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = (a.n + kQjlTile - 1) / kQjlTile;
+  int dev = 0, sms = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = int(ntiles < sms ? ntiles : sms);  // persistent: one CTA per SM
+  k<<<grid, kQjlThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_qjl_t(const QjlArgs& a, cudaStream_t stream) {
+  switch (a.p.bits) {
+    case 1: return launch_qjl_tb<T, 1>(a, stream);
+    case 2: return launch_qjl_tb<T, 2>(a, stream);
+    case 3: return launch_qjl_tb<T, 3>(a, stream);
+    case 4: return launch_qjl_tb<T, 4>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_encode_qjl(const void* x, int dtype, int64_t n, int d, const QuantParams& p,
+                              const uint16_t* S, uint8_t* codes, float* norms, uint8_t* qjl_bits,
+                              float* qjl_rnorm, cudaStream_t stream) {
+  if (d != kQjlD) return cudaErrorInvalidValue;
+  QjlArgs a{x, n, S, codes, norms, qjl_bits, qjl_rnorm, p};
+  switch (dtype) {
+    case RRQ_F16: return launch_qjl_t<__half>(a, stream);
+    case RRQ_BF16: return launch_qjl_t<__nv_bfloat16>(a, stream);
+    case RRQ_F32: return launch_qjl_t<float>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rrq
