@@ -52,7 +52,7 @@ def check_qjl(x, dtype, bits, what, codebook=None):
     P.assert_codes_match(gc, enc.enc.codes, enc.enc.u, tau, what)
     P.assert_norms_close(norms, enc.enc.norm64, d, what)
     assert np.all(np.isfinite(rn)), f"{what}: a tensor-core stage timed out (NaN residual norm)"
-    same = np.all(gc == enc.enc.codes, axis=1) & (norms == enc.enc.norms)
+    same = np.all(gc == enc.enc.codes, axis=1)  # norms may differ by an ulp (r moves ~1e-7·ρ)
     assert same.mean() > 0.99
     rho = enc.rnorm.astype(np.float64)
     rel = np.abs(rn[same] - rho[same]) / np.maximum(rho[same], 1e-30)
@@ -90,13 +90,14 @@ def test_qjl_custom_asymmetric_codebook():
 
 
 def test_qjl_codes_equal_plain_encode():
-    """The fused QJL kernel writes the same codes and norms as the plain encoder."""
+    """The fused QJL kernel writes the same codes as the plain encoder (norms: summation order)."""
     x = to_dev(W.turbo(n=2048).flat(), "bf16")
     s_dev = B.rrq_qjl_matrix(4242, 128, device=DEV)
     c1, n1, _, _ = B.rrq_encode(x, 2, 42, qjl_S=s_dev)
     c2, n2 = B.rrq_encode(x, 2, 42)
     torch.cuda.synchronize()
-    assert torch.equal(c1, c2) and torch.equal(n1, n2)
+    assert torch.equal(c1, c2)
+    assert torch.all((n1 - n2).abs() <= 128 * 2.0 ** -24 * n2)
 
 
 def test_qjl_full_size_sampled():
