@@ -362,11 +362,95 @@ def run_gpu(args):
             "gpu_launches": 2 * args.steps,
             "clocks": clocks,
         }
+        if world == 1 and not args.no_extras:
+            line["kernels"] = extra_kernels(torch, dev, flush, 20, peak)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(x_host)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def time_kernel(torch, stream, flush, fn, reps):
+    """Average device time (ms) of fn() with L2 flushed (untimed) before each call."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for _ in range(3):
+        flush.fill_(3)
+        fn()
+    for e0, e1 in evs:
+        flush.fill_(4)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return sum(e0.elapsed_time(e1) for e0, e1 in evs) / reps
+
+
+def extra_kernels(torch, dev, flush, reps, peak):
+    """Other hot-path kernels on their own workloads (not part of the headline step)."""
+    from random_rotation_kv_b200 import binding as B
+    from random_rotation_kv_b200 import workloads as W
+    stream = torch.cuda.current_stream(dev)
+    mp = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+    except Exception:
+        pass
+    tc_peak = float(mp["bf16_tflops"]) if mp else 1590.0
+    out = {}
+
+    # workload 5: scores of 32 query heads against 131072 tokens x 8 KV heads, 4-bit codes
+    w = W.scores()
+    k = torch.from_numpy(w.flat()).to(dev)
+    codes, norms = B.rrq_encode(k, 4, 42)
+    del k
+    q = torch.from_numpy(w.extra["q"]).to(dev)
+    sc = torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev)
+    ms = time_kernel(torch, stream, flush,
+                     lambda: B.rrq_qk_scores(q, codes, norms, 8, 128, 4, 42, out=sc), reps)
+    nkh = w.x.shape[0] * 8
+    by = nkh * (64 + 4) + 32 * w.x.shape[0] * 4
+    out["qk_scores"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128 b=4",
+                        "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
+                        "frac_of_hbm": by / ms / 1e6 / peak}
+    del codes, norms, sc
+
+    # workload 3: rotate-then-q4_0, 1,048,576 fp16 vectors
+    w = W.attnrot()
+    x = torch.from_numpy(w.flat()).to(dev)
+    n = x.shape[0]
+    blk = torch.empty(n, 72, dtype=torch.uint8, device=dev)
+    xo = torch.empty_like(x)
+    ms_e = time_kernel(torch, stream, flush, lambda: B.rrq_q4_0_rot(x, 42, out=blk), reps)
+    ms_d = time_kernel(torch, stream, flush,
+                       lambda: B.rrq_q4_0_rot_decode(blk, 128, 42, out=xo), reps)
+    by = n * (256 + 72)
+    out["q4_0_rot"] = {"workload": "fp16 [131072 x 8 x 128], rotate + q4_0", "encode_us": 1e3 * ms_e,
+                       "decode_us": 1e3 * ms_d, "encode_gbs": by / ms_e / 1e6,
+                       "decode_gbs": by / ms_d / 1e6, "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
+                       "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
+    del x, blk, xo
+
+    # workload 4: 2-bit codes + QJL sketch, 1,048,576 bf16 vectors (tcgen05 projection)
+    w = W.turbo()
+    x = torch.from_numpy(w.flat()).to(dev).to(torch.bfloat16)
+    n = x.shape[0]
+    S = B.rrq_qjl_matrix(4242, 128, device=dev)
+    cq = torch.empty(n, 32, dtype=torch.uint8, device=dev)
+    nq = torch.empty(n, dtype=torch.float32, device=dev)
+    qb = torch.empty(n, 16, dtype=torch.uint8, device=dev)
+    rq = torch.empty(n, dtype=torch.float32, device=dev)
+    ms = time_kernel(torch, stream, flush, lambda: B.rrq_encode(
+        x, 2, 42, codes=cq, norms=nq, qjl_S=S, qjl_bits=qb, qjl_rnorm=rq), reps)
+    by = n * (256 + 32 + 4 + 16 + 4)
+    flops = n * 3 * 2 * 128 * 128
+    out["encode_qjl"] = {"workload": "bf16 [1048576 x 128], b=2 + QJL (3 bf16 MMAs per tile)",
+                         "us": 1e3 * ms, "gbs": by / ms / 1e6, "frac_of_hbm": by / ms / 1e6 / peak,
+                         "tensor_tflops": flops / ms / 1e9,
+                         "frac_of_tensor_peak": flops / ms / 1e9 / tc_peak}
+    return out
 
 
 def main():
@@ -384,6 +468,8 @@ def main():
                     help="seconds of untimed steps before timing, so clocks reach steady state")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip timing the other kernels (scores, q4_0, QJL) on their workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps, always
     if args.impl == "reference":
