@@ -233,6 +233,27 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------- GPU arm
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's own batch of the KV workload (weak scaling: a new batch per rank)."""
+    return 1002 + rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks: one MAX all-reduce that every rank calls in turn."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -> float:
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return world * units_per_rank * steps / (max_ms / 1e3)
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -254,7 +275,7 @@ def run_gpu(args):
     from random_rotation_kv_b200 import binding as B
     from random_rotation_kv_b200 import workloads as W
 
-    w = W.kv(seed=1002 + rank)  # each rank its own batch
+    w = W.kv(seed=rank_seed(rank))  # each rank its own batch
     x_host = w.flat()
     x = torch.from_numpy(x_host).to(dev)
     codes = torch.empty(N_VEC, D * BITS // 8, dtype=torch.uint8, device=dev)
@@ -296,13 +317,9 @@ def run_gpu(args):
     clocks = ClockSampler.summarize(sampler.stop(), t0, t1) if sampler else None
     enc_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms = sum(enc_ms) + sum(dec_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(enc_ms) + sum(dec_ms), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * N_VEC * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, N_VEC, args.steps, total_ms)
 
     # end to end through the public API: pinned host -> device -> encode -> decode -> host
     x_pin = torch.from_numpy(x_host).pin_memory()
@@ -324,12 +341,8 @@ def run_gpu(args):
         e2e_step()
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * N_VEC * args.e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(world, N_VEC, args.e2e_steps, e2e_ms)
     assert torch.equal(out_pin, out.cpu())
 
     if rank == 0:
