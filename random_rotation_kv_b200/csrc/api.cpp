@@ -70,6 +70,46 @@ const DefaultCodebooks& default_codebooks() {
 }
 
 // Fill the per-call parameter block; returns RRQ_ERR_INVALID for a bad codebook.
+// Cell table of the batch encoder's code search (see rrq::CellTable): the
+// smallest N in {16, 32, 64} whose closed cells [(j − 1/2)/N, (j + 1/2)/N]
+// each hold at most one threshold t_k = fp32(τ_k·A + 1/2); cells = 0 if none.
+// All quantities are exact binary fractions except t_k, which is rounded
+// exactly as stored, so the table decides #{k : s > t_k} with no error.
+void make_cell_table(const float* thr, int nthr, rrq::CellTable* ct) {
+  float tmax = 0.f;
+  for (int k = 0; k < nthr; ++k) tmax = std::fmax(tmax, std::fabs(thr[k]));
+  float R = 1.f;
+  while (!(R > tmax)) R *= 2.f;
+  if (!std::isfinite(R) || R > 1048576.f) {
+    ct->cells = 0;
+    return;
+  }
+  const float A = 0.5f / R;  // exact: R is a power of two
+  float t[rrq::kMaxLevels];
+  for (int k = 0; k < nthr; ++k) t[k] = thr[k] * A + 0.5f;  // τ·A exact; one rounding
+  for (int N = 16; N <= rrq::kMaxCells; N *= 2) {
+    bool ok = true;
+    for (int j = 0; j <= N && ok; ++j) {
+      const double lo = (j - 0.5) / N, hi = (j + 0.5) / N;
+      int inside = 0, below = 0;
+      float tin = 2.f;
+      for (int k = 0; k < nthr; ++k) {
+        if (t[k] < lo) ++below;
+        else if (t[k] <= hi) { ++inside; tin = t[k]; }
+      }
+      if (inside > 1) ok = false;
+      ct->thr[j] = tin;
+      ct->lo[j] = static_cast<uint32_t>(below);
+    }
+    if (ok) {
+      ct->cells = N;
+      ct->a = A;
+      return;
+    }
+  }
+  ct->cells = 0;
+}
+
 int make_params(int bits, const float* codebook, uint64_t seed, int d, rrq::QuantParams* p) {
   std::memset(p, 0, sizeof(*p));
   const int L = 1 << bits;
@@ -88,6 +128,7 @@ int make_params(int bits, const float* codebook, uint64_t seed, int d, rrq::Quan
   p->seed = seed;
   p->inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   p->inv_d = 1.0f / static_cast<float>(d);
+  make_cell_table(p->thr, L - 1, &p->cell);
   return RRQ_OK;
 }
 

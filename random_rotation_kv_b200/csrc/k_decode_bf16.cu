@@ -1,5 +1,5 @@
 // Instantiates the bf16-output decode kernels (split per element type to build in parallel).
-#include "quant_kernels.cuh"
+#include "batch_kernels.cuh"
 
 namespace rrq {
 template cudaError_t decode_typed<__nv_bfloat16>(const uint8_t*, const float*, int64_t, int,

@@ -1,5 +1,5 @@
 // Instantiates the f16 encode kernels (split per element type to build in parallel).
-#include "quant_kernels.cuh"
+#include "batch_kernels.cuh"
 
 namespace rrq {
 template cudaError_t encode_typed<__half>(const __half*, int64_t, int, const QuantParams&, uint8_t*,

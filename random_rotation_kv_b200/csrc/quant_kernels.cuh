@@ -557,9 +557,20 @@ rotate_kernel(const T* __restrict__ x, int64_t n, float* __restrict__ y, uint64_
 template <int C_>
 constexpr int vectors_per_block(int d) { return (kThreads / 32) * (32 / (d / (d < C_ ? d : C_))); }
 
+// One-lane-per-vector encoder for d ≤ 128 and 16-bit inputs (batch_kernels.cuh).
+template <typename T, int D, int B>
+cudaError_t launch_encode_batch(const T* x, int64_t n, const QuantParams& p, uint8_t* codes,
+                                float* norms, cudaStream_t stream);
+
 template <typename T, int D, int B>
 cudaError_t encode_db(const T* x, int64_t n, const QuantParams& p, uint8_t* codes, float* norms,
                       cudaStream_t stream) {
+  if constexpr (Elem<T>::kBytes == 2 && D <= 128) {
+    if (p.cell.cells > 0) {
+      const cudaError_t e = launch_encode_batch<T, D, B>(x, n, p, codes, norms, stream);
+      if (e != cudaErrorNotSupported) return e;
+    }
+  }
   constexpr int vpb = vectors_per_block<EncC<D>::value>(D);
   const int64_t work = (n + vpb - 1) / vpb;
   if (p.sym) {
@@ -598,9 +609,18 @@ cudaError_t encode_typed(const T* x, int64_t n, int d, const QuantParams& p, uin
   return cudaErrorInvalidValue;
 }
 
+// One-lane-per-vector decoder for 4-bit codes and d ≤ 128 (batch_kernels.cuh).
+template <typename T, int D>
+cudaError_t launch_decode_batch(const uint8_t* codes, const float* norms, int64_t n,
+                                const QuantParams& p, T* out, cudaStream_t stream);
+
 template <typename T, int D, int B>
 cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const QuantParams& p,
                       T* out, cudaStream_t stream) {
+  if constexpr (B == 4 && D <= 128) {
+    const cudaError_t e = launch_decode_batch<T, D>(codes, norms, n, p, out, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   using SM = DecodeSmem<T, D, B>;
   constexpr int vpb = SM::WARPS * (32 / (D / DecC<D>::value));
   const int64_t work = (n + vpb - 1) / vpb;

@@ -10,6 +10,23 @@
 namespace rrq {
 
 constexpr int kMaxLevels = 16;  // bits <= 4
+constexpr int kMaxCells = 64;   // cell-table search: at most 64 + 1 cells
+
+// Cell table for the code search of the batch encoder.  The decision value
+// u = y'/ν is mapped to s = sat(u·A + 1/2) ∈ [0, 1] with A = 1/(2R), R a
+// power of two above every |τ_k|; the thresholds in that domain are
+// t_k = fp32(τ_k·A + 1/2).  Cell j (j = 0..N) is the closed interval
+// [(j − 1/2)/N, (j + 1/2)/N], the values s with round(s·N) = j.  `lo[j]` =
+// #{k : t_k < (j − 1/2)/N} and `thr[j]` = the one t_k inside cell j, or 2 when
+// the cell holds none, so code = lo[j] + (s > thr[j]) = #{k : s > t_k}.
+// cells = 0: some cell of every allowed size would hold two thresholds, and
+// the encoder uses its compare/select search instead.
+struct CellTable {
+  int cells;                      // N (16, 32 or 64), or 0
+  float a;                        // A = 1/(2R) (a power of two)
+  float thr[kMaxCells + 1];
+  uint32_t lo[kMaxCells + 1];
+};
 
 // Codebook and rotation constants of one call.  levels: ascending c_0..c_{L-1};
 // thr: τ_k = (c_k + c_{k+1})/2 for k = 0..L-2.  sym: the codebook is exactly
@@ -23,6 +40,7 @@ struct QuantParams {
   int sym;
   float inv_sqrt_d;  // fp32(1/√d)
   float inv_d;       // 1/d (exact)
+  CellTable cell;
 };
 
 // Launchers (one per kernel family); all asynchronous on `stream`.

@@ -137,6 +137,46 @@ def test_symmetric_custom_codebook_fast_path():
     check_encode(x, "bf16", 4, codebook=cb, what="uniform symmetric")
 
 
+def test_close_thresholds_take_the_compare_search():
+    """Two thresholds 0.0005 apart cannot share the cell table; the encoder falls back."""
+    cb = np.array([-1.0, 0.0, 0.001, 1.0], dtype=np.float32)
+    x = W.gaussian(600, 128, "f16", seed=21).flat()
+    check_encode(x, "f16", 2, codebook=cb, what="close thresholds")
+
+
+@pytest.mark.parametrize("scale", [40.0, 1e-3])
+def test_wide_and_narrow_codebooks(scale):
+    """Thresholds far outside [−1, 1] (and far inside) move the cell table's range R."""
+    cb = (ocb.lloyd_max(4) * scale).astype(np.float32)
+    x = W.gaussian(700, 128, "bf16", seed=22).flat()
+    check_encode(x, "bf16", 4, codebook=cb, what=f"codebook x{scale}")
+
+
+@pytest.mark.parametrize("dtype,d,bits", [("f16", 128, 4), ("bf16", 128, 3), ("f16", 64, 2),
+                                          ("bf16", 64, 1)])
+def test_batch_encoder_several_rounds(dtype, d, bits):
+    """Enough batches that every warp of a full grid takes three or more (stage and tile
+    reuse, mbarrier phases), plus a ragged last batch; every row against the oracle."""
+    n = 148 * 8 * 32 * 3 + 19
+    x = W.gaussian(n, d, dtype, seed=23 + bits, scale=1.7).flat()
+    check_encode(x, dtype, bits, what=f"rounds {dtype} d={d} b={bits}")
+
+
+@pytest.mark.parametrize("out_dtype,d", [("f16", 128), ("bf16", 128), ("f32", 128), ("f16", 64)])
+def test_batch_decoder_several_rounds(out_dtype, d):
+    """4-bit decode over enough batches that every warp of a full grid takes several
+    (ring stages, tile reuse, tensor-store clipping of the ragged last batch)."""
+    n = 148 * 10 * 32 * 2 + 13
+    x = W.gaussian(n, d, "f32", seed=31 + d, scale=1.3).flat().astype(np.float64)
+    enc = orc.encode(x, 4, 42)
+    out = B.rrq_decode(torch.from_numpy(enc.packed).to(DEV), torch.from_numpy(enc.norms).to(DEV), d, 4,
+                       42, out_dtype=TORCH_DT[out_dtype])
+    torch.cuda.synchronize()
+    ref = orc.decode(enc.packed, enc.norms, 4, d, 42, out_dtype=out_dtype)
+    P.assert_reconstruction_close(host_f64(out), ref, np.linalg.norm(x, axis=1),
+                                  f"rounds decode {out_dtype} d={d}")
+
+
 def test_edge_cases_zero_ties_extremes():
     d = 128
     x = np.zeros((9, d), dtype=np.float16)
