@@ -332,7 +332,7 @@ template <typename T, int D, int WARPS_, int NS_ = 2, int PF_ = 2> struct DecBat
   static_assert(total() <= 227 * 1024, "shared memory");
 };
 
-template <typename T> constexpr int dec_batch_warps() { return Elem<T>::kBytes == 4 ? 8 : 12; }
+template <typename T> constexpr int dec_batch_warps() { return Elem<T>::kBytes == 4 ? 6 : 12; }
 
 template <typename T, int D, int WARPS_, int NS_ = 2, int PF_ = 2>
 __global__ void __launch_bounds__(WARPS_ * 32, 1)
