@@ -36,7 +36,7 @@ namespace {
 constexpr int kScoreWarpsMax = 16;  // warps per CTA: 16, or 8 / 4 when the tiles do not fit
 constexpr int kScoreTile = 32;   // tokens per warp tile
 constexpr int kScoreStages = 3;  // ring depth (steps)
-constexpr int kScoreU = 2;       // iterations per step
+template <int W> constexpr int score_u() { return W >= 16 ? 2 : 4; }  // iterations per step
 
 struct ScoreArgs {
   const __half* q;
@@ -48,6 +48,51 @@ struct ScoreArgs {
   float scale;
   QuantParams p;
 };
+
+// q' = H·D·q for every query head (fp32, one warp per head), scaled per head
+// by a power of two s with max|q'·s| ≤ 1 (s = 1 for an all-zero head);
+// qf[h·D + i] = q'_{h,i}·s and inv_s[h] = 1/s.
+template <int D>
+__device__ void rotate_queries(const ScoreArgs& a, float* qf, float* inv_s, int warp, int lane,
+                               int nwarps) {
+  constexpr int QC = D / 32;  // values per lane
+  const QuantParams& p = a.p;
+  for (int h = warp; h < a.hq; h += nwarps) {
+    float v[QC];
+#pragma unroll
+    for (int j = 0; j < QC; ++j) {
+      const int i = lane * QC + j;
+      const float x = __half2float(a.q[int64_t(h) * D + i]);
+      v[j] = sign_bit(p.seed, i) ? -x : x;
+    }
+#pragma unroll
+    for (int m = 1; m < QC; m <<= 1)
+#pragma unroll
+      for (int j = 0; j < QC; ++j)
+        if ((j & m) == 0) {
+          const float x0 = v[j], x1 = v[j | m];
+          v[j] = x0 + x1;
+          v[j | m] = x0 - x1;
+        }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const float sg = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+      for (int j = 0; j < QC; ++j) v[j] = fmaf(v[j], sg, __shfl_xor_sync(kFull, v[j], m));
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int j = 0; j < QC; ++j) mx = fmaxf(mx, fabsf(v[j]));
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+    int ex = 0;
+    frexpf(mx, &ex);  // mx = f·2^ex, 0.5 ≤ f < 1
+    const float s = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
+#pragma unroll
+    for (int j = 0; j < QC; ++j) qf[h * D + lane * QC + j] = v[j] * s;
+    if (lane == 0) inv_s[h] = 1.f / s;
+  }
+}
 
 template <int D, int B>
 struct ScoreGeom {
@@ -61,13 +106,13 @@ struct ScoreGeom {
   static constexpr int ROW_WORDS = PRMT ? 64 : 32; // table words per entry
   static constexpr int TABLE_WORDS = (1 << (2 * B)) * ROW_WORDS;
   static constexpr int IT_STRIDE = (IT_BYTES + KPW * 4 + 15) / 16 * 16;  // codes | norms
-  static constexpr int RING_STAGE = kScoreU * IT_STRIDE;
 };
 
 // Shared memory: pair table | q'' (fp16 pairs) | inverse head scales | warp tiles | rings
 template <int D, int B, int W>
 struct ScoreSmem {
   using Gm = ScoreGeom<D, B>;
+  static constexpr int RING_STAGE = score_u<W>() * Gm::IT_STRIDE;
   __host__ __device__ static constexpr size_t table() { return size_t(Gm::TABLE_WORDS) * 4; }
   __host__ __device__ static size_t q(int hq) { return size_t(hq) * D * 2; }
   __host__ __device__ static size_t inv(int hq) { return (size_t(hq) * 4 + 15) / 16 * 16; }
@@ -76,7 +121,7 @@ struct ScoreSmem {
     return (hkv > Gm::KPW ? Gm::KPW : hkv) * (hq / hkv);
   }
   __host__ __device__ static size_t tile(int hq, int hkv) { return size_t(W) * bheads(hq, hkv) * kScoreTile * 4; }
-  __host__ __device__ static constexpr size_t ring() { return size_t(W) * kScoreStages * Gm::RING_STAGE; }
+  __host__ __device__ static constexpr size_t ring() { return size_t(W) * kScoreStages * RING_STAGE; }
   __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }  // fp32 q' (prologue; aliases tiles+rings)
   __host__ __device__ static size_t total(int hq, int hkv) {
     const size_t main = tile(hq, hkv) + ring();
@@ -86,7 +131,7 @@ struct ScoreSmem {
 
 template <int D, int B, int GQ, int W>
 __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a) {
-  constexpr int kScoreWarps = W, kScoreThreads = W * 32;
+  constexpr int kScoreWarps = W, kScoreThreads = W * 32, kScoreU = score_u<W>();
   using Gm = ScoreGeom<D, B>;
   using Sm = ScoreSmem<D, B, W>;
   constexpr int LPK = Gm::LPK, KPW = Gm::KPW, CB = Gm::CB;
@@ -109,46 +154,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a)
     ptab[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
 
-  // ---- rotate the queries: q' = H·D·q (fp32), one warp per head
-  {
-    constexpr int QC = D / 32;  // values per lane
-    for (int h = warp; h < a.hq; h += kScoreWarps) {
-      float v[QC];
-#pragma unroll
-      for (int j = 0; j < QC; ++j) {
-        const int i = lane * QC + j;
-        const float x = __half2float(a.q[int64_t(h) * D + i]);
-        v[j] = sign_bit(p.seed, i) ? -x : x;
-      }
-#pragma unroll
-      for (int m = 1; m < QC; m <<= 1)
-#pragma unroll
-        for (int j = 0; j < QC; ++j)
-          if ((j & m) == 0) {
-            const float x0 = v[j], x1 = v[j | m];
-            v[j] = x0 + x1;
-            v[j | m] = x0 - x1;
-          }
-#pragma unroll
-      for (int m = 1; m < 32; m <<= 1) {
-        const float sg = (lane & m) ? -1.f : 1.f;
-#pragma unroll
-        for (int j = 0; j < QC; ++j) v[j] = fmaf(v[j], sg, __shfl_xor_sync(kFull, v[j], m));
-      }
-      float mx = 0.f;
-#pragma unroll
-      for (int j = 0; j < QC; ++j) mx = fmaxf(mx, fabsf(v[j]));
-#pragma unroll
-      for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-      // power-of-two scale with max·s ≤ 1 (s = 1 for an all-zero head)
-      int ex = 0;
-      frexpf(mx, &ex);  // mx = f·2^ex, 0.5 ≤ f < 1
-      const float s = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
-#pragma unroll
-      for (int j = 0; j < QC; ++j) qf[h * D + lane * QC + j] = v[j] * s;
-      if (lane == 0) inv_s[h] = 1.f / s;
-    }
-  }
+  rotate_queries<D>(a, qf, inv_s, warp, lane, kScoreWarps);
   __syncthreads();
   for (int i = tid; i < a.hq * D / 2; i += kScoreThreads) {
     const __half2 v = __floats2half2_rn(qf[2 * i], qf[2 * i + 1]);
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a)
   uint32_t qr[GQ][16];
   float qscale[GQ];
 
-  uint8_t* ring = rings + warp * kScoreStages * Gm::RING_STAGE;
+  uint8_t* ring = rings + warp * kScoreStages * Sm::RING_STAGE;
   float* tile = tiles + warp * Sm::bheads(a.hq, a.hkv) * kScoreTile;
   const uint32_t* lane_tab = ptab + lane;
   const char* tab_bytes = reinterpret_cast<const char*>(ptab);
@@ -198,7 +204,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a)
       const bool full = i0 + kScoreU <= n_it && iter_row0(i0 + kScoreU - 1) + KPW <= nrows;
 #pragma unroll
       for (int u = 0; u < kScoreU; ++u) {
-        uint8_t* st = ring + stage * Gm::RING_STAGE + u * Gm::IT_STRIDE;
+        uint8_t* st = ring + stage * Sm::RING_STAGE + u * Gm::IT_STRIDE;
         const bool ok_it = i0 + u < n_it;
         const int64_t row0 = ok_it ? iter_row0(i0 + u) : 0;
         if (full) {
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a)
       const int64_t i0 = q * kScoreU;
       cp_async_wait<kScoreStages - 2>();
       __syncwarp();
-      const uint8_t* stb = ring + stage * Gm::RING_STAGE;
+      const uint8_t* stb = ring + stage * Sm::RING_STAGE;
       uint32_t cw[kScoreU][B];
       float nu[kScoreU];
 #pragma unroll
@@ -374,9 +380,15 @@ cudaError_t launch_scores_dbgw(const ScoreArgs& a, cudaStream_t stream) {
 template <int D, int B>
 int score_warps(int hq, int hkv) {
   constexpr size_t kMax = 227 * 1024;
-  if (ScoreSmem<D, B, 16>::total(hq, hkv) <= kMax) return 16;
-  if (ScoreSmem<D, B, 8>::total(hq, hkv) <= kMax) return 8;
-  if (ScoreSmem<D, B, 4>::total(hq, hkv) <= kMax) return 4;
+  constexpr int KPW = ScoreGeom<D, B>::KPW;
+  const int hb = hkv > KPW ? hkv / KPW : 1;
+  const int icp = kScoreTile / (hkv > KPW ? 1 : KPW / hkv);  // iterations per chunk
+  // a step (score_u iterations) must not straddle chunks
+  auto ok = [&](int w) { return icp % (w >= 16 ? 2 : 4) == 0 && w % hb == 0; };
+  if (ok(12) && ScoreSmem<D, B, 12>::total(hq, hkv) <= kMax) return 12;
+  if (ok(16) && ScoreSmem<D, B, 16>::total(hq, hkv) <= kMax) return 16;
+  if (ok(8) && ScoreSmem<D, B, 8>::total(hq, hkv) <= kMax) return 8;
+  if (ok(4) && ScoreSmem<D, B, 4>::total(hq, hkv) <= kMax) return 4;
   return 0;
 }
 
@@ -384,14 +396,232 @@ template <int D, int B, int GQ>
 cudaError_t launch_scores_dbg(const ScoreArgs& a, cudaStream_t stream) {
   switch (score_warps<D, B>(a.hq, a.hkv)) {
     case 16: return launch_scores_dbgw<D, B, GQ, 16>(a, stream);
+    case 12: return launch_scores_dbgw<D, B, GQ, 12>(a, stream);
     case 8: return launch_scores_dbgw<D, B, GQ, 8>(a, stream);
     case 4: return launch_scores_dbgw<D, B, GQ, 4>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
 
+// ------------------------------------------------ one lane per key-head
+// 4-bit codes, d = 64 or 128, GQA group G ∈ {1, 2, 4, 8}.  A work unit is 32
+// consecutive tokens of one kv head g: lane t owns key-head (t0 + t, g) and
+// computes its G scores alone.  The G rotated query heads of g sit in shared
+// memory pair-major ([g][pair][head] half2), so one broadcast load serves
+// every lane; each code byte is one byte-permute table lookup (level pair);
+// G packed fp16 FMAs per pair, folded to fp32 every 16 pairs.  A unit's codes
+// (32 rows of d/2 bytes, hkv rows apart) and norms stream through a per-warp
+// cp.async ring into padded rows; the warps split the units evenly.  Scores
+// leave as 128-byte rows (32 consecutive tokens of one head).
+template <int D, int W>
+struct LaneScoreSmem {
+  static constexpr int CB = D / 2;          // code bytes per key-head
+  static constexpr int RP = CB + 16;        // padded ring row
+  static constexpr int NS = 3;              // ring stages
+  static constexpr int STAGE = 32 * RP + 32 * 4;
+  __host__ __device__ static constexpr size_t table() { return 256 * 64 * 4; }  // entry e at byte e·256 + lane·4
+  __host__ __device__ static size_t q(int hq) { return size_t(hq) * D * 2; }
+  __host__ __device__ static size_t inv(int hq) { return (size_t(hq) * 4 + 15) / 16 * 16; }
+  __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }  // prologue only (aliases the rings)
+  __host__ __device__ static constexpr size_t rings() { return size_t(W) * NS * STAGE; }
+  __host__ __device__ static size_t total(int hq) {
+    return table() + q(hq) + inv(hq) + (qf(hq) > rings() ? qf(hq) : rings());
+  }
+};
+
+template <int G> struct QPairs;  // the G query half2 values of one code pair
+template <> struct QPairs<1> { uint32_t v[1]; };
+template <> struct QPairs<2> { uint32_t v[2]; };
+template <> struct QPairs<4> { uint32_t v[4]; };
+template <> struct QPairs<8> { uint32_t v[8]; };
+template <int G>
+__device__ __forceinline__ QPairs<G> load_qpairs(const uint32_t* q) {
+  QPairs<G> r;
+  if constexpr (G == 1) {
+    r.v[0] = q[0];
+  } else if constexpr (G == 2) {
+    const uint2 t = *reinterpret_cast<const uint2*>(q);
+    r.v[0] = t.x; r.v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < G / 4; ++i) {
+      const uint4 t = reinterpret_cast<const uint4*>(q)[i];
+      r.v[4 * i] = t.x; r.v[4 * i + 1] = t.y; r.v[4 * i + 2] = t.z; r.v[4 * i + 3] = t.w;
+    }
+  }
+  return r;
+}
+
+template <int D, int G, int W>
+__global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreArgs a) {
+  using Sm = LaneScoreSmem<D, W>;
+  constexpr int P = D / 2, CB = Sm::CB, RP = Sm::RP, NS = Sm::NS;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t* ptab = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* qp = reinterpret_cast<uint32_t*>(smem + Sm::table());  // [hkv][P][G] half2
+  float* inv_s = reinterpret_cast<float*>(smem + Sm::table() + Sm::q(a.hq));
+  uint8_t* work = smem + Sm::table() + Sm::q(a.hq) + Sm::inv(a.hq);
+  float* qf = reinterpret_cast<float*>(work);  // prologue only
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const QuantParams& p = a.p;
+
+  for (int i = tid; i < 256 * 64; i += W * 32) {
+    const int e = i >> 6;
+    const __half2 v = __floats2half2_rn(p.levels[e & 15], p.levels[e >> 4]);
+    ptab[i] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  rotate_queries<D>(a, qf, inv_s, warp, lane, W);
+  __syncthreads();
+  for (int i = tid; i < a.hq * P; i += W * 32) {
+    const int h = i / P, pr = i - h * P;  // head h = g·G + j
+    const __half2 v = __floats2half2_rn(qf[h * D + 2 * pr], qf[h * D + 2 * pr + 1]);
+    qp[((h / G) * P + pr) * G + (h % G)] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  __syncthreads();  // qf is dead: its space becomes the rings
+
+  const int lg_hkv = __ffs(a.hkv) - 1;  // hkv is a power of two
+  const int64_t nbt = (a.T + 31) >> 5;
+  const int64_t units = nbt << lg_hkv;
+  const int64_t nw = int64_t(gridDim.x) * W, gw = int64_t(blockIdx.x) * W + warp;
+  const int64_t u_begin = units * gw / nw, u_end = units * (gw + 1) / nw;
+  uint8_t* ring = work + warp * NS * Sm::STAGE;
+  const char* tab_bytes = reinterpret_cast<const char*>(ptab);
+  const uint32_t lane4 = uint32_t(lane) * 4u;
+  const float post = a.scale * p.inv_d;
+
+  // Copy k of a unit moves chunk c = lane % CPR of row t = lane / CPR + k·(32 / CPR):
+  // per-lane offsets are fixed, the unit adds one base.
+  constexpr int CPR = CB / 16;  // 16-byte chunks per row
+  const int lt = lane / CPR, lc = lane % CPR;
+  const int64_t row_bytes = int64_t(a.hkv) * CB;  // global stride between tokens
+  const int64_t lane_src = lt * row_bytes + lc * 16;
+  const uint32_t lane_dst = uint32_t(lt * RP + lc * 16);
+  auto issue = [&](int stage, int64_t u) {
+    if (u < u_end) {
+      const int g = int(u & (a.hkv - 1));
+      const int64_t t0 = (u >> lg_hkv) << 5;
+      const uint8_t* src = a.codes + (t0 * a.hkv + g) * CB + lane_src;
+      const uint32_t dst = smem_addr(ring + stage * Sm::STAGE) + lane_dst;
+      if (t0 + 32 <= a.T) {
+#pragma unroll
+        for (int k = 0; k < CPR; ++k)
+          cp_async16(dst + k * (32 / CPR) * RP, src + k * (32 / CPR) * row_bytes, 16);
+        cp_async4(dst - lane_dst + 32 * RP + lane * 4, a.norms + (t0 + lane) * a.hkv + g, 4);
+      } else {
+#pragma unroll
+        for (int k = 0; k < CPR; ++k) {
+          const bool ok = t0 + lt + k * (32 / CPR) < a.T;
+          cp_async16(dst + k * (32 / CPR) * RP, ok ? src + k * (32 / CPR) * row_bytes : a.codes, ok ? 16 : 0);
+        }
+        const bool ok = t0 + lane < a.T;
+        cp_async4(dst - lane_dst + 32 * RP + lane * 4, a.norms + (ok ? (t0 + lane) * a.hkv + g : 0), ok ? 4 : 0);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int k = 0; k < NS - 1; ++k) issue(k, u_begin + k);
+
+  int stage = 0;
+  for (int64_t u = u_begin; u < u_end; ++u) {
+    cp_async_wait<NS - 2>();
+    __syncwarp();
+    const uint8_t* st = ring + stage * Sm::STAGE;
+    uint32_t cw[CB / 4];
+#pragma unroll
+    for (int i = 0; i < CB / 16; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(st + lane * RP + 16 * i);
+      cw[4 * i] = v.x; cw[4 * i + 1] = v.y; cw[4 * i + 2] = v.z; cw[4 * i + 3] = v.w;
+    }
+    const float nu = reinterpret_cast<const float*>(st + 32 * RP)[lane];
+    __syncwarp();  // every lane has read this stage before it is refilled
+    issue(stage == 0 ? NS - 1 : stage - 1, u + NS - 1);
+    stage = (stage + 1 == NS) ? 0 : stage + 1;
+
+    const int g = int(u & (a.hkv - 1));
+    const int64_t t = ((u >> lg_hkv) << 5) + lane;
+    const uint32_t* qg = qp + g * P * G;
+    float dot[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) dot[j] = 0.f;
+#pragma unroll
+    for (int blk = 0; blk < P; blk += 16) {
+      __half2 acc[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) acc[j] = __float2half2_rn(0.f);
+#pragma unroll
+      for (int pr = blk; pr < blk + 16; ++pr) {
+        const uint32_t off = __byte_perm(cw[pr >> 2], lane4, 0x5504u | ((pr & 3) << 4));
+        const uint32_t cv = *reinterpret_cast<const uint32_t*>(tab_bytes + off);
+        const __half2 c = *reinterpret_cast<const __half2*>(&cv);
+        const QPairs<G> qv = load_qpairs<G>(qg + pr * G);
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+          acc[j] = __hfma2(*reinterpret_cast<const __half2*>(&qv.v[j]), c, acc[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float2 f = __half22float2(acc[j]);
+        dot[j] += f.x + f.y;
+      }
+    }
+    if (t < a.T) {
+      const float sc = nu * post;
+      float* out = a.scores + int64_t(g * G) * a.T + t;
+      const float* is = inv_s + g * G;
+#pragma unroll
+      for (int j = 0; j < G; ++j) out[j * a.T] = dot[j] * sc * is[j];
+    }
+  }
+  cp_async_wait<0>();
+}
+
+template <int D, int G, int W>
+cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
+  auto k = qk_scores_lane_kernel<D, G, W>;
+  const size_t smem = LaneScoreSmem<D, W>::total(a.hq);
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t units = ((a.T + 31) / 32) * a.hkv;
+  const int grid = grid_for(reinterpret_cast<const void*>(k), W * 32, smem, (units + W - 1) / W);
+  k<<<grid, W * 32, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// The lane-per-key-head kernel applies (4-bit codes, d ≤ 128, a power-of-two
+// group ≤ 8, and its shared memory fits with 16 or 8 warps); returns its warps or 0.
+template <int D>
+int lane_score_warps(int bits, int hq, int hkv) {
+  const int group = hq / hkv;
+  if (bits != 4 || (D != 64 && D != 128) || group > 8 || (group & (group - 1))) return 0;
+  if (LaneScoreSmem<D, 16>::total(hq) <= 227 * 1024) return 16;
+  if (LaneScoreSmem<D, 8>::total(hq) <= 227 * 1024) return 8;
+  return 0;
+}
+
+template <int D, int G>
+cudaError_t launch_scores_lane_g(const ScoreArgs& a, cudaStream_t stream) {
+  if (lane_score_warps<D>(4, a.hq, a.hkv) == 16) return launch_scores_lane_w<D, G, 16>(a, stream);
+  return launch_scores_lane_w<D, G, 8>(a, stream);
+}
+
+template <int D>
+cudaError_t launch_scores_lane(const ScoreArgs& a, cudaStream_t stream) {
+  switch (a.group) {
+    case 1: return launch_scores_lane_g<D, 1>(a, stream);
+    case 2: return launch_scores_lane_g<D, 2>(a, stream);
+    case 4: return launch_scores_lane_g<D, 4>(a, stream);
+    case 8: return launch_scores_lane_g<D, 8>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int D, int B>
 cudaError_t launch_scores_db(const ScoreArgs& a, cudaStream_t stream) {
+  if constexpr (B == 4 && D <= 128) {
+    if (lane_score_warps<D>(B, a.hq, a.hkv) > 0) return launch_scores_lane<D>(a, stream);
+  }
   switch (a.group) {
     case 1: return launch_scores_dbg<D, B, 1>(a, stream);
     case 2: return launch_scores_dbg<D, B, 2>(a, stream);
@@ -426,7 +656,11 @@ bool qk_scores_supported(int d, int bits, int hq, int hkv) {
 #undef RRQ_SM
     default: return false;
   }
-  return w > 0 && hb <= w;  // a warp's head block is fixed: head blocks divide the warps
+  (void)hb;
+  if (w > 0) return true;  // a warp's head block is fixed: head blocks divide the warps
+  if (d == 64) return lane_score_warps<64>(bits, hq, hkv) > 0;
+  if (d == 128) return lane_score_warps<128>(bits, hq, hkv) > 0;
+  return false;
 }
 
 cudaError_t launch_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norms,
