@@ -10,8 +10,8 @@
 // whole transform runs in one lane's registers with no shuffles.
 //  * Staging.  One lane per warp moves a whole batch (32 rows, contiguous in
 //    global memory) with TMA tensor copies of 32 × 128-byte boxes, completing
-//    on the stage's mbarrier; two stages per warp, and the batches after those
-//    are prefetched into L2.  The boxes land 128-byte swizzled (tensor_map.h),
+//    on the stage's mbarrier; two stages per warp (an optional L2 prefetch of
+//    later batches measured slower, and is off).  The boxes land 128-byte swizzled (tensor_map.h),
 //    so each lane reads its own row in 16-byte chunks without bank conflicts,
 //    and rows past the end of the array arrive as zeros.  (A bulk copy per
 //    lane would do the same work, but bulk and tensor copies take warp-uniform
@@ -73,13 +73,13 @@ __device__ __forceinline__ void put_code(uint32_t* words, int i, uint32_t c) {
   if (off + B > 32) words[wi + 1] |= c >> (32 - off);
 }
 
-template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 2> struct EncBatch {
+template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 0> struct EncBatch {
   static_assert(D <= 128 && D % 64 == 0 && Elem<T>::kBytes == 2,
                 "batch encoder: d = 64 or 128, 16-bit inputs");
   static constexpr int ROW = D * 2;            // input row bytes
   static constexpr int BOXES = ROW / 128;      // 128-byte boxes per row
   static constexpr int NS = NS_;               // shared-memory stages per warp
-  static constexpr int PF = PF_;               // further batches prefetched into L2
+  static constexpr int PF = PF_;               // further batches prefetched into L2 (measured: none is best)
   static constexpr int CB = D * B / 8;         // code bytes per vector
   static constexpr int STAGE = 32 * ROW;       // BOXES boxes of 32 × 128 bytes (1024-aligned)
   static constexpr int CTILE = 32 * CB;        // one batch of codes, as in global memory
@@ -95,7 +95,7 @@ template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 2> st
   static_assert(total() <= 227 * 1024, "shared memory");
 };
 
-template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 2>
+template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 0>
 __global__ void __launch_bounds__(EncBatch<T, D, B, WARPS_, NS_, PF_>::THREADS, 1)
 encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t* __restrict__ codes,
                     float* __restrict__ norms, const QuantParams p) {
@@ -121,7 +121,9 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
 
   const int64_t nb = (n + 31) >> 5;
   const int64_t tw = int64_t(gridDim.x) * SM::WARPS;
-  const int64_t gw = int64_t(blockIdx.x) * SM::WARPS + warp;
+  // warp-major numbering: consecutive batches go to consecutive SMs, so every
+  // SM gets the same number of batches (±1) whatever the warps per CTA
+  const int64_t gw = int64_t(warp) * gridDim.x + blockIdx.x;
   const uint32_t bar0 = smem_addr(&bars[warp * NS]);
   const uint32_t stage0 = smem_addr(wmem);
   const uint32_t tab_lane = smem_addr(tab) + lane * 8;
@@ -358,7 +360,9 @@ decode_batch_kernel(const uint8_t* __restrict__ codes, const float* __restrict__
 
   const int64_t nb = (n + 31) >> 5;
   const int64_t tw = int64_t(gridDim.x) * SM::WARPS;
-  const int64_t gw = int64_t(blockIdx.x) * SM::WARPS + warp;
+  // warp-major numbering: consecutive batches go to consecutive SMs, so every
+  // SM gets the same number of batches (±1) whatever the warps per CTA
+  const int64_t gw = int64_t(warp) * gridDim.x + blockIdx.x;
   const char* lane_tab = reinterpret_cast<const char*>(tab);
   const uint32_t lane8 = uint32_t(lane) * 8u;
 
