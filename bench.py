@@ -458,8 +458,8 @@ def extra_kernels(torch, dev, flush, reps, peak):
     ms = time_kernel(torch, stream, flush, lambda: B.rrq_encode(
         x, 2, 42, codes=cq, norms=nq, qjl_S=S, qjl_bits=qb, qjl_rnorm=rq), reps)
     by = n * (256 + 32 + 4 + 16 + 4)
-    flops = n * 3 * 2 * 128 * 128
-    out["encode_qjl"] = {"workload": "bf16 [1048576 x 128], b=2 + QJL (3 bf16 MMAs per tile)",
+    flops = n * 2 * 2 * 128 * 128  # two fp16 MMA passes (residual split r_hi + r_lo)
+    out["encode_qjl"] = {"workload": "bf16 [1048576 x 128], b=2 + QJL (2 fp16 MMA passes per tile)",
                          "us": 1e3 * ms, "gbs": by / ms / 1e6, "frac_of_hbm": by / ms / 1e6 / peak,
                          "tensor_tflops": flops / ms / 1e9,
                          "frac_of_tensor_peak": flops / ms / 1e9 / tc_peak}
