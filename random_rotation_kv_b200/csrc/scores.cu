@@ -419,13 +419,36 @@ struct LaneScoreSmem {
   static constexpr int RP = CB + 16;        // padded ring row
   static constexpr int NS = 3;              // ring stages
   static constexpr int STAGE = 32 * RP + 32 * 4;
+  static constexpr int RING = NS * STAGE;   // per warp
   __host__ __device__ static constexpr size_t table() { return 256 * 64 * 4; }  // entry e at byte e·256 + lane·4
   __host__ __device__ static size_t q(int hq) { return size_t(hq) * D * 2; }
   __host__ __device__ static size_t inv(int hq) { return (size_t(hq) * 4 + 15) / 16 * 16; }
-  __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }  // prologue only (aliases the rings)
-  __host__ __device__ static constexpr size_t rings() { return size_t(W) * NS * STAGE; }
+  __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }  // prologue only (aliases rings)
+  __host__ __device__ static constexpr size_t rings() { return size_t(W) * RING; }
+  // Plain layout: [table | q'' | inv | rings (qf aliased)].
   __host__ __device__ static size_t total(int hq) {
     return table() + q(hq) + inv(hq) + (qf(hq) > rings() ? qf(hq) : rings());
+  }
+  // Folded layout, for a dynamic base at shared address kFoldBase: the table
+  // sits at shared address 0x10000 so that the byte-permuted offset
+  // 0x10000 | byte·256 | lane·4 is the load address itself.  Below it: q'',
+  // inv and the first `front` rings; above it: the other rings (qf aliased).
+  static constexpr uint32_t kFoldBase = 0x400, kFoldTable = 0x10000;
+  __host__ __device__ static size_t fold_front_rings(int hq) {
+    const size_t start = (q(hq) + inv(hq) + 15) / 16 * 16;
+    const size_t room = kFoldTable - kFoldBase;
+    const size_t n = start < room ? (room - start) / RING : 0;
+    return n < size_t(W) ? n : size_t(W);
+  }
+  __host__ __device__ static size_t fold_back(int hq) { return kFoldTable - kFoldBase + table(); }
+  __host__ __device__ static size_t fold_ring(int hq, int w) {
+    const size_t nf = fold_front_rings(hq);
+    return size_t(w) < nf ? (q(hq) + inv(hq) + 15) / 16 * 16 + size_t(w) * RING
+                          : fold_back(hq) + (size_t(w) - nf) * RING;
+  }
+  __host__ __device__ static size_t fold_total(int hq) {
+    const size_t back = (size_t(W) - fold_front_rings(hq)) * RING;
+    return fold_back(hq) + (qf(hq) > back ? qf(hq) : back);
   }
 };
 
@@ -452,18 +475,38 @@ __device__ __forceinline__ QPairs<G> load_qpairs(const uint32_t* q) {
   return r;
 }
 
-template <int D, int G, int W>
+template <int D, int G, int W, bool FOLD>
 __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreArgs a) {
   using Sm = LaneScoreSmem<D, W>;
   constexpr int P = D / 2, CB = Sm::CB, RP = Sm::RP, NS = Sm::NS;
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* ptab = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* qp = reinterpret_cast<uint32_t*>(smem + Sm::table());  // [hkv][P][G] half2
-  float* inv_s = reinterpret_cast<float*>(smem + Sm::table() + Sm::q(a.hq));
-  uint8_t* work = smem + Sm::table() + Sm::q(a.hq) + Sm::inv(a.hq);
-  float* qf = reinterpret_cast<float*>(work);  // prologue only
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const QuantParams& p = a.p;
+  uint32_t* ptab;
+  uint32_t* qp;
+  float* inv_s;
+  float* qf;
+  uint8_t* ring;
+  if constexpr (FOLD) {
+    if (smem_addr(smem) != Sm::kFoldBase) {
+      // not the layout the launch assumed: mark every score as invalid
+      for (int64_t i = int64_t(blockIdx.x) * W * 32 + tid; i < int64_t(a.hq) * a.T; i += int64_t(gridDim.x) * W * 32)
+        a.scores[i] = __int_as_float(0x7fc00000);
+      return;
+    }
+    qp = reinterpret_cast<uint32_t*>(smem);
+    inv_s = reinterpret_cast<float*>(smem + Sm::q(a.hq));
+    ptab = reinterpret_cast<uint32_t*>(smem + (Sm::kFoldTable - Sm::kFoldBase));
+    qf = reinterpret_cast<float*>(smem + Sm::fold_back(a.hq));
+    ring = smem + Sm::fold_ring(a.hq, warp);
+  } else {
+    ptab = reinterpret_cast<uint32_t*>(smem);
+    qp = reinterpret_cast<uint32_t*>(smem + Sm::table());  // [hkv][P][G] half2
+    inv_s = reinterpret_cast<float*>(smem + Sm::table() + Sm::q(a.hq));
+    uint8_t* work = smem + Sm::table() + Sm::q(a.hq) + Sm::inv(a.hq);
+    qf = reinterpret_cast<float*>(work);  // prologue only
+    ring = work + warp * NS * Sm::STAGE;
+  }
 
   for (int i = tid; i < 256 * 64; i += W * 32) {
     const int e = i >> 6;
@@ -484,9 +527,9 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
   const int64_t units = nbt << lg_hkv;
   const int64_t nw = int64_t(gridDim.x) * W, gw = int64_t(blockIdx.x) * W + warp;
   const int64_t u_begin = units * gw / nw, u_end = units * (gw + 1) / nw;
-  uint8_t* ring = work + warp * NS * Sm::STAGE;
   const char* tab_bytes = reinterpret_cast<const char*>(ptab);
-  const uint32_t lane4 = uint32_t(lane) * 4u;
+  // FOLD: byte 2 of the permute's second operand is the table's address bit 16
+  const uint32_t lane4 = uint32_t(lane) * 4u | (FOLD ? Sm::kFoldTable : 0u);
   const float post = a.scale * p.inv_d;
 
   // Copy k of a unit moves chunk c = lane % CPR of row t = lane / CPR + k·(32 / CPR):
@@ -551,8 +594,14 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
       for (int j = 0; j < G; ++j) acc[j] = __float2half2_rn(0.f);
 #pragma unroll
       for (int pr = blk; pr < blk + 16; ++pr) {
-        const uint32_t off = __byte_perm(cw[pr >> 2], lane4, 0x5504u | ((pr & 3) << 4));
-        const uint32_t cv = *reinterpret_cast<const uint32_t*>(tab_bytes + off);
+        uint32_t cv;
+        if constexpr (FOLD) {  // address 0x10000 | byte·256 | lane·4
+          const uint32_t addr = __byte_perm(cw[pr >> 2], lane4, 0x7604u | ((pr & 3) << 4));
+          asm("ld.shared.b32 %0, [%1];" : "=r"(cv) : "r"(addr));
+        } else {
+          const uint32_t off = __byte_perm(cw[pr >> 2], lane4, 0x5504u | ((pr & 3) << 4));
+          cv = *reinterpret_cast<const uint32_t*>(tab_bytes + off);
+        }
         const __half2 c = *reinterpret_cast<const __half2*>(&cv);
         const QPairs<G> qv = load_qpairs<G>(qg + pr * G);
 #pragma unroll
@@ -578,8 +627,13 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
 
 template <int D, int G, int W>
 cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
-  auto k = qk_scores_lane_kernel<D, G, W>;
-  const size_t smem = LaneScoreSmem<D, W>::total(a.hq);
+  using Sm = LaneScoreSmem<D, W>;
+  int dev = 0, reserved = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  const bool fold = reserved == int(Sm::kFoldBase) && Sm::fold_total(a.hq) <= 227 * 1024;
+  auto k = fold ? qk_scores_lane_kernel<D, G, W, true> : qk_scores_lane_kernel<D, G, W, false>;
+  const size_t smem = fold ? Sm::fold_total(a.hq) : Sm::total(a.hq);
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
