@@ -44,6 +44,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["random_rotation_kv_b200/csrc/rrq_device.cuh",
                   "random_rotation_kv_b200/csrc/quant_kernels.cuh",
+                  "random_rotation_kv_b200/csrc/batch_kernels.cuh",
+                  "random_rotation_kv_b200/csrc/tensor_map.h",
                   "random_rotation_kv_b200/csrc/rrq_params.h"]
 
 
@@ -349,10 +351,10 @@ def run_gpu(args):
         peak, peak_kind = peaks()
         enc_avg = sum(enc_ms) / len(enc_ms)
         dec_avg = sum(dec_ms) / len(dec_ms)
-        dom, dom_ms, dom_bytes = (("encode", enc_avg, BYTES_PER_VEC_ENC) if enc_avg >= dec_avg
-                                  else ("decode", dec_avg, BYTES_PER_VEC_DEC))
+        dom, dom_ms, dom_bytes = (("encode_batch_kernel", enc_avg, BYTES_PER_VEC_ENC) if enc_avg >= dec_avg
+                                  else ("decode_batch_kernel", dec_avg, BYTES_PER_VEC_DEC))
         achieved = dom_bytes * N_VEC / (dom_ms / 1e3) / 1e9
-        traffic = recorded_traffic(dom + "_kernel")
+        traffic = recorded_traffic(dom)
         step_gbs = (BYTES_PER_VEC_ENC + BYTES_PER_VEC_DEC) * N_VEC / (ms_per_step / 1e3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -360,7 +362,7 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": workload_config({"parallelism": f"dp{world} (independent batches)"}),
-            "roofline": {"bound": "hbm", "kernel": dom + "_kernel", "achieved": achieved,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved,
                          "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_source": f"{peak_kind} copy bandwidth",
                          "traffic": traffic,
