@@ -21,7 +21,7 @@ import math
 
 import numpy as np
 
-from .rrq import as_f64
+from .rrq import as_f64, pack_codes, rotate
 
 
 def marginal_density(x, d: int) -> np.ndarray:
@@ -53,3 +53,30 @@ def drive_decode(rotation: np.ndarray, x, scale) -> np.ndarray:
     rx = x @ p.T
     sgn = np.where(rx >= 0, 1.0, -1.0)
     return np.asarray(scale, dtype=np.float64)[..., None] * (sgn @ p)
+
+
+class DriveEncoded:
+    """signs [N, d] int64 (1 where (Πx)_i > 0), packed [N, d/8] u8 (LSB first),
+    scale [N] float64 (S), stored [N] float32 (fp32(S·√d), the per-vector value
+    that the rrq 1-bit decoder and score path read as their norm)."""
+
+    def __init__(self, signs, packed, scale, stored, rx):
+        self.signs, self.packed, self.scale, self.stored, self.rx = signs, packed, scale, stored, rx
+
+
+def drive_encode(x, seed: int, unbiased: bool) -> DriveEncoded:
+    """DRIVE's one-bit encoder ("History", DRIVE bullet): sign(Πx) and the scale S.
+
+    S = ‖Πx‖₁/d (biased, MSE-optimal) or S = ‖x‖₂²/‖Πx‖₁ (unbiased).  A code is
+    1 when (Πx)_i > 0 (strict, the rule of the b-bit encoder with τ = 0), so
+    with the codebook {−1, +1} and the stored value S·√d the b-bit decoder
+    returns S·Πᵀ·sign(Πx), the mean decoder of "Three decoders, one rotation".
+    """
+    x = as_f64(x)
+    d = x.shape[-1]
+    rx = rotate(x, seed)
+    s = drive_scale_unbiased(x, rx) if unbiased else drive_scale_biased(rx)
+    s = np.where(np.sum(np.abs(rx), axis=-1) > 0, s, 0.0)
+    signs = (rx > 0).astype(np.int64)
+    stored = (s * math.sqrt(d)).astype(np.float32)
+    return DriveEncoded(signs, pack_codes(signs, 1), s, stored, rx)

@@ -359,6 +359,26 @@ def test_drive_unbiased_scale(d):
     assert np.linalg.norm(mean - x) < 0.05 * np.linalg.norm(x)
 
 
+@pytest.mark.parametrize("unbiased", [False, True])
+def test_drive_encode_through_the_one_bit_decoder(unbiased):
+    """drive_encode + the b-bit decoder (codebook {−1, +1}, stored S·√d) is the DRIVE
+    mean decoder S·Πᵀ·sign(Πx); the scores path gives S·⟨Πq, sign(Πx)⟩."""
+    rg = np.random.default_rng(7)
+    x = rg.standard_normal((40, 16)) * rg.uniform(0.5, 3, size=(40, 1))
+    enc = sphere.drive_encode(x, 11, unbiased)
+    p = hadamard.rotation_matrix(11, 16)
+    want = sphere.drive_decode(p, x, enc.scale)
+    pm = np.array([-1.0, 1.0])
+    got = rrq.decode_exact(enc.packed, enc.stored.astype(np.float64), 1, 16, 11, levels=pm)
+    assert np.allclose(got, want, rtol=1e-6, atol=1e-12)
+    q = rg.standard_normal((2, 16))
+    sc = rrq.scores(q, enc.packed, enc.stored.astype(np.float64), 40, 1, 16, 1, 11, levels=pm)
+    want_s = enc.scale[None, :] * ((q @ p.T) @ (2.0 * enc.signs.T - 1.0))
+    assert np.allclose(sc, want_s, rtol=1e-6, atol=1e-12)
+    if unbiased:
+        assert np.allclose(np.sum(got * x, 1), np.sum(x * x, 1), rtol=1e-6)  # <x̂, x> = ‖x‖²
+
+
 # ------------------------------------------------------------------------- q4_0
 def _q4_inputs(name):
     x = np.zeros(32)
