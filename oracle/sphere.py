@@ -46,13 +46,21 @@ def drive_scale_unbiased(x, rx) -> np.ndarray:
     return np.sum(x * x, axis=-1) / np.sum(np.abs(rx), axis=-1)
 
 
+def drive_mean_decode(rotation: np.ndarray, bits, scale) -> np.ndarray:
+    """x̂ = S·Πᵀ·(2·bit − 1) for rows of sign bits ("Three decoders, one
+    rotation", mean decoder)."""
+    p = as_f64(rotation)
+    sgn = 2.0 * np.asarray(bits, dtype=np.float64) - 1.0
+    return np.asarray(scale, dtype=np.float64)[..., None] * (sgn @ p)
+
+
 def drive_decode(rotation: np.ndarray, x, scale) -> np.ndarray:
-    """x̂ = S·Πᵀ·sign(Πx) for rows of x; sign(0) taken as +1."""
+    """x̂ = S·Πᵀ·sign(Πx) for rows of x.  sign(0) is taken as −1: the page
+    leaves it open, and −1 is the b-bit encoder's rule with τ = 0 (a value on
+    a threshold takes the lower code)."""
     x = as_f64(x)
     p = as_f64(rotation)
-    rx = x @ p.T
-    sgn = np.where(rx >= 0, 1.0, -1.0)
-    return np.asarray(scale, dtype=np.float64)[..., None] * (sgn @ p)
+    return drive_mean_decode(p, (x @ p.T) > 0, scale)
 
 
 class DriveEncoded:

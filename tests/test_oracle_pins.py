@@ -379,6 +379,26 @@ def test_drive_encode_through_the_one_bit_decoder(unbiased):
         assert np.allclose(np.sum(got * x, 1), np.sum(x * x, 1), rtol=1e-6)  # <x̂, x> = ‖x‖²
 
 
+def test_drive_zero_coordinates_take_the_minus_one_sign():
+    """A coordinate with (Πx)_i = 0 exactly gets bit 0 (−1) in the encoder and
+    in the mean decoder alike.  d = 16 makes Π's entries ±1/4 (exact), so
+    x = Πᵀ·(4, 0, …, 0) rotates back to exactly (4, 0, …, 0)."""
+    p = hadamard.rotation_matrix(5, 16)
+    y = np.zeros(16)
+    y[0] = 4.0
+    x = (p.T @ y)[None]
+    assert np.array_equal(rrq.rotate(x, 5)[0], y)
+    for unbiased in (False, True):
+        enc = sphere.drive_encode(x, 5, unbiased)
+        assert enc.signs[0].tolist() == [1] + [0] * 15
+        assert enc.scale[0] == (4.0 / 16 if not unbiased else 16.0 / 4.0)
+        want = sphere.drive_decode(p, x, enc.scale)
+        got = rrq.decode_exact(enc.packed, enc.stored.astype(np.float64), 1, 16, 5,
+                               levels=np.array([-1.0, 1.0]))
+        assert np.allclose(got, want, rtol=1e-6, atol=1e-12)
+        assert np.allclose(want[0], enc.scale[0] * (p.T @ np.where(y > 0, 1.0, -1.0)))
+
+
 # ------------------------------------------------------------------------- q4_0
 def _q4_inputs(name):
     x = np.zeros(32)
