@@ -446,7 +446,24 @@ def extra_kernels(torch, dev, flush, reps, peak):
                        "decode_us": 1e3 * ms_d, "encode_gbs": by / ms_e / 1e6,
                        "decode_gbs": by / ms_d / 1e6, "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
                        "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
-    del x, blk, xo
+    del blk, xo
+
+    # DRIVE one-bit encode (unbiased scale) of the same vectors, and the
+    # one-bit decode back to fp16
+    dc = torch.empty(n, 16, dtype=torch.uint8, device=dev)
+    ds = torch.empty(n, dtype=torch.float32, device=dev)
+    xo = torch.empty_like(x)
+    ms_e = time_kernel(torch, stream, flush,
+                       lambda: B.rrq_drive_encode(x, 42, True, codes=dc, scales=ds), reps)
+    ms_d = time_kernel(torch, stream, flush, lambda: B.rrq_decode(
+        dc, ds, 128, 1, 42, codebook=[-1.0, 1.0], out=xo), reps)
+    by = n * (256 + 16 + 4)
+    out["drive_1bit"] = {"workload": "fp16 [131072 x 8 x 128], DRIVE sign + unbiased scale",
+                         "encode_us": 1e3 * ms_e, "decode_us": 1e3 * ms_d,
+                         "encode_gbs": by / ms_e / 1e6, "decode_gbs": by / ms_d / 1e6,
+                         "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
+                         "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
+    del x, dc, ds, xo
 
     # workload 4: 2-bit codes + QJL sketch, 1,048,576 bf16 vectors (tcgen05 projection)
     w = W.turbo()

@@ -124,8 +124,10 @@ int rrq_rotate(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int 
  *     r = Πx − ŷ,  ŷ = (ν/√d)·c[code]  (the decoder's rotated-domain value),
  *     qjl_bits bit i = [ (S·r)_i > 0 ],  qjl_rnorm = ‖r‖₂,
  * with S the d×d matrix at qjl_S (bf16, row-major, see rrq_qjl_matrix).
- * The product S·r runs on the tensor cores (tcgen05) with r split into three
- * bf16 parts, so the signs are those of an fp32-accurate product.
+ * The product S·r runs on the tensor cores (tcgen05): for fp32 x with r split
+ * exactly into three bf16 parts (an fp32-accurate product); for 16-bit x with
+ * r scaled by a power of two and split into two fp16 parts and S rounded to
+ * fp16 (the sign of an output can differ only where |(S·r)_i| < 1e-5·‖r‖₂).
  *   x          [n × d] of x_dtype
  *   codes      [n × d·bits/8] bytes (output)
  *   norms      [n] float (output)
@@ -152,6 +154,27 @@ int rrq_encode(const void* x, int x_dtype, int64_t n, int d, int bits, uint64_t 
  */
 int rrq_decode(const uint8_t* codes, const float* norms, int64_t n, int d, int bits,
                uint64_t seed, const float* codebook, void* out, int out_dtype, void* stream);
+
+/*
+ * rrq_drive_encode — DRIVE's one-bit encoder.
+ * "Random-rotation quantization" page, "History", DRIVE bullet (one bit per
+ * coordinate, sign(R(x)), plus one scale; ‖R(x)‖₁/d is the biased, MSE-optimal
+ * choice and ‖x‖₂²/‖R(x)‖₁ the unbiased one), and "Three decoders, one
+ * rotation", mean decoder x̂ = S·Πᵀ·sign(Πx).  For each vector x:
+ *     bit_i = [ (Πx)_i > 0 ]   (0 decodes to −1, 1 to +1),
+ *     S = ‖Πx‖₁/d (unbiased = 0) or ‖x‖₂²/‖Πx‖₁ (unbiased = 1; 0 when x = 0),
+ *     scales = fp32(S·√d).
+ * Bits are packed as rrq_encode's one-bit codes, and the stored value is what
+ * rrq_decode and rrq_qk_scores read as the norm, so rrq_decode(bits = 1,
+ * codebook {−1, +1}) returns S·Πᵀ·sign(Πx) and rrq_qk_scores with the same
+ * codebook returns scale·S·⟨Πq, sign(Πx)⟩.
+ *   x       [n × d] of x_dtype
+ *   codes   [n × d/8] bytes (output);  scales [n] float (output)
+ * Errors: RRQ_ERR_INVALID (d, dtype, unbiased not 0/1, null or misaligned
+ * pointer), RRQ_ERR_CUDA.
+ */
+int rrq_drive_encode(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int unbiased,
+                     uint8_t* codes, float* scales, void* stream);
 
 /*
  * rrq_qk_scores — decode-time attention scores against a quantised K cache,

@@ -83,7 +83,8 @@ def drive_encode(x, seed: int, unbiased: bool) -> DriveEncoded:
     x = as_f64(x)
     d = x.shape[-1]
     rx = rotate(x, seed)
-    s = drive_scale_unbiased(x, rx) if unbiased else drive_scale_biased(rx)
+    with np.errstate(invalid="ignore", divide="ignore"):  # x = 0: S = 0 below
+        s = drive_scale_unbiased(x, rx) if unbiased else drive_scale_biased(rx)
     s = np.where(np.sum(np.abs(rx), axis=-1) > 0, s, 0.0)
     signs = (rx > 0).astype(np.int64)
     stored = (s * math.sqrt(d)).astype(np.float32)

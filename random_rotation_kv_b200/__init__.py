@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     lib,
     rrq_codebook,
     rrq_decode,
+    rrq_drive_encode,
     rrq_encode,
     rrq_format_version,
     rrq_q4_0_rot,

@@ -35,6 +35,7 @@ SIGNATURES = {
     "rrq_rotate": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
     "rrq_encode": (_int, [_vp, _int, _c_i64, _int, _int, _c_u64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rrq_decode": (_int, [_vp, _vp, _c_i64, _int, _int, _c_u64, _vp, _vp, _int, _vp]),
+    "rrq_drive_encode": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp, _vp]),
     "rrq_qk_scores": (_int, [_vp, _int, _vp, _vp, _c_i64, _int, _int, _int, _c_u64, _vp,
                              ctypes.c_float, _vp, _vp]),
     "rrq_q4_0_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
@@ -167,6 +168,30 @@ def rrq_encode(x: torch.Tensor, bits: int, seed: int, codebook=None, codes=None,
     if qjl_S is not None:
         return codes, norms, qjl_bits, qjl_rnorm
     return codes, norms
+
+
+def rrq_drive_encode(x: torch.Tensor, seed: int, unbiased: bool, codes=None, scales=None):
+    """DRIVE one-bit encode of rows of x [..., d].
+
+    Returns (codes uint8 [..., d/8], scales float32 [...]); scales hold S·√d,
+    which rrq_decode / rrq_qk_scores with bits=1 and codebook [-1, 1] read as
+    the norm.
+    """
+    _dev_tensor(x, "x", DTYPE_CODE)
+    d = x.shape[-1]
+    n = x.numel() // d if d else 0
+    lead = x.shape[:-1]
+    if codes is None:
+        codes = torch.empty(*lead, d // 8, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead, dtype=torch.float32, device=x.device)
+    _dev_tensor(codes, "codes", (torch.uint8,))
+    _dev_tensor(scales, "scales", (torch.float32,))
+    if codes.numel() != n * (d // 8) or scales.numel() != n:
+        raise ValueError("codes / scales have the wrong size")
+    _check(lib().rrq_drive_encode(_ptr(x), DTYPE_CODE[x.dtype], n, d, seed, int(bool(unbiased)),
+                                  _ptr(codes), _ptr(scales), _stream(x)), "rrq_drive_encode")
+    return codes, scales
 
 
 def rrq_decode(codes: torch.Tensor, norms: torch.Tensor, d: int, bits: int, seed: int,

@@ -195,6 +195,19 @@ int rrq_decode(const uint8_t* codes, const float* norms, int64_t n, int d, int b
   return status_of(rrq::launch_decode(codes, norms, n, d, p, out, out_dtype, as_stream(stream)));
 }
 
+int rrq_drive_encode(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int unbiased,
+                     uint8_t* codes, float* scales, void* stream) {
+  if (n < 0 || !d_ok(d) || !dtype_ok(x_dtype) || (unbiased != 0 && unbiased != 1))
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 32) || !arr_ok(codes, n, 32) || !arr_ok(scales, n, 4)) return RRQ_ERR_INVALID;
+  static const float kSigns[2] = {-1.0f, 1.0f};
+  rrq::QuantParams p;
+  if (make_params(1, kSigns, seed, d, &p) != RRQ_OK) return RRQ_ERR_INVALID;
+  p.norm_mode = 1 + unbiased;
+  if (n == 0) return RRQ_OK;
+  return status_of(rrq::launch_encode(x, x_dtype, n, d, p, codes, scales, as_stream(stream)));
+}
+
 int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norms, int64_t T,
                   int hkv, int d, int bits, uint64_t seed, const float* codebook, float scale,
                   float* scores, void* stream) {

@@ -95,7 +95,9 @@ template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 0> st
   static_assert(total() <= 227 * 1024, "shared memory");
 };
 
-template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 0>
+// DRV: DRIVE's one-bit encoder (B = 1, ±1 codebook): code = (y' > 0) and the
+// stored value is the scale that p.norm_mode selects (QuantParams::norm_mode).
+template <typename T, int D, int B, int WARPS_ = 8, int NS_ = 2, int PF_ = 0, bool DRV = false>
 __global__ void __launch_bounds__(EncBatch<T, D, B, WARPS_, NS_, PF_>::THREADS, 1)
 encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t* __restrict__ codes,
                     float* __restrict__ norms, const QuantParams p) {
@@ -195,7 +197,8 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
     for (int k = 0; k < P; ++k) acc[k & 3] = fma2(w[k], w[k], acc[k & 3]);
     const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
     const float2 a4 = add2(a01, a23);
-    const float nu = sqrtf(0.5f * (a4.x + a4.y));
+    const float ss = 0.5f * (a4.x + a4.y);  // ‖x‖₂² (the butterfly doubled it)
+    const float nu = sqrtf(ss);
 
 #pragma unroll
     for (int mm = 1; mm < P; mm <<= 1) {
@@ -209,12 +212,26 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
       }
     }
 
-    const float sc = nu > 0.f ? __fdiv_rn(A, nu) : 0.f;  // s = sat(y'·A/ν + 1/2)
     uint32_t words[NW];
 #pragma unroll
     for (int i = 0; i < NW; ++i) words[i] = 0u;
+    float stored = nu;
+    if constexpr (DRV) {
+      static_assert(B == 1, "DRIVE codes are one bit");
+      float2 l1[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int k = 0; k < P; ++k) {
+      for (int k = 0; k < P; ++k) {
+        l1[k & 1] = add2(l1[k & 1], make_float2(fabsf(w[k].x), fabsf(w[k].y)));
+        put_code<1>(words, 2 * k, w[k].x > 0.f ? 1u : 0u);
+        put_code<1>(words, 2 * k + 1, w[k].y > 0.f ? 1u : 0u);
+      }
+      const float2 l = add2(l1[0], l1[1]);
+      const float s1 = l.x + l.y;  // ‖y'‖₁ = √d·‖Πx‖₁
+      stored = p.norm_mode == 1 ? s1 * p.inv_d : (s1 > 0.f ? __fdiv_rn(ss * float(D), s1) : 0.f);
+    }
+    const float sc = nu > 0.f ? __fdiv_rn(A, nu) : 0.f;  // s = sat(y'·A/ν + 1/2)
+#pragma unroll
+    for (int k = 0; k < (DRV ? 0 : P); ++k) {
       const float sx = __saturatef(fmaf(w[k].x, sc, 0.5f));
       const float sy = __saturatef(fmaf(w[k].y, sc, 0.5f));
       const float2 f = fma2(make_float2(sx, sy), make_float2(Nf, Nf), make_float2(8388608.f, 8388608.f));
@@ -248,7 +265,7 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
         for (int i = 0; i < CB / 8; ++i)
           reinterpret_cast<uint2*>(dst)[i] = make_uint2(words[2 * i], words[2 * i + 1]);
       }
-      norms[v0 + lane] = nu;
+      norms[v0 + lane] = stored;
     }
     if (bulk) {
       fence_proxy_async_smem();
@@ -282,6 +299,9 @@ cudaError_t launch_encode_batch(const T* x, int64_t n, const QuantParams& p, uin
   CUtensorMap xmap;
   if (!row_tensor_map(&xmap, x, n, D, 2, 32)) return cudaErrorNotSupported;
   auto k = encode_batch_kernel<T, D, B>;
+  if constexpr (B == 1) {
+    if (p.norm_mode != 0) k = encode_batch_kernel<T, D, 1, 8, 2, 0, true>;
+  }
   constexpr size_t smem = SM::total();
   const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

@@ -287,8 +287,20 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
     float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < P; ++k) ss2 = fma2(w[k], w[k], ss2);
-    const float nu = sqrtf(group_sum<G>(ss2.x + ss2.y));
+    const float ss = group_sum<G>(ss2.x + ss2.y);  // ‖x‖₂²
+    const float nu = sqrtf(ss);
     fwht2<D, C>(w, h);
+    float stored = nu;
+    if constexpr (B == 1) {
+      if (p.norm_mode != 0) {  // DRIVE scale × √d (QuantParams::norm_mode)
+        float2 l1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < P; ++k) l1 = add2(l1, make_float2(fabsf(w[k].x), fabsf(w[k].y)));
+        const float s1 = group_sum<G>(l1.x + l1.y);  // ‖y'‖₁
+        stored = p.norm_mode == 1 ? s1 * p.inv_d
+                                  : (s1 > 0.f ? __fdiv_rn(ss * float(D), s1) : 0.f);
+      }
+    }
     const float ns = nu > 0.f ? nu : 1.f;  // ν = 0: y' = 0, u = 0 against the plain thresholds
     uint8_t* crow = codes + vec * CB;
 
@@ -337,7 +349,7 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
       for (int s = 0; s < SEC; ++s)
         if (valid) store_sector_codes<B>(crow, Lay::sector(s, h), sec[s]);
     }
-    if (valid && h == 0) norms[vec] = nu;
+    if (valid && h == 0) norms[vec] = stored;
   }
 }
 
@@ -566,7 +578,7 @@ template <typename T, int D, int B>
 cudaError_t encode_db(const T* x, int64_t n, const QuantParams& p, uint8_t* codes, float* norms,
                       cudaStream_t stream) {
   if constexpr (Elem<T>::kBytes == 2 && D <= 128) {
-    if (p.cell.cells > 0) {
+    if (p.cell.cells > 0 || p.norm_mode != 0) {  // DRIVE codes need no table
       const cudaError_t e = launch_encode_batch<T, D, B>(x, n, p, codes, norms, stream);
       if (e != cudaErrorNotSupported) return e;
     }

@@ -40,6 +40,12 @@ struct QuantParams {
   int sym;
   float inv_sqrt_d;  // fp32(1/√d)
   float inv_d;       // 1/d (exact)
+  // Per-vector value the encoders store: 0 = ν = ‖x‖₂; with a ±1 one-bit
+  // codebook, DRIVE's scale S times √d ("History", DRIVE bullet): 1 = biased,
+  // S = ‖Πx‖₁/d (stored ‖y'‖₁/d); 2 = unbiased, S = ‖x‖₂²/‖Πx‖₁ (stored
+  // ‖x‖₂²·d/‖y'‖₁, 0 when y' = 0).  The decoder and score paths read the stored
+  // value as ν, so x̂ = S·Πᵀ·sign(Πx) and ⟨q, x̂⟩ = S·⟨Πq, sign(Πx)⟩.
+  int norm_mode;
   CellTable cell;
 };
 

@@ -118,3 +118,8 @@ def test_other_entry_points_validate():
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 96, 0, 1, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 128, 0, 3, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot_decode(P, 4, 128, 0, 1, P, 5, None) == B.RRQ_ERR_INVALID
+    # DRIVE: unbiased must be 0/1, d a supported size, scales 4-byte aligned
+    assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 128, 0, 2, P, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 100, 0, 0, P, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 128, 0, 1, P, P_MIS, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_drive_encode(ctypes.c_void_p(None), B.RRQ_F16, 0, 128, 0, 1, P, P, None) == B.RRQ_OK
