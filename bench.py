@@ -5,11 +5,16 @@ Workload (one step): the fp16 K cache [32768 tokens × 8 KV heads × 128]
 (262,144 vectors; 2 % outlier channels ×15, log-normal per-token scale),
 encoded at 4 bits (randomized Hadamard rotation + N(0,1) Lloyd–Max codes +
 fp32 norm) and decoded back to fp16, through the C ABI (rrq_encode,
-rrq_decode).  Inputs are resident in HBM before timing starts; the 126 MB L2 is
-flushed (a 256 MiB write) before every timed kernel, and only the kernels are
-inside the CUDA-event pairs.  Multi-GPU (torchrun): every rank processes its
-own batch of the same size (weak scaling, no collective on the data path);
-the time is the maximum over ranks.
+rrq_decode).  Inputs are resident in HBM before timing starts.  The timed
+steps run back to back between one pair of CUDA events, over 4 rotating
+batches (4 × 84.9 MB per kernel kind, larger than the 126 MB L2): step k
+encodes batch k mod 4 and decodes the codes of batch (k + 2) mod 4, written two
+steps earlier and evicted from L2 since.  The per-kernel figures (roofline)
+come from encode-only and decode-only loops timed the same way; a flushed
+single-launch figure (256 MiB write before each launch) is reported beside
+them.  Multi-GPU (torchrun): every rank processes its own batches of the same
+size (weak scaling, no collective on the data path); the time is the maximum
+over ranks.
 
 ``--impl reference`` times the CPU oracle (the plain fp64 restatement under
 ``oracle/``) on a bounded sample of the same workload instead.
@@ -41,6 +46,7 @@ N_VEC = TOKENS * HEADS
 BYTES_PER_VEC_ENC = D * 2 + D * BITS // 8 + 4   # read fp16, write codes + fp32 norm
 BYTES_PER_VEC_DEC = D * BITS // 8 + 4 + D * 2   # read codes + norm, write fp16
 NOMINAL_HBM_GBS = 8000.0
+ROT = 4  # rotating batches: 4 x 84.9 MB per kernel kind, larger than the 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["random_rotation_kv_b200/csrc/rrq_device.cuh",
                   "random_rotation_kv_b200/csrc/quant_kernels.cuh",
@@ -54,7 +60,8 @@ def workload_config(extra=None):
                        "encode+decode",
            "vectors_per_gpu": N_VEC, "d": D, "bits": BITS, "io_dtype": "f16",
            "rotation_seed": 42,
-           "l2": "flushed by a 256 MiB write before every timed kernel"}
+           "l2": "inputs larger than L2: 4 rotating batches; step k encodes batch k mod 4 and "
+                 "decodes the codes of batch (k+2) mod 4, written two steps earlier"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -277,51 +284,57 @@ def run_gpu(args):
     from random_rotation_kv_b200 import binding as B
     from random_rotation_kv_b200 import workloads as W
 
-    w = W.kv(seed=rank_seed(rank))  # each rank its own batch
-    x_host = w.flat()
-    x = torch.from_numpy(x_host).to(dev)
-    codes = torch.empty(N_VEC, D * BITS // 8, dtype=torch.uint8, device=dev)
-    norms = torch.empty(N_VEC, dtype=torch.float32, device=dev)
-    out = torch.empty(N_VEC, D, dtype=torch.float16, device=dev)
+    # ROT batches per rank, each its own seeded KV batch (weak scaling: new data per rank)
+    x_host = W.kv(seed=rank_seed(rank)).flat()
+    xs = [torch.from_numpy(x_host).to(dev)]
+    for j in range(1, ROT):
+        xs.append(torch.from_numpy(W.kv(seed=rank_seed(rank) + 1000 * j).flat()).to(dev))
+    codes = [torch.empty(N_VEC, D * BITS // 8, dtype=torch.uint8, device=dev) for _ in range(ROT)]
+    norms = [torch.empty(N_VEC, dtype=torch.float32, device=dev) for _ in range(ROT)]
+    outs = [torch.empty(N_VEC, D, dtype=torch.float16, device=dev) for _ in range(ROT)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(evs=None):
-        flush.fill_(1)
-        if evs:
-            evs[0].record(stream)
-        B.rrq_encode(x, BITS, 42, codes=codes, norms=norms)
-        if evs:
-            evs[1].record(stream)
-        flush.fill_(2)
-        if evs:
-            evs[2].record(stream)
-        B.rrq_decode(codes, norms, D, BITS, 42, out_dtype=torch.float16, out=out)
-        if evs:
-            evs[3].record(stream)
+    def enc(j):
+        B.rrq_encode(xs[j], BITS, 42, codes=codes[j], norms=norms[j])
 
-    for _ in range(args.warmup):
-        step()
+    def dec(j, o):
+        B.rrq_decode(codes[j], norms[j], D, BITS, 42, out_dtype=torch.float16, out=outs[o])
+
+    def step(k):
+        enc(k % ROT)
+        dec((k + 2) % ROT, k % ROT)  # codes written two steps earlier
+
+    for j in range(ROT):  # every batch has codes before the first decode reads them
+        enc(j)
+    for k in range(args.warmup):
+        step(k)
     # keep the clocks in steady state before the timed region
     t_end = time.time() + args.settle_s
+    k = 0
     while time.time() < t_end:
-        step()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        step(k)
+        k += 1
     sampler = ClockSampler(gpu_id_for(torch, dev)) if rank == 0 and not args.no_clocks else None
     if sampler:
         sampler.start()
     barrier()
     t0 = time.time()
-    for k in range(args.steps):
-        step(evs[k])
+    step_ms = time_loop(torch, stream, step, args.steps)
     barrier()
     t1 = time.time()
     clocks = ClockSampler.summarize(sampler.stop(), t0, t1) if sampler else None
-    enc_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms = max_over_ranks(sum(enc_ms) + sum(dec_ms), world, dev)
+    total_ms = max_over_ranks(step_ms * args.steps, world, dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(world, N_VEC, args.steps, total_ms)
+    # per-kernel average launch durations, the same way (rotating batches, back to back)
+    enc_avg = max_over_ranks(time_loop(torch, stream, lambda k: enc(k % ROT), args.steps), world, dev)
+    dec_avg = max_over_ranks(time_loop(torch, stream, lambda k: dec((k + 2) % ROT, k % ROT),
+                                       args.steps), world, dev)
+    # single launches with L2 flushed before each (carry the fixed launch + event cost)
+    enc_iso = time_kernel(torch, stream, flush, lambda: enc(0), 20)
+    dec_iso = time_kernel(torch, stream, flush, lambda: dec(0, 0), 20)
+    x, out, codes0, norms0 = xs[0], outs[0], codes[0], norms[0]
 
     # end to end through the public API: pinned host -> device -> encode -> decode -> host
     x_pin = torch.from_numpy(x_host).pin_memory()
@@ -330,8 +343,8 @@ def run_gpu(args):
 
     def e2e_step():
         x_e2e.copy_(x_pin, non_blocking=True)
-        B.rrq_encode(x_e2e, BITS, 42, codes=codes, norms=norms)
-        B.rrq_decode(codes, norms, D, BITS, 42, out_dtype=torch.float16, out=out)
+        B.rrq_encode(x_e2e, BITS, 42, codes=codes0, norms=norms0)
+        B.rrq_decode(codes0, norms0, D, BITS, 42, out_dtype=torch.float16, out=out)
         out_pin.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -349,8 +362,6 @@ def run_gpu(args):
 
     if rank == 0:
         peak, peak_kind = peaks()
-        enc_avg = sum(enc_ms) / len(enc_ms)
-        dec_avg = sum(dec_ms) / len(dec_ms)
         dom, dom_ms, dom_bytes = (("encode_batch_kernel", enc_avg, BYTES_PER_VEC_ENC) if enc_avg >= dec_avg
                                   else ("decode_batch_kernel", dec_avg, BYTES_PER_VEC_DEC))
         achieved = dom_bytes * N_VEC / (dom_ms / 1e3) / 1e9
@@ -368,6 +379,8 @@ def run_gpu(args):
                          "traffic": traffic,
                          "algorithmic_bytes_per_launch": dom_bytes * N_VEC},
             "hbm": {"encode_us": 1e3 * enc_avg, "decode_us": 1e3 * dec_avg,
+                    "isolated_flushed_encode_us": 1e3 * enc_iso,
+                    "isolated_flushed_decode_us": 1e3 * dec_iso,
                     "encode_gbs": BYTES_PER_VEC_ENC * N_VEC / (enc_avg / 1e3) / 1e9,
                     "decode_gbs": BYTES_PER_VEC_DEC * N_VEC / (dec_avg / 1e3) / 1e9,
                     "step_gbs": step_gbs, "step_frac_of_measured": step_gbs / peak,
@@ -378,12 +391,27 @@ def run_gpu(args):
             "clocks": clocks,
         }
         if world == 1 and not args.no_extras:
-            line["kernels"] = extra_kernels(torch, dev, flush, 20, peak)
+            line["kernels"] = extra_kernels(torch, dev, flush, 50, peak)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(x_host)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def time_loop(torch, stream, fn, steps):
+    """Average device time (ms) of fn(k), k = 0..steps-1, run back to back between
+    one pair of CUDA events on `stream`, after 3 untimed calls."""
+    for k in range(3):
+        fn(k)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for k in range(steps):
+        fn(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
 
 
 def time_kernel(torch, stream, flush, fn, reps):
@@ -403,7 +431,9 @@ def time_kernel(torch, stream, flush, fn, reps):
 
 
 def extra_kernels(torch, dev, flush, reps, peak):
-    """Other hot-path kernels on their own workloads (not part of the headline step)."""
+    """Other hot-path kernels on their own workloads (not part of the headline step),
+    each timed as `reps` back-to-back launches whose inputs exceed L2 (the 1M-vector
+    inputs are 268 MB; the scores rotate over 3 copies of its 71 MB cache)."""
     from random_rotation_kv_b200 import binding as B
     from random_rotation_kv_b200 import workloads as W
     stream = torch.cuda.current_stream(dev)
@@ -422,15 +452,18 @@ def extra_kernels(torch, dev, flush, reps, peak):
     codes, norms = B.rrq_encode(k, 4, 42)
     del k
     q = torch.from_numpy(w.extra["q"]).to(dev)
-    sc = torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev)
-    ms = time_kernel(torch, stream, flush,
-                     lambda: B.rrq_qk_scores(q, codes, norms, 8, 128, 4, 42, out=sc), reps)
+    cs = [codes] + [codes.clone() for _ in range(2)]
+    ns = [norms] + [norms.clone() for _ in range(2)]
+    scs = [torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev) for _ in range(3)]
+    ms = time_loop(torch, stream,
+                   lambda k: B.rrq_qk_scores(q, cs[k % 3], ns[k % 3], 8, 128, 4, 42, out=scs[k % 3]),
+                   reps)
     nkh = w.x.shape[0] * 8
     by = nkh * (64 + 4) + 32 * w.x.shape[0] * 4
     out["qk_scores"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128 b=4",
                         "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
                         "frac_of_hbm": by / ms / 1e6 / peak}
-    del codes, norms, sc
+    del codes, norms, cs, ns, scs
 
     # workload 3: rotate-then-q4_0, 1,048,576 fp16 vectors
     w = W.attnrot()
@@ -438,9 +471,8 @@ def extra_kernels(torch, dev, flush, reps, peak):
     n = x.shape[0]
     blk = torch.empty(n, 72, dtype=torch.uint8, device=dev)
     xo = torch.empty_like(x)
-    ms_e = time_kernel(torch, stream, flush, lambda: B.rrq_q4_0_rot(x, 42, out=blk), reps)
-    ms_d = time_kernel(torch, stream, flush,
-                       lambda: B.rrq_q4_0_rot_decode(blk, 128, 42, out=xo), reps)
+    ms_e = time_loop(torch, stream, lambda k: B.rrq_q4_0_rot(x, 42, out=blk), reps)
+    ms_d = time_loop(torch, stream, lambda k: B.rrq_q4_0_rot_decode(blk, 128, 42, out=xo), reps)
     by = n * (256 + 72)
     out["q4_0_rot"] = {"workload": "fp16 [131072 x 8 x 128], rotate + q4_0", "encode_us": 1e3 * ms_e,
                        "decode_us": 1e3 * ms_d, "encode_gbs": by / ms_e / 1e6,
@@ -453,9 +485,9 @@ def extra_kernels(torch, dev, flush, reps, peak):
     dc = torch.empty(n, 16, dtype=torch.uint8, device=dev)
     ds = torch.empty(n, dtype=torch.float32, device=dev)
     xo = torch.empty_like(x)
-    ms_e = time_kernel(torch, stream, flush,
-                       lambda: B.rrq_drive_encode(x, 42, True, codes=dc, scales=ds), reps)
-    ms_d = time_kernel(torch, stream, flush, lambda: B.rrq_decode(
+    ms_e = time_loop(torch, stream,
+                     lambda k: B.rrq_drive_encode(x, 42, True, codes=dc, scales=ds), reps)
+    ms_d = time_loop(torch, stream, lambda k: B.rrq_decode(
         dc, ds, 128, 1, 42, codebook=[-1.0, 1.0], out=xo), reps)
     by = n * (256 + 16 + 4)
     out["drive_1bit"] = {"workload": "fp16 [131072 x 8 x 128], DRIVE sign + unbiased scale",
@@ -474,7 +506,7 @@ def extra_kernels(torch, dev, flush, reps, peak):
     nq = torch.empty(n, dtype=torch.float32, device=dev)
     qb = torch.empty(n, 16, dtype=torch.uint8, device=dev)
     rq = torch.empty(n, dtype=torch.float32, device=dev)
-    ms = time_kernel(torch, stream, flush, lambda: B.rrq_encode(
+    ms = time_loop(torch, stream, lambda k: B.rrq_encode(
         x, 2, 42, codes=cq, norms=nq, qjl_S=S, qjl_bits=qb, qjl_rnorm=rq), reps)
     by = n * (256 + 32 + 4 + 16 + 4)
     flops = n * 2 * 2 * 128 * 128  # two fp16 MMA passes (residual split r_hi + r_lo)

@@ -103,6 +103,7 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
                     float* __restrict__ norms, const QuantParams p) {
   using SM = EncBatch<T, D, B, WARPS_, NS_, PF_>;
   constexpr int P = D / 2, CB = SM::CB, NW = (CB + 3) / 4, NS = SM::NS;
+  pdl_release();
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = dsm_raw + ((1024u - (smem_addr(dsm_raw) & 1023u)) & 1023u);
   float2* tab = reinterpret_cast<float2*>(dsm);
@@ -120,6 +121,7 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
     fence_mbarrier_init();
   }
   __syncthreads();
+  pdl_wait();  // the shared tables are built: from here on, global memory
 
   const int64_t nb = (n + 31) >> 5;
   const int64_t tw = int64_t(gridDim.x) * SM::WARPS;
@@ -309,8 +311,7 @@ cudaError_t launch_encode_batch(const T* x, int64_t n, const QuantParams& p, uin
   const int64_t batches = (n + 31) / 32;
   const int grid = grid_for(reinterpret_cast<const void*>(k), SM::THREADS, smem,
                             (batches + SM::WARPS - 1) / SM::WARPS);
-  k<<<grid, SM::THREADS, smem, stream>>>(xmap, n, codes, norms, p);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, SM::THREADS, smem, stream, xmap, n, codes, norms, p);
 }
 
 }  // namespace rrq
@@ -362,6 +363,7 @@ decode_batch_kernel(const uint8_t* __restrict__ codes, const float* __restrict__
                     const __grid_constant__ CUtensorMap omap, const QuantParams p) {
   using SM = DecBatch<T, D, WARPS_, NS_, PF_>;
   constexpr int P = D / 2, CB = SM::CB, NS = SM::NS;
+  pdl_release();
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = dsm_raw + ((1024u - (smem_addr(dsm_raw) & 1023u)) & 1023u);
   float2* tab = reinterpret_cast<float2*>(dsm);
@@ -377,6 +379,7 @@ decode_batch_kernel(const uint8_t* __restrict__ codes, const float* __restrict__
   }
   build_sign_mask<T, D>(smask, p.seed);
   __syncthreads();
+  pdl_wait();  // the shared tables are built: from here on, global memory
 
   const int64_t nb = (n + 31) >> 5;
   const int64_t tw = int64_t(gridDim.x) * SM::WARPS;
@@ -497,8 +500,7 @@ cudaError_t launch_decode_batch(const uint8_t* codes, const float* norms, int64_
   const int64_t batches = (n + 31) / 32;
   const int grid = grid_for(reinterpret_cast<const void*>(k), SM::THREADS, smem,
                             (batches + SM::WARPS - 1) / SM::WARPS);
-  k<<<grid, SM::THREADS, smem, stream>>>(codes, norms, n, omap, p);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, SM::THREADS, smem, stream, codes, norms, n, omap, p);
 }
 
 }  // namespace rrq

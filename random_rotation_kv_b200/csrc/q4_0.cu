@@ -96,6 +96,7 @@ template <typename T, int D, bool ROT>
 __global__ void __launch_bounds__(kQThreads) q4_encode_kernel(const T* __restrict__ x, int64_t n,
                                                               uint8_t* __restrict__ blocks,
                                                               uint64_t seed, float inv_sqrt_d) {
+  pdl_release();
   using Lay = typename QLay<D>::L;
   constexpr int C = QLay<D>::C;
   constexpr int G = Lay::G, P = Lay::P, SEC = Lay::SEC, VPW = Lay::VPW;
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kQThreads) q4_encode_kernel(const T* __restric
   __shared__ __align__(16) uint8_t stage[kQThreads / 32][kWarpBytes];
   if constexpr (ROT) build_sign_mask<T, D>(smask, seed);
   __syncthreads();
+  pdl_wait();  // from here on, global memory
 
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   uint8_t* buf = stage[threadIdx.x >> 5];
@@ -177,6 +179,7 @@ template <typename T, int D, bool ROT>
 __global__ void __launch_bounds__(kQThreads) q4_decode_kernel(const uint8_t* __restrict__ blocks,
                                                               int64_t n, T* __restrict__ out,
                                                               uint64_t seed, float inv_sqrt_d) {
+  pdl_release();
   using Lay = typename QLay<D>::L;
   constexpr int C = QLay<D>::C;
   constexpr int G = Lay::G, P = Lay::P, SEC = Lay::SEC, VPW = Lay::VPW;
@@ -185,6 +188,7 @@ __global__ void __launch_bounds__(kQThreads) q4_decode_kernel(const uint8_t* __r
   __shared__ __align__(16) uint8_t stage[kQThreads / 32][kWarpBytes];
   if constexpr (ROT) build_sign_mask<T, D>(smask, seed);
   __syncthreads();
+  pdl_wait();  // from here on, global memory
 
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   uint8_t* buf = stage[threadIdx.x >> 5];
@@ -228,11 +232,13 @@ cudaError_t q4_enc_d(const T* x, int64_t n, uint64_t seed, int rotate, float isd
   if (rotate) {
     auto k = q4_encode_kernel<T, D, true>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kQThreads, 0, work);
-    k<<<grid, kQThreads, 0, stream>>>(x, n, blocks, seed, isd);
+    const cudaError_t e = launch_pdl(k, grid, kQThreads, 0, stream, x, n, blocks, seed, isd);
+    if (e != cudaSuccess) return e;
   } else {
     auto k = q4_encode_kernel<T, D, false>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kQThreads, 0, work);
-    k<<<grid, kQThreads, 0, stream>>>(x, n, blocks, seed, isd);
+    const cudaError_t e = launch_pdl(k, grid, kQThreads, 0, stream, x, n, blocks, seed, isd);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -245,11 +251,13 @@ cudaError_t q4_dec_d(const uint8_t* blocks, int64_t n, uint64_t seed, int rotate
   if (rotate) {
     auto k = q4_decode_kernel<T, D, true>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kQThreads, 0, work);
-    k<<<grid, kQThreads, 0, stream>>>(blocks, n, out, seed, isd);
+    const cudaError_t e = launch_pdl(k, grid, kQThreads, 0, stream, blocks, n, out, seed, isd);
+    if (e != cudaSuccess) return e;
   } else {
     auto k = q4_decode_kernel<T, D, false>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kQThreads, 0, work);
-    k<<<grid, kQThreads, 0, stream>>>(blocks, n, out, seed, isd);
+    const cudaError_t e = launch_pdl(k, grid, kQThreads, 0, stream, blocks, n, out, seed, isd);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -141,6 +141,8 @@ struct QjlArgs {
 
 template <typename T, int B, bool SYM>
 __global__ void __launch_bounds__(kQjlThreads, 1) qjl_encode_kernel(const QjlArgs a) {
+  pdl_release();
+  pdl_wait();  // the prologue reads S: wait for the previous kernel first
   using Sm = QjlSmem<T>;
   constexpr int D = kQjlD, P = D / 2, SEC = D / 16, L = 1 << B, CB = D * B / 8;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -405,6 +407,8 @@ struct Qjl2Smem {
 
 template <typename T, int B>
 __global__ void __launch_bounds__(kQ2Threads, 1) qjl_batch_kernel(const __grid_constant__ QjlArgs a) {
+  pdl_release();
+  pdl_wait();  // the prologue reads S: wait for the previous kernel first
   using Sm = Qjl2Smem;
   constexpr int D = kQjlD, P = D / 2, CB = D * B / 8, NW = (CB + 3) / 4;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -661,8 +665,7 @@ cudaError_t launch_qjl_tb(const QjlArgs& a, cudaStream_t stream) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       const int64_t want = (ntiles + kQ2Groups - 1) / kQ2Groups;
       const int grid = int(want < sms ? want : sms);  // persistent: one CTA per SM
-      k2<<<grid, kQ2Threads, smem2, stream>>>(a2);
-      return cudaGetLastError();
+      return launch_pdl(k2, grid, kQ2Threads, smem2, stream, a2);
     }
   }
   auto k = a.p.sym ? qjl_encode_kernel<T, B, true> : qjl_encode_kernel<T, B, false>;
@@ -675,8 +678,7 @@ cudaError_t launch_qjl_tb(const QjlArgs& a, cudaStream_t stream) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = int(ntiles < sms ? ntiles : sms);  // persistent: one CTA per SM
-  k<<<grid, kQjlThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, kQjlThreads, smem, stream, a);
 }
 
 template <typename T>

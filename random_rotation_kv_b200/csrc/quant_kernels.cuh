@@ -262,6 +262,7 @@ template <typename T, int D, int B, bool SYM>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
 encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
               float* __restrict__ norms, const QuantParams p) {
+  pdl_release();
   constexpr int C = EncC<D>::value;
   using Lay = Layout<D, C>;
   constexpr int G = Lay::G, P = Lay::P, SEC = Lay::SEC, VPW = Lay::VPW;
@@ -270,6 +271,7 @@ encode_kernel(const T* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
   __shared__ __align__(16) uint32_t smask[mask_words<T, D>()];
   build_sign_mask<T, D>(smask, p.seed);
   __syncthreads();
+  pdl_wait();  // from here on, global memory
 
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   const int64_t gwarp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -401,6 +403,7 @@ template <typename T, int D, int B>
 __global__ void __launch_bounds__(DecodeSmem<T, D, B>::THREADS, 1)
 decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms, int64_t n,
               T* __restrict__ out, const QuantParams p) {
+  pdl_release();
   constexpr int C = DecC<D>::value;
   using Lay = Layout<D, C>;
   using SM = DecodeSmem<T, D, B>;
@@ -426,6 +429,7 @@ decode_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ norms
     }
   }
   __syncthreads();
+  pdl_wait();  // from here on, global memory
 
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   const int64_t gwarp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -540,6 +544,7 @@ template <typename T, int D, bool INV>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
 rotate_kernel(const T* __restrict__ x, int64_t n, float* __restrict__ y, uint64_t seed,
               float inv_sqrt_d) {
+  pdl_release();
   constexpr int C = EncC<D>::value;
   using Lay = Layout<D, C>;
   constexpr int G = Lay::G, P = Lay::P, VPW = Lay::VPW;
@@ -548,6 +553,7 @@ rotate_kernel(const T* __restrict__ x, int64_t n, float* __restrict__ y, uint64_
   if constexpr (!INV) build_sign_mask<T, D>(smask_in, seed);
   else build_sign_mask<float, D>(smask_out, seed);
   __syncthreads();
+  pdl_wait();  // from here on, global memory
 
   const int lane = threadIdx.x & 31, h = lane & (G - 1), vsub = lane / G;
   const int64_t gwarp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -588,11 +594,13 @@ cudaError_t encode_db(const T* x, int64_t n, const QuantParams& p, uint8_t* code
   if (p.sym) {
     auto k = encode_kernel<T, D, B, true>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
-    k<<<grid, kThreads, 0, stream>>>(x, n, codes, norms, p);
+    const cudaError_t e = launch_pdl(k, grid, kThreads, 0, stream, x, n, codes, norms, p);
+    if (e != cudaSuccess) return e;
   } else {
     auto k = encode_kernel<T, D, B, false>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
-    k<<<grid, kThreads, 0, stream>>>(x, n, codes, norms, p);
+    const cudaError_t e = launch_pdl(k, grid, kThreads, 0, stream, x, n, codes, norms, p);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -644,7 +652,8 @@ cudaError_t decode_db(const uint8_t* codes, const float* norms, int64_t n, const
     if (e != cudaSuccess) return e;
   }
   const int grid = grid_for(reinterpret_cast<const void*>(k), SM::THREADS, smem, work);
-  k<<<grid, SM::THREADS, smem, stream>>>(codes, norms, n, out, p);
+  const cudaError_t e = launch_pdl(k, grid, SM::THREADS, smem, stream, codes, norms, n, out, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -680,11 +689,13 @@ cudaError_t rotate_d(const T* x, int64_t n, uint64_t seed, int inverse, float in
   if (inverse) {
     auto k = rotate_kernel<T, D, true>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
-    k<<<grid, kThreads, 0, stream>>>(x, n, y, seed, inv_sqrt_d);
+    const cudaError_t e = launch_pdl(k, grid, kThreads, 0, stream, x, n, y, seed, inv_sqrt_d);
+    if (e != cudaSuccess) return e;
   } else {
     auto k = rotate_kernel<T, D, false>;
     const int grid = grid_for(reinterpret_cast<const void*>(k), kThreads, 0, work);
-    k<<<grid, kThreads, 0, stream>>>(x, n, y, seed, inv_sqrt_d);
+    const cudaError_t e = launch_pdl(k, grid, kThreads, 0, stream, x, n, y, seed, inv_sqrt_d);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

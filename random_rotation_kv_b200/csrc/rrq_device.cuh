@@ -24,9 +24,43 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "rrq_params.h"
 
 namespace rrq {
+
+// ------------------------------------------------ programmatic dependent launch
+// Every rrq kernel is launched with programmatic stream serialization allowed
+// (`launch_pdl`), so when the kernel before it in the stream lets its
+// dependents start, this kernel's CTAs launch early and build their
+// shared-memory tables while that kernel drains.  `pdl_wait()` blocks until
+// the previous kernel has completed and its memory is visible; every kernel
+// calls it before its first global-memory access (read or write).  Launched
+// without a dependency, it returns at once.  `pdl_release()` lets the next
+// kernel in the stream launch; its CTAs still wait for this kernel's
+// completion before touching memory.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kernel` on `stream` with programmatic stream serialization allowed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr unsigned kFull = 0xffffffffu;
 

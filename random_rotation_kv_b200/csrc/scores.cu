@@ -131,6 +131,7 @@ struct ScoreSmem {
 
 template <int D, int B, int GQ, int W>
 __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a) {
+  pdl_release();
   constexpr int kScoreWarps = W, kScoreThreads = W * 32, kScoreU = score_u<W>();
   using Gm = ScoreGeom<D, B>;
   using Sm = ScoreSmem<D, B, W>;
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_kernel(const ScoreArgs a)
     ptab[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
 
+  pdl_wait();  // from here on, global memory
   rotate_queries<D>(a, qf, inv_s, warp, lane, kScoreWarps);
   __syncthreads();
   for (int i = tid; i < a.hq * D / 2; i += kScoreThreads) {
@@ -372,8 +374,7 @@ cudaError_t launch_scores_dbgw(const ScoreArgs& a, cudaStream_t stream) {
   const int64_t ntiles = (a.T + kScoreTile - 1) / kScoreTile;
   const int hb = a.hkv > ScoreGeom<D, B>::KPW ? a.hkv / ScoreGeom<D, B>::KPW : 1;
   const int grid = grid_for(reinterpret_cast<const void*>(k), W * 32, smem, (ntiles * hb + W - 1) / W);
-  k<<<grid, W * 32, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, W * 32, smem, stream, a);
 }
 
 // The largest warp count whose tiles and rings fit in one CTA's shared memory.
@@ -477,6 +478,7 @@ __device__ __forceinline__ QPairs<G> load_qpairs(const uint32_t* q) {
 
 template <int D, int G, int W, bool FOLD>
 __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreArgs a) {
+  pdl_release();
   using Sm = LaneScoreSmem<D, W>;
   constexpr int P = D / 2, CB = Sm::CB, RP = Sm::RP, NS = Sm::NS;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -490,6 +492,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
   if constexpr (FOLD) {
     if (smem_addr(smem) != Sm::kFoldBase) {
       // not the layout the launch assumed: mark every score as invalid
+      pdl_wait();
       for (int64_t i = int64_t(blockIdx.x) * W * 32 + tid; i < int64_t(a.hq) * a.T; i += int64_t(gridDim.x) * W * 32)
         a.scores[i] = __int_as_float(0x7fc00000);
       return;
@@ -513,6 +516,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
     const __half2 v = __floats2half2_rn(p.levels[e & 15], p.levels[e >> 4]);
     ptab[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
+  pdl_wait();  // from here on, global memory
   rotate_queries<D>(a, qf, inv_s, warp, lane, W);
   __syncthreads();
   for (int i = tid; i < a.hq * P; i += W * 32) {
@@ -639,8 +643,7 @@ cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int64_t units = ((a.T + 31) / 32) * a.hkv;
   const int grid = grid_for(reinterpret_cast<const void*>(k), W * 32, smem, (units + W - 1) / W);
-  k<<<grid, W * 32, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, W * 32, smem, stream, a);
 }
 
 // The lane-per-key-head kernel applies (4-bit codes, d ≤ 128, a power-of-two
