@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 
 import oracle.codebook as ocb
+import oracle.ggml_blocks as ogg
 import oracle.hadamard as oh
 import oracle.q4_0 as oq4
 import oracle.qjl as oqjl
@@ -150,3 +151,63 @@ def test_mutation_qjl_constant(monkeypatch, factor):
 
     monkeypatch.setattr(oqjl, "estimate_residual_dot", bad)
     assert _fails(pins.test_qjl_estimator_unbiased_monte_carlo)
+
+
+def test_mutation_q8_0_rounds_half_to_even(monkeypatch):
+    """q8_0 codes with numpy's round-half-to-even instead of halves away from zero."""
+    good = ogg.block_decisions
+
+    def bad(y32, fmt, pick=None):
+        q, s32, m32, margin = good(y32, fmt, pick)
+        if fmt == "q8_0":
+            inv = np.where(s32 != 0, np.float32(1.0) / np.where(s32 != 0, s32, 1), 0).astype(np.float32)
+            q = np.round((np.asarray(y32, np.float32) * inv[..., None]).astype(np.float32)).astype(np.int64)
+        return q, s32, m32, margin
+
+    monkeypatch.setattr(ogg, "block_decisions", bad)
+    assert _fails(pins.test_ggml_hand_worked_blocks)
+
+
+def test_mutation_q5_high_bits_reversed(monkeypatch):
+    """The q5 high-bit word with bit 31 − j instead of bit j."""
+    good = ogg.serialize
+
+    def bad(fmt, q, scale32, min32):
+        if fmt in ("q5_0", "q5_1"):
+            q = q[..., ::-1].copy() & 16 | (q & 15)
+        return good(fmt, q, scale32, min32)
+
+    monkeypatch.setattr(ogg, "serialize", bad)
+    assert _fails(pins.test_ggml_hand_worked_blocks)
+
+
+def test_mutation_q4_1_min_and_scale_swapped(monkeypatch):
+    """q4_1 / q5_1 with the min stored before the scale."""
+    good = ogg.serialize
+
+    def bad(fmt, q, scale32, min32):
+        if fmt in ("q4_1", "q5_1"):
+            return good(fmt, q, min32, scale32)
+        return good(fmt, q, scale32, min32)
+
+    monkeypatch.setattr(ogg, "serialize", bad)
+    assert _fails(pins.test_ggml_hand_worked_blocks)
+
+
+def test_mutation_q5_0_scale_from_unsigned_max(monkeypatch):
+    """q5_0 with Δ = max|y|/−16 (the sign of the largest element dropped)."""
+    good = ogg.block_decisions
+
+    def bad(y32, fmt, pick=None):
+        if fmt != "q5_0":
+            return good(y32, fmt, pick)
+        y32 = np.asarray(y32, np.float32)
+        a = np.max(np.abs(y32), axis=-1)
+        delta = (a / np.float32(-16.0)).astype(np.float32)
+        inv = np.where(delta != 0, np.float32(1.0) / np.where(delta != 0, delta, 1), 0).astype(np.float32)
+        r = ((y32 * inv[..., None]).astype(np.float32) + np.float32(16.5)).astype(np.float32)
+        q = np.clip(np.floor(r), 0, 31).astype(np.int64)
+        return q, delta, np.zeros_like(delta), np.zeros(y32.shape)
+
+    monkeypatch.setattr(ogg, "block_decisions", bad)
+    assert _fails(pins.test_ggml_hand_worked_blocks)

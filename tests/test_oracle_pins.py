@@ -16,7 +16,7 @@ import pytest
 import scipy.linalg
 import scipy.stats
 
-from oracle import codebook, hadamard, q4_0, qjl, rng, rrq, sphere
+from oracle import codebook, ggml_blocks, hadamard, q4_0, qjl, rng, rrq, sphere
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -489,3 +489,93 @@ def test_qjl_estimator_unbiased_monte_carlo():
     assert abs(est.mean() - truth) < 4 * est.std() / math.sqrt(est.size)
     # the residual chain corrects the MSE shrinkage on average
     assert np.linalg.norm(r[0]) > 0
+
+
+# ---------------------------------------------------------- other GGML block types
+def _ggml_inputs(name):
+    j = np.arange(32)
+    if name == "ramp16":
+        return (j % 16) * 0.25 - 2.0
+    if name == "ramp32":
+        return j * 0.125 - 2.0
+    if name == "halves":
+        x = np.zeros(32)
+        x[:6] = [127.0, 0.5, -0.5, 1.5, -2.5, 2.5]
+        return x
+    return _q4_inputs(name)
+
+
+def test_ggml_hand_worked_blocks():
+    lines = _golden_lines("ggml_blocks.txt")
+    assert {ln.split("|")[0].strip() for ln in lines} == set(ggml_blocks.FORMATS)
+    for ln in lines:
+        fmt, name, hexbytes = (p.strip() for p in ln.split("|"))
+        want = bytes.fromhex(hexbytes.replace(" ", ""))
+        assert len(want) == ggml_blocks.BLOCK_BYTES[fmt], (fmt, name)
+        enc = ggml_blocks.encode(_ggml_inputs(name)[None], 0, fmt, rotate_first=False)
+        assert bytes(enc.blocks[0]) == want, (fmt, name, enc.blocks[0].tobytes().hex())
+
+
+@pytest.mark.parametrize("fmt", ggml_blocks.FORMATS)
+def test_ggml_grid_round_trip_exact(fmt):
+    """Inputs on each type's own grid (step 2^-k, range fixed by the block) come back exactly."""
+    rg = np.random.default_rng(5)
+    n, d = 40, 128
+    nb = d // 32
+    if fmt in ("q4_1", "q5_1"):
+        levels = 15 if fmt == "q4_1" else 31
+        step = 2.0 ** rg.integers(-6, 2, size=(n, nb, 1))
+        lo = rg.integers(-64, 64, size=(n, nb, 1)) * step
+        q = rg.integers(0, levels + 1, size=(n, nb, 32))
+        q[:, :, 0], q[:, :, 1] = 0, levels  # the block spans the whole range
+        x = lo + q * step
+    elif fmt == "q5_0":
+        step = 2.0 ** rg.integers(-6, 2, size=(n, nb, 1))
+        q = rg.integers(1, 32, size=(n, nb, 32))
+        q[:, :, 0] = 0  # the first element of largest magnitude is -16 steps
+        x = (q - 16) * step
+    else:
+        step = 2.0 ** rg.integers(-6, 2, size=(n, nb, 1))
+        q = rg.integers(-126, 127, size=(n, nb, 32))
+        q[:, :, 3] = 127
+        x = q * step
+    x = x.reshape(n, d)
+    enc = ggml_blocks.encode(x, 0, fmt, rotate_first=False)
+    assert np.array_equal(ggml_blocks.decode_exact(enc.blocks, d, 0, fmt, rotate_first=False), x)
+
+
+@pytest.mark.parametrize("fmt", ggml_blocks.FORMATS)
+def test_ggml_rotation_equivalence_and_error_bound(fmt):
+    """rotate = 1 encodes Πx exactly as rotate = 0 encodes it; every decoded block value
+    lies within half a step (plus the fp16 rounding of the stored scalars) of its input."""
+    rg = np.random.default_rng(6)
+    x = rg.standard_normal((30, 128)) * rg.uniform(0.1, 10, size=(30, 1))
+    e1 = ggml_blocks.encode(x, 42, fmt, rotate_first=True)
+    e0 = ggml_blocks.encode(rrq.rotate(x, 42), 0, fmt, rotate_first=False)
+    assert np.array_equal(e1.blocks, e0.blocks)
+    y = rrq.rotate(x, 42)
+    v = ggml_blocks.dequantize(e1.blocks, 128, fmt)
+    scale, mn, q = ggml_blocks.parse_blocks(e1.blocks, 128, fmt)
+    step = np.repeat(np.abs(scale), 32, axis=1)
+    # the clamp of the top code (q5_0, q4_0-like) costs up to one step on the
+    # largest element of the opposite sign; everything else is within half a step
+    slack = 1.0 if fmt == "q5_0" else 0.5
+    err = np.abs(v - y)
+    bound = slack * step + 2e-3 * np.repeat(np.max(np.abs(y.reshape(30, 4, 32)), axis=2), 32, axis=1)
+    assert np.all(err <= bound)
+    back = ggml_blocks.decode_exact(e1.blocks, 128, 42, fmt, rotate_first=True)
+    assert np.allclose(rrq.rotate(back, 42), v)
+
+
+def test_ggml_q8_rounds_half_away_from_zero_and_q4_1_matches_q4_0_on_symmetric_grids():
+    x = np.zeros((1, 32))
+    x[0, :4] = [127.0, 126.5, -126.5, -0.5]
+    enc = ggml_blocks.encode(x, 0, "q8_0", rotate_first=False)
+    assert enc.q[0, :4].tolist() == [127, 127, -127, -1]
+    # both types reproduce a block whose values sit on their shared grid exactly
+    g = ((np.arange(32) * 5) % 16 - 8) * 0.5
+    g[0], g[1] = -4.0, 3.5
+    e40 = q4_0.encode(g[None], 0, rotate_first=False)
+    e41 = ggml_blocks.encode(g[None], 0, "q4_1", rotate_first=False)
+    assert np.array_equal(q4_0.decode_exact(e40.blocks, 32, 0, rotate_first=False), g[None])
+    assert np.array_equal(ggml_blocks.decode_exact(e41.blocks, 32, 0, "q4_1", rotate_first=False), g[None])
