@@ -13,10 +13,12 @@ the decisions taken in fp32 (y rounded to fp32 first; every product, sum and
 quotient below rounded to fp32, no fused multiply-add), in blocks of 32
 consecutive coordinates:
 
-* q4_1 (20 bytes): lo = min y, hi = max y; Δ = (hi − lo)/15; inv = 1/Δ (0 when
+* q4_1 (20 bytes): lo = min y, hi = max y (the first such element in index
+  order, so that of −0 and +0 the first is kept); Δ = (hi − lo)/15; inv = 1/Δ (0 when
   Δ = 0); q_j = min(15, ⌊(y_j − lo)·inv + 0.5⌋); stored fp16(Δ), fp16(lo), then
   byte j = q_j | q_{j+16} << 4.  Decode: q_j·Δ + lo.
-* q5_0 (22 bytes): m = the element of largest |y| with its sign (first on ties);
+* q5_0 (22 bytes): m = the element of largest |y| with its sign (first on ties;
+  +0 when the block is all zeros);
   Δ = m/−16; q_j = min(31, ⌊y_j·inv + 16.5⌋); stored fp16(Δ), then a 32-bit
   little-endian word whose bit j is bit 4 of q_j (j = 0..31), then byte
   j = (q_j & 15) | (q_{j+16} & 15) << 4.  Decode: (q_j − 16)·Δ.
@@ -59,8 +61,17 @@ class BlockEncoded:
 
 
 def _signed_absmax(y32: np.ndarray) -> np.ndarray:
-    """The element of largest |y| with its sign, first index on ties; over the last axis."""
+    """The element of largest |y| with its sign, first index on ties, over the last
+    axis; +0 for a block of zeros (whatever the signs of its zeros)."""
     idx = np.argmax(np.abs(y32), axis=-1)
+    m = np.take_along_axis(y32, idx[..., None], axis=-1)[..., 0]
+    return np.where(np.abs(m) > 0, m, F32(0.0)).astype(F32)
+
+
+def _first_extreme(y32: np.ndarray, largest: bool) -> np.ndarray:
+    """The first element (in index order) of smallest or largest value: −0 and +0
+    compare equal, so the first of them is kept."""
+    idx = np.argmax(y32, axis=-1) if largest else np.argmin(y32, axis=-1)
     return np.take_along_axis(y32, idx[..., None], axis=-1)[..., 0]
 
 
@@ -83,8 +94,8 @@ def block_decisions(y32: np.ndarray, fmt: str, pick=None):
     zero = np.zeros(y32.shape[:-1], dtype=F32)
     if fmt in ("q4_1", "q5_1"):
         levels = 15 if fmt == "q4_1" else 31
-        lo = np.min(y32, axis=-1)
-        hi = np.max(y32, axis=-1)
+        lo = _first_extreme(y32, largest=False)
+        hi = _first_extreme(y32, largest=True)
         delta = ((hi - lo).astype(F32) / F32(levels)).astype(F32)
         inv = _inverse(delta)
         t = ((y32 - lo[..., None]).astype(F32) * inv[..., None]).astype(F32)

@@ -579,3 +579,16 @@ def test_ggml_q8_rounds_half_away_from_zero_and_q4_1_matches_q4_0_on_symmetric_g
     e41 = ggml_blocks.encode(g[None], 0, "q4_1", rotate_first=False)
     assert np.array_equal(q4_0.decode_exact(e40.blocks, 32, 0, rotate_first=False), g[None])
     assert np.array_equal(ggml_blocks.decode_exact(e41.blocks, 32, 0, "q4_1", rotate_first=False), g[None])
+
+
+def test_ggml_signed_zero_rules():
+    """A block of −0: the absmax types take the scale from +0 (Δ = +0/−16 = −0, fp16
+    8000), the min/max types keep the first extreme in index order (here −0)."""
+    x = np.full((1, 32), -0.0)
+    b50 = ggml_blocks.encode(x, 0, "q5_0", rotate_first=False).blocks[0]
+    assert b50[:2].tobytes() == b"\x00\x80"
+    b41 = ggml_blocks.encode(x, 0, "q4_1", rotate_first=False).blocks[0]
+    assert b41[:4].tobytes() == b"\x00\x00\x00\x80"
+    x[0, 0] = 0.0  # +0 first, then −0: the min is the first, +0
+    b41 = ggml_blocks.encode(x, 0, "q4_1", rotate_first=False).blocks[0]
+    assert b41[:4].tobytes() == b"\x00\x00\x00\x00"
