@@ -480,6 +480,21 @@ def extra_kernels(torch, dev, flush, reps, peak):
                        "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
     del blk, xo
 
+    # the other GGML block types on the same vectors (rotate, then blocks of 32)
+    for fmt in ("q4_1", "q5_0", "q5_1", "q8_0"):
+        per = 4 * B.rrq_ggml_block_bytes(fmt)
+        gb = torch.empty(n, per, dtype=torch.uint8, device=dev)
+        xo = torch.empty_like(x)
+        ms_e = time_loop(torch, stream, lambda k: B.rrq_ggml_rot(x, 42, fmt, out=gb), reps)
+        ms_d = time_loop(torch, stream, lambda k: B.rrq_ggml_rot_decode(gb, 128, 42, fmt, out=xo), reps)
+        by = n * (256 + per)
+        out[f"{fmt}_rot"] = {"workload": f"fp16 [131072 x 8 x 128], rotate + {fmt}",
+                             "encode_us": 1e3 * ms_e, "decode_us": 1e3 * ms_d,
+                             "encode_gbs": by / ms_e / 1e6, "decode_gbs": by / ms_d / 1e6,
+                             "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
+                             "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
+        del gb, xo
+
     # DRIVE one-bit encode (unbiased scale) of the same vectors, and the
     # one-bit decode back to fp16
     dc = torch.empty(n, 16, dtype=torch.uint8, device=dev)

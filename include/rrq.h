@@ -78,6 +78,13 @@ extern "C" {
 #define RRQ_F16 1
 #define RRQ_BF16 2
 
+/* GGML block types for rrq_ggml_rot (the numbers of ggml's own type enumeration) */
+#define RRQ_GGML_Q4_0 2
+#define RRQ_GGML_Q4_1 3
+#define RRQ_GGML_Q5_0 6
+#define RRQ_GGML_Q5_1 7
+#define RRQ_GGML_Q8_0 8
+
 /* Packed-format version this library writes and reads. */
 int rrq_format_version(void);
 
@@ -217,6 +224,53 @@ int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, in
  *   blocks  [n × d/32 × 18] bytes;  out [n × d] of out_dtype
  */
 int rrq_q4_0_rot_decode(const void* blocks, int64_t n, int d, uint64_t seed, int rotate,
+                        void* out, int out_dtype, void* stream);
+
+/*
+ * rrq_ggml_block_bytes — bytes of one block of 32 values of a GGML block type:
+ * 18 (q4_0), 20 (q4_1), 22 (q5_0), 24 (q5_1), 34 (q8_0); 0 for any other type.
+ */
+int rrq_ggml_block_bytes(int type);
+
+/*
+ * rrq_ggml_rot — "Attn-rot" with any of the GGML block types the page lists:
+ * rotate (rotate = 1: y = Πx, orthonormal; rotate = 0: y = x), then blocks of 32.
+ * "Attn-rot (TurboQuant lite) in llama.cpp" page, "How to use it": q4_0 first of
+ * all, also q4_1, q5_0, q5_1 (and q8_0).  The page names the types without
+ * defining them; the public llama.cpp blocks are used, kept identical for
+ * interoperability, with every decision in fp32 (y rounded to fp32, each
+ * product, sum and quotient rounded, no fused multiply-add), inv = fp32(1/Δ),
+ * 0 when Δ = 0:
+ *   q4_0  as rrq_q4_0_rot (18 bytes);
+ *   q4_1  lo, hi = first min / max in index order, Δ = (hi − lo)/15,
+ *         q_j = min(15, ⌊(y_j − lo)·inv + 0.5⌋); 20 bytes: fp16 Δ, fp16 lo, then
+ *         byte j = q_j | q_{j+16} << 4;
+ *   q5_0  m = first element of largest |y| (+0 for a block of zeros), Δ = m/−16,
+ *         q_j = min(31, ⌊y_j·inv + 16.5⌋); 22 bytes: fp16 Δ, a little-endian
+ *         32-bit word whose bit j is bit 4 of q_j, then byte j = (q_j & 15) |
+ *         (q_{j+16} & 15) << 4;
+ *   q5_1  as q4_1 with Δ = (hi − lo)/31 and no clamp; 24 bytes: fp16 Δ, fp16 lo,
+ *         the high-bit word, the nibble bytes;
+ *   q8_0  Δ = max|y|/127, q_j = round(y_j·inv) (halves away from zero); 34
+ *         bytes: fp16 Δ, then q_j as signed bytes.
+ *   x       [n × d] of x_dtype (d in {64, 128, 256, 512})
+ *   type    RRQ_GGML_Q4_0 / _Q4_1 / _Q5_0 / _Q5_1 / _Q8_0
+ *   blocks  [n × d/32 × rrq_ggml_block_bytes(type)] bytes (output; 16-byte aligned)
+ * Errors: RRQ_ERR_INVALID (type, d, dtype, rotate, null or misaligned pointer),
+ * RRQ_ERR_CUDA.
+ */
+int rrq_ggml_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate, int type,
+                 void* blocks, void* stream);
+
+/*
+ * rrq_ggml_rot_decode — inverse of rrq_ggml_rot: with the stored fp16 values,
+ * ŷ_j = q_j·Δ + lo (q4_1, q5_1), (q_j − 16)·Δ (q5_0), q_j·Δ (q8_0), (q_j − 8)·Δ
+ * (q4_0); then x̂ = Πᵀŷ when rotate = 1.  fp32 arithmetic (q·Δ + lo as one fused
+ * multiply-add), rounded to out_dtype.
+ *   blocks  [n × d/32 × rrq_ggml_block_bytes(type)] bytes;  out [n × d] of out_dtype
+ * Errors: RRQ_ERR_INVALID, RRQ_ERR_CUDA.
+ */
+int rrq_ggml_rot_decode(const void* blocks, int type, int64_t n, int d, uint64_t seed, int rotate,
                         void* out, int out_dtype, void* stream);
 
 /*

@@ -21,6 +21,9 @@ from .binding import (  # noqa: F401
     rrq_drive_encode,
     rrq_encode,
     rrq_format_version,
+    rrq_ggml_block_bytes,
+    rrq_ggml_rot,
+    rrq_ggml_rot_decode,
     rrq_q4_0_rot,
     rrq_q4_0_rot_decode,
     rrq_qjl_matrix,

@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librrq.so")
 RRQ_OK, RRQ_ERR_INVALID, RRQ_ERR_CUDA, RRQ_ERR_UNSUPPORTED = 0, 1, 2, 3
 RRQ_F32, RRQ_F16, RRQ_BF16 = 0, 1, 2
 DTYPE_CODE = {torch.float32: RRQ_F32, torch.float16: RRQ_F16, torch.bfloat16: RRQ_BF16}
+# GGML block types (ggml's own type numbers), as in include/rrq.h
+GGML_TYPES = {"q4_0": 2, "q4_1": 3, "q5_0": 6, "q5_1": 7, "q8_0": 8}
 
 _c_i64 = ctypes.c_int64
 _c_u64 = ctypes.c_uint64
@@ -40,6 +42,9 @@ SIGNATURES = {
                              ctypes.c_float, _vp, _vp]),
     "rrq_q4_0_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
     "rrq_q4_0_rot_decode": (_int, [_vp, _c_i64, _int, _c_u64, _int, _vp, _int, _vp]),
+    "rrq_ggml_block_bytes": (_int, [_int]),
+    "rrq_ggml_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _int, _vp, _vp]),
+    "rrq_ggml_rot_decode": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _int, _vp]),
     "rrq_qjl_matrix": (_int, [_c_u64, _int, _vp]),
 }
 
@@ -268,6 +273,44 @@ def rrq_q4_0_rot_decode(blocks: torch.Tensor, d: int, seed: int, rotate: bool = 
     _check(lib().rrq_q4_0_rot_decode(_ptr(blocks), n, d, seed, int(bool(rotate)), _ptr(out),
                                      DTYPE_CODE[out.dtype], _stream(blocks)),
            "rrq_q4_0_rot_decode")
+    return out
+
+
+def rrq_ggml_block_bytes(fmt: str) -> int:
+    """Bytes of one block of 32 values of a GGML block type ('q4_0', 'q4_1', 'q5_0', 'q5_1', 'q8_0')."""
+    return lib().rrq_ggml_block_bytes(GGML_TYPES[fmt])
+
+
+def rrq_ggml_rot(x: torch.Tensor, seed: int, fmt: str, rotate: bool = True, out=None):
+    """Rotate (optionally) then quantise rows of x [..., d] into GGML blocks of type `fmt`:
+    uint8 [..., d/32*block_bytes]."""
+    _dev_tensor(x, "x", DTYPE_CODE)
+    d = x.shape[-1]
+    n = x.numel() // d if d else 0
+    per = d // 32 * rrq_ggml_block_bytes(fmt)
+    if out is None:
+        out = torch.empty(*x.shape[:-1], per, dtype=torch.uint8, device=x.device)
+    _dev_tensor(out, "out", (torch.uint8,))
+    if out.numel() != n * per:
+        raise ValueError("out has the wrong size")
+    _check(lib().rrq_ggml_rot(_ptr(x), DTYPE_CODE[x.dtype], n, d, seed, int(bool(rotate)),
+                              GGML_TYPES[fmt], _ptr(out), _stream(x)), "rrq_ggml_rot")
+    return out
+
+
+def rrq_ggml_rot_decode(blocks: torch.Tensor, d: int, seed: int, fmt: str, rotate: bool = True,
+                        out_dtype=torch.float16, out=None):
+    _dev_tensor(blocks, "blocks", (torch.uint8,))
+    per = d // 32 * rrq_ggml_block_bytes(fmt)
+    if blocks.shape[-1] != per:
+        raise ValueError(f"blocks must be [..., d/32*{per // (d // 32)}]")
+    n = blocks.numel() // per
+    if out is None:
+        out = torch.empty(*blocks.shape[:-1], d, dtype=out_dtype, device=blocks.device)
+    _dev_tensor(out, "out", DTYPE_CODE)
+    _check(lib().rrq_ggml_rot_decode(_ptr(blocks), GGML_TYPES[fmt], n, d, seed, int(bool(rotate)),
+                                     _ptr(out), DTYPE_CODE[out.dtype], _stream(blocks)),
+           "rrq_ggml_rot_decode")
     return out
 
 

@@ -8,6 +8,7 @@
 #include <cstring>
 
 #include "rrq.h"
+#include "ggml_blocks.h"
 #include "rrq_params.h"
 
 namespace {
@@ -236,6 +237,47 @@ int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, in
   const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   return status_of(rrq::launch_q4_0(x, x_dtype, n, d, seed, rotate, inv_sqrt_d, blocks,
                                     as_stream(stream)));
+}
+
+int rrq_ggml_block_bytes(int type) {
+  switch (type) {
+    case RRQ_GGML_Q4_0: return 18;
+    case RRQ_GGML_Q4_1: return 20;
+    case RRQ_GGML_Q5_0: return 22;
+    case RRQ_GGML_Q5_1: return 24;
+    case RRQ_GGML_Q8_0: return 34;
+  }
+  return 0;
+}
+
+int rrq_ggml_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate, int type,
+                 void* blocks, void* stream) {
+  if (n < 0 || !d_ok(d) || !dtype_ok(x_dtype) || (rotate != 0 && rotate != 1) ||
+      rrq_ggml_block_bytes(type) == 0)
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(x, n, 32) || !arr_ok(blocks, n, 16)) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  if (type == RRQ_GGML_Q4_0)
+    return status_of(rrq::launch_q4_0(x, x_dtype, n, d, seed, rotate, inv_sqrt_d, blocks,
+                                      as_stream(stream)));
+  return status_of(rrq::launch_ggml_blocks(x, x_dtype, n, d, seed, rotate, type, inv_sqrt_d, blocks,
+                                           as_stream(stream)));
+}
+
+int rrq_ggml_rot_decode(const void* blocks, int type, int64_t n, int d, uint64_t seed, int rotate,
+                        void* out, int out_dtype, void* stream) {
+  if (n < 0 || !d_ok(d) || !dtype_ok(out_dtype) || (rotate != 0 && rotate != 1) ||
+      rrq_ggml_block_bytes(type) == 0)
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(blocks, n, 16) || !arr_ok(out, n, 32)) return RRQ_ERR_INVALID;
+  if (n == 0) return RRQ_OK;
+  const float inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  if (type == RRQ_GGML_Q4_0)
+    return status_of(rrq::launch_q4_0_decode(blocks, n, d, seed, rotate, inv_sqrt_d, out, out_dtype,
+                                             as_stream(stream)));
+  return status_of(rrq::launch_ggml_blocks_decode(blocks, type, n, d, seed, rotate, inv_sqrt_d, out,
+                                                  out_dtype, as_stream(stream)));
 }
 
 int rrq_q4_0_rot_decode(const void* blocks, int64_t n, int d, uint64_t seed, int rotate, void* out,

@@ -118,6 +118,14 @@ def test_other_entry_points_validate():
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 96, 0, 1, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 128, 0, 3, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot_decode(P, 4, 128, 0, 1, P, 5, None) == B.RRQ_ERR_INVALID
+    # GGML block types: sizes, unknown types, bad rotate flag
+    assert [lib.rrq_ggml_block_bytes(t) for t in (2, 3, 6, 7, 8, 1, 9)] == [18, 20, 22, 24, 34, 0, 0]
+    assert lib.rrq_ggml_rot(P, B.RRQ_F16, 4, 128, 0, 1, 4, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_ggml_rot(P, B.RRQ_F16, 4, 128, 0, 2, 3, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_ggml_rot(P, B.RRQ_F16, 4, 96, 0, 1, 3, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_ggml_rot_decode(P, 5, 4, 128, 0, 1, P, B.RRQ_F16, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_ggml_rot_decode(P_MIS, 3, 4, 128, 0, 1, P, B.RRQ_F16, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_ggml_rot(ctypes.c_void_p(None), B.RRQ_F16, 0, 128, 0, 1, 8, P, None) == B.RRQ_OK
     # DRIVE: unbiased must be 0/1, d a supported size, scales 4-byte aligned
     assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 128, 0, 2, P, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 100, 0, 0, P, P, None) == B.RRQ_ERR_INVALID
