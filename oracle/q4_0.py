@@ -14,7 +14,8 @@ llama.cpp/GGML q4_0 block, kept identical for interoperability):
 * the decisions are taken in fp32, the precision of the format's reference
   arithmetic (the pages fix none): y is rounded to fp32 first;
 * m = the block element of largest magnitude, with its sign (first index on
-  ties); Δ = m / −8 (exact); inv = fp32(1/Δ) (0 when Δ = 0);
+  ties; +0 when every element is ±0, as the public reference quantiser starts
+  from +0); Δ = m / −8 (exact); inv = fp32(1/Δ) (0 when Δ = 0);
 * q_j = min(15, ⌊fp32(fp32(y_j·inv) + 8.5)⌋) (the argument is ≥ 0.5 since
   |y_j·inv| ≤ 8);
 * stored: fp16(Δ) (2 bytes, little endian) then 16 bytes; byte j holds q_j in
@@ -56,6 +57,7 @@ def encode(x, seed: int, rotate_first: bool = True) -> Q4Encoded:
     y32 = yb.astype(np.float32)
     idx = np.argmax(np.abs(y32), axis=2)  # first index on ties
     m = np.take_along_axis(y32, idx[:, :, None], axis=2)[:, :, 0]
+    m = np.where(np.abs(m) > 0, m, np.float32(0.0)).astype(np.float32)  # all-zero block: +0
     delta = (m / np.float32(-8.0)).astype(np.float32)
     inv = np.zeros_like(delta)
     nz = delta != 0

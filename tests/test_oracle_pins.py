@@ -592,3 +592,9 @@ def test_ggml_signed_zero_rules():
     x[0, 0] = 0.0  # +0 first, then −0: the min is the first, +0
     b41 = ggml_blocks.encode(x, 0, "q4_1", rotate_first=False).blocks[0]
     assert b41[:4].tobytes() == b"\x00\x00\x00\x00"
+
+
+def test_q4_0_block_of_negative_zeros_stores_minus_zero_scale():
+    """A block of −0: the scale comes from +0 (Δ = +0/−8 = −0, fp16 8000), every q = 8."""
+    enc = q4_0.encode(np.full((1, 32), -0.0), 0, rotate_first=False)
+    assert enc.blocks[0].tobytes() == bytes.fromhex("0080" + "88" * 16)
