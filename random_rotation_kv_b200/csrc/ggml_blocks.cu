@@ -1,11 +1,14 @@
-// ggml_blocks.cu — "Attn-rot" with the other GGML block types: randomized
-// Hadamard rotation, then q4_1, q5_0, q5_1 or q8_0 blocks of 32, and back.
+// ggml_blocks.cu — "Attn-rot" with the GGML block types: randomized Hadamard
+// rotation, then q4_0, q4_1, q5_0, q5_1 or q8_0 blocks of 32, and back (the q4_0
+// decoder in q4_0.cu is used for q4_0 blocks; it reads them faster).
 //
 // "Attn-rot (TurboQuant lite) in llama.cpp" page, section "How to use it":
 // besides q4_0, the cache types q4_1, q5_0 and q5_1 (and q8_0).  The page names
 // them without defining them; the public llama.cpp blocks are used, kept
 // identical for interoperability, with every decision in fp32 (each product,
 // sum and quotient rounded, no fused multiply-add):
+//   q4_0 (18 B): m = first element of largest |y| (+0 for a block of zeros),
+//        Δ = m/−8, q = min(15, ⌊y·inv + 8.5⌋); fp16 Δ, 16 bytes q_j | q_{j+16} << 4.
 //   q4_1 (20 B): lo/hi = first min/max in index order, Δ = (hi − lo)/15,
 //        q = min(15, ⌊(y − lo)·inv + 0.5⌋); fp16 Δ, fp16 lo, 16 nibble bytes.
 //   q5_0 (22 B): m = first element of largest |y| (+0 for a block of zeros),
@@ -34,6 +37,7 @@ constexpr int kWarpBlocks = 64;  // blocks of 32 per warp pass (2048 values)
 constexpr int kRow = 33;         // shared row stride of a block, in floats
 
 template <int F> struct BlockType;
+template <> struct BlockType<RRQ_GGML_Q4_0> { static constexpr int kBytes = 18; };
 template <> struct BlockType<RRQ_GGML_Q4_1> { static constexpr int kBytes = 20; };
 template <> struct BlockType<RRQ_GGML_Q5_0> { static constexpr int kBytes = 22; };
 template <> struct BlockType<RRQ_GGML_Q5_1> { static constexpr int kBytes = 24; };
@@ -89,20 +93,26 @@ __device__ __forceinline__ void encode_block(const float* v, uint8_t* out) {
     } else {
       put_nibbles(out + 4, q);
     }
-  } else if constexpr (F == RRQ_GGML_Q5_0) {
-    float amax = 0.f, m = 0.f;
+  } else if constexpr (F == RRQ_GGML_Q4_0 || F == RRQ_GGML_Q5_0) {
+    constexpr float kHalf = F == RRQ_GGML_Q4_0 ? 8.f : 16.f;
+    constexpr int kTop = F == RRQ_GGML_Q4_0 ? 15 : 31;
+    float amax = 0.f, m = 0.f;  // m stays +0 for a block of zeros
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const float a = fabsf(v[j]);
       if (amax < a) { amax = a; m = v[j]; }
     }
-    const float dlt = __fdiv_rn(m, -16.f);
+    const float dlt = __fdiv_rn(m, -kHalf);
     const float inv = dlt != 0.f ? __fdiv_rn(1.f, dlt) : 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) q[j] = min(31, int(__fadd_rn(__fmul_rn(v[j], inv), 16.5f)));
+    for (int j = 0; j < 32; ++j) q[j] = min(kTop, int(__fadd_rn(__fmul_rn(v[j], inv), kHalf + 0.5f)));
     st16(out, half_bits(dlt));
-    put_high_bits(out + 2, q);
-    put_nibbles(out + 6, q);
+    if constexpr (F == RRQ_GGML_Q5_0) {
+      put_high_bits(out + 2, q);
+      put_nibbles(out + 6, q);
+    } else {
+      put_nibbles(out + 2, q);
+    }
   } else {
     float amax = 0.f;
 #pragma unroll
@@ -354,6 +364,7 @@ cudaError_t dec_f(const void* blocks, int64_t n, int d, uint64_t seed, int rotat
 cudaError_t launch_ggml_blocks(const void* x, int dtype, int64_t n, int d, uint64_t seed, int rotate,
                                int type, float inv_sqrt_d, void* blocks, cudaStream_t stream) {
   switch (type) {
+    case RRQ_GGML_Q4_0: return enc_f<RRQ_GGML_Q4_0>(x, dtype, n, d, seed, rotate, inv_sqrt_d, blocks, stream);
     case RRQ_GGML_Q4_1: return enc_f<RRQ_GGML_Q4_1>(x, dtype, n, d, seed, rotate, inv_sqrt_d, blocks, stream);
     case RRQ_GGML_Q5_0: return enc_f<RRQ_GGML_Q5_0>(x, dtype, n, d, seed, rotate, inv_sqrt_d, blocks, stream);
     case RRQ_GGML_Q5_1: return enc_f<RRQ_GGML_Q5_1>(x, dtype, n, d, seed, rotate, inv_sqrt_d, blocks, stream);

@@ -1,6 +1,6 @@
 // ggml_blocks.h — launchers of the GGML block-type kernels (ggml_blocks.cu),
-// called by the C ABI (api.cpp).  Both are asynchronous on `stream`; `type` is
-// one of RRQ_GGML_Q4_1, RRQ_GGML_Q5_0, RRQ_GGML_Q5_1, RRQ_GGML_Q8_0.
+// called by the C ABI (api.cpp) and by the q4_0 encoder entry (q4_0.cu).  Both
+// are asynchronous on `stream`; `type` is one of the RRQ_GGML_* block types.
 #pragma once
 
 #include <cuda_runtime.h>

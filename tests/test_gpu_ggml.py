@@ -189,3 +189,23 @@ def test_ggml_full_size_sampled_and_rotation_gain(fmt):
         back = B.rrq_ggml_rot_decode(blk, 128, 42, fmt, rotate=rot, out_dtype=torch.float32)
         mse[rot] = float(torch.mean((back - xd.float()) ** 2))
     assert mse[True] < mse[False], (fmt, mse)
+
+
+def test_q4_0_through_the_block_type_entry_and_signed_zero_blocks():
+    """rrq_ggml_rot(q4_0) writes what rrq_q4_0_rot writes, and its decode matches;
+    blocks of −0 store the −0 scale (GGML starts its signed max at +0)."""
+    from oracle import q4_0 as oq
+    x = W.gaussian(257, 256, "bf16", seed=77, scale=1.3).flat().copy()
+    x[5] = -0.0
+    xd = to_dev(x, "bf16")
+    a = B.rrq_ggml_rot(xd, 42, "q4_0", rotate=False)
+    b = B.rrq_q4_0_rot(xd, 42, rotate=False)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    enc = oq.encode(x.astype(np.float64), 42, rotate_first=False)
+    assert np.array_equal(a.cpu().numpy(), enc.blocks)
+    assert a[5].cpu().numpy().reshape(8, 18)[:, :2].tobytes() == b"\x00\x80" * 8
+    da = B.rrq_ggml_rot_decode(a, 256, 42, "q4_0", rotate=False, out_dtype=torch.float32)
+    db = B.rrq_q4_0_rot_decode(b, 256, 42, rotate=False, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(da, db)
