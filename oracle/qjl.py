@@ -70,3 +70,27 @@ def estimate_residual_dot(q_rot, s_matrix, packed_signs, rnorm) -> np.ndarray:
     sq = s @ as_f64(q_rot)
     signs = unpack_signs(packed_signs, d)
     return np.sqrt(np.pi / 2.0) / m * as_f64(rnorm) * (signs @ sq)
+
+
+def scores_unbiased(q, packed, norms, qjl_bits, rnorm, t_len: int, hkv: int, d: int, bits: int,
+                    seed: int, s_matrix, levels=None, scale: float = 1.0) -> np.ndarray:
+    """Unbiased attention scores on TurboQuant-style keys, float64 [Hq, T].
+
+    "Random-rotation quantization" page, TurboQuant bullet (an MSE quantiser
+    followed by an unbiased one-bit stage on the residual) and "Three decoders,
+    one rotation", inner-product decoder:
+        s[h, t] = scale · ( <q_h, x̂_{t,g}> + √(π/2)/m · ρ_{t,g} · <S Π q_h, sign_{t,g}> ),
+    g = ⌊h·Hkv/Hq⌋, the first term the b-bit MSE score (``rrq.scores``), the
+    second the residual estimate (``estimate_residual_dot``).  Rows of packed /
+    norms / qjl_bits / rnorm are n = t·Hkv + g.
+    """
+    q = as_f64(q)
+    hq = q.shape[0]
+    out = rrq.scores(q, packed, norms, t_len, hkv, d, bits, seed, levels, scale)
+    qr = rrq.rotate(q, seed)
+    qb = np.asarray(qjl_bits, dtype=np.uint8).reshape(t_len, hkv, d // 8)
+    rn = as_f64(rnorm).reshape(t_len, hkv)
+    for h in range(hq):
+        g = rrq.kv_group(h, hq, hkv)
+        out[h] += scale * estimate_residual_dot(qr[h], s_matrix, qb[:, g, :], rn[:, g])
+    return out

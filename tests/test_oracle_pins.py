@@ -598,3 +598,30 @@ def test_q4_0_block_of_negative_zeros_stores_minus_zero_scale():
     """A block of −0: the scale comes from +0 (Δ = +0/−8 = −0, fp16 8000), every q = 8."""
     enc = q4_0.encode(np.full((1, 32), -0.0), 0, rotate_first=False)
     assert enc.blocks[0].tobytes() == bytes.fromhex("0080" + "88" * 16)
+
+
+
+def test_qjl_unbiased_scores_average_to_the_true_inner_product():
+    """scores_unbiased averaged over independent Gaussian projections S equals
+    scale·<q, x> (the MSE score alone is biased low), for every head and token."""
+    d, hq, hkv, t_len = 16, 4, 2, 3
+    rg = np.random.default_rng(21)
+    x = rg.standard_normal((t_len * hkv, d)) * 2.0
+    q = rg.standard_normal((hq, d))
+    g = np.arange(hq) // (hq // hkv)
+    truth = 0.5 * np.einsum("hi,thi->ht", q, x.reshape(t_len, hkv, d)[:, g, :])
+    acc, acc2, n = 0.0, 0.0, 3000
+    for _ in range(n):
+        s = rg.standard_normal((d, d))
+        enc = qjl.encode(x, 2, 7, s)
+        sc = qjl.scores_unbiased(q, enc.enc.packed, enc.enc.norms, enc.bits, enc.rnorm.astype(np.float64),
+                                 t_len, hkv, d, 2, 7, s, scale=0.5)
+        acc, acc2 = acc + sc, acc2 + sc * sc
+    mean = acc / n
+    sem = np.sqrt(np.maximum(acc2 / n - mean * mean, 0) / n)
+    assert np.all(np.abs(mean - truth) < 4.5 * sem + 1e-9)
+    mse_only = rrq.scores(q, enc.enc.packed, enc.enc.norms, t_len, hkv, d, 2, 7, scale=0.5)
+    # the MSE part is the same for every S; the unbiased score differs from it by the estimate
+    assert np.allclose(sc - mse_only,
+                       np.stack([0.5 * qjl.estimate_residual_dot(rrq.rotate(q, 7)[h], s, enc.bits.reshape(t_len, hkv, 2)[:, g[h]],
+                                                                  enc.rnorm.reshape(t_len, hkv)[:, g[h]]) for h in range(hq)]))
