@@ -465,6 +465,24 @@ def extra_kernels(torch, dev, flush, reps, peak):
                         "frac_of_hbm": by / ms / 1e6 / peak}
     del codes, norms, cs, ns, scs
 
+    # unbiased scores on the same keys stored TurboQuant-style: 2-bit codes + QJL bits
+    S = B.rrq_qjl_matrix(4242, 128, device=dev)
+    k = torch.from_numpy(w.flat()).to(dev)
+    sets = []
+    for _ in range(3):  # 3 copies of 56 MB: larger than L2 in rotation
+        c2, n2, b2, r2 = B.rrq_encode(k, 2, 42, qjl_S=S)
+        sets.append((c2, n2, b2, r2))
+    del k
+    sc = [torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev) for _ in range(3)]
+    ms = time_loop(torch, stream, lambda i: B.rrq_qk_scores_qjl(
+        q, *sets[i % 3], S, 8, 128, 2, 42, out=sc[i % 3]), reps)
+    by = nkh * (32 + 4 + 16 + 4) + 32 * w.x.shape[0] * 4
+    out["qk_scores_qjl"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128, "
+                                        "2-bit codes + QJL bits (unbiased)",
+                            "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
+                            "frac_of_hbm": by / ms / 1e6 / peak}
+    del sets, sc
+
     # workload 3: rotate-then-q4_0, 1,048,576 fp16 vectors
     w = W.attnrot()
     x = torch.from_numpy(w.flat()).to(dev)

@@ -203,6 +203,34 @@ int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norm
                   float* scores, void* stream);
 
 /*
+ * rrq_qk_scores_qjl — unbiased decode-time attention scores on keys stored as
+ * b-bit MSE codes plus the QJL one-bit residual sketch (rrq_encode with qjl_S).
+ * "Random-rotation quantization" page: "History", TurboQuant bullet (a biased
+ * MSE quantiser followed by an unbiased one-bit stage on the residual) and QJL
+ * bullet; "Three decoders, one rotation", inner-product decoder; "Bias vs
+ * unbiasedness".  With g = ⌊h·hkv/hq⌋:
+ *     scores[h][t] = scale · ( <q_h, x̂_{t,g}>
+ *                              + √(π/2)/d · ρ_{t,g} · <S·Π·q_h, sign_{t,g}> ),
+ * x̂ the b-bit MSE reconstruction (as rrq_qk_scores), sign_i = +1 where QJL bit i
+ * is set and −1 elsewhere, ρ the stored residual norm.  Averaged over the
+ * Gaussian S the score is unbiased for scale·<q_h, x_{t,g}>.
+ *   q          [hq × d] fp16 (unrotated)
+ *   codes      [T·hkv × d·bits/8] bytes, row t·hkv + g;  norms [T·hkv] float
+ *   qjl_bits   [T·hkv × d/8] bytes;  qjl_rnorm [T·hkv] float (as rrq_encode writes)
+ *   qjl_S      bf16 [d × d] (the S given to rrq_encode)
+ *   scores     [hq × T] float (output)
+ * d must be 128; hq a multiple of hkv with hq/hkv in {1, 2, 4, 8}.
+ * Accuracy: both dot products in fp16 pairs with fp32 partial sums (every 32
+ * products), each head's query and projected query scaled by a power of two.
+ * Errors: RRQ_ERR_INVALID, RRQ_ERR_UNSUPPORTED (d other than 128, group size),
+ * RRQ_ERR_CUDA.
+ */
+int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* norms,
+                      const uint8_t* qjl_bits, const float* qjl_rnorm, const uint16_t* qjl_S,
+                      int64_t T, int hkv, int d, int bits, uint64_t seed, const float* codebook,
+                      float scale, float* scores, void* stream);
+
+/*
  * rrq_q4_0_rot — "Attn-rot" (TurboQuant lite): rotate, then q4_0.
  * "Attn-rot (TurboQuant lite) in llama.cpp" page: rotate K/V before an
  * ordinary block format, q4_0 first of all.  With y = Πx (rotate = 1) or

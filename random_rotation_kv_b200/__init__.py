@@ -28,6 +28,7 @@ from .binding import (  # noqa: F401
     rrq_q4_0_rot_decode,
     rrq_qjl_matrix,
     rrq_qk_scores,
+    rrq_qk_scores_qjl,
     rrq_rotate,
     strerror,
 )

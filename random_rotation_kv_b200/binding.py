@@ -40,6 +40,8 @@ SIGNATURES = {
     "rrq_drive_encode": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp, _vp]),
     "rrq_qk_scores": (_int, [_vp, _int, _vp, _vp, _c_i64, _int, _int, _int, _c_u64, _vp,
                              ctypes.c_float, _vp, _vp]),
+    "rrq_qk_scores_qjl": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _vp, _c_i64, _int, _int, _int,
+                                 _c_u64, _vp, ctypes.c_float, _vp, _vp]),
     "rrq_q4_0_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
     "rrq_q4_0_rot_decode": (_int, [_vp, _c_i64, _int, _c_u64, _int, _vp, _int, _vp]),
     "rrq_ggml_block_bytes": (_int, [_int]),
@@ -242,6 +244,38 @@ def rrq_qk_scores(q: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor, hkv
     cb = _HostFloats(codebook)
     _check(lib().rrq_qk_scores(_ptr(q), hq, _ptr(codes), _ptr(norms), t_len, hkv, d, bits, seed,
                                cb.ptr, float(scale), _ptr(out), _stream(q)), "rrq_qk_scores")
+    return out
+
+
+def rrq_qk_scores_qjl(q: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,
+                      qjl_bits: torch.Tensor, qjl_rnorm: torch.Tensor, qjl_S: torch.Tensor, hkv: int,
+                      d: int, bits: int, seed: int, codebook=None, scale: float = 1.0, out=None):
+    """Unbiased scores [hq, T] of unrotated fp16 queries q [hq, d] against keys stored as
+    b-bit codes + norms plus the QJL sign bits and residual norms (rows t*hkv + g), with
+    the projection qjl_S (bf16 [d, d]) they were encoded with."""
+    _dev_tensor(q, "q", (torch.float16,))
+    _dev_tensor(codes, "codes", (torch.uint8,))
+    _dev_tensor(norms, "norms", (torch.float32,))
+    _dev_tensor(qjl_bits, "qjl_bits", (torch.uint8,))
+    _dev_tensor(qjl_rnorm, "qjl_rnorm", (torch.float32,))
+    _dev_tensor(qjl_S, "qjl_S", (torch.bfloat16,))
+    hq = q.shape[0]
+    if q.shape != (hq, d) or qjl_S.shape != (d, d):
+        raise ValueError("q must be [hq, d] and qjl_S [d, d]")
+    rows = norms.numel()
+    if rows % hkv:
+        raise ValueError("norms must hold T*hkv values")
+    t_len = rows // hkv
+    if (codes.numel() != rows * (d * bits // 8) or qjl_bits.numel() != rows * (d // 8)
+            or qjl_rnorm.numel() != rows):
+        raise ValueError("codes / norms / qjl sizes disagree")
+    if out is None:
+        out = torch.empty(hq, t_len, dtype=torch.float32, device=q.device)
+    _dev_tensor(out, "out", (torch.float32,))
+    cb = _HostFloats(codebook)
+    _check(lib().rrq_qk_scores_qjl(_ptr(q), hq, _ptr(codes), _ptr(norms), _ptr(qjl_bits),
+                                   _ptr(qjl_rnorm), _ptr(qjl_S), t_len, hkv, d, bits, seed, cb.ptr,
+                                   float(scale), _ptr(out), _stream(q)), "rrq_qk_scores_qjl")
     return out
 
 

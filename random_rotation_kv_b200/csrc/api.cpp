@@ -9,6 +9,7 @@
 
 #include "rrq.h"
 #include "ggml_blocks.h"
+#include "scores_qjl.h"
 #include "rrq_params.h"
 
 namespace {
@@ -226,6 +227,38 @@ int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norm
   if (T == 0) return RRQ_OK;
   return status_of(rrq::launch_qk_scores(q, hq, codes, norms, T, hkv, d, p, scale, scores,
                                          as_stream(stream)));
+}
+
+int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* norms,
+                      const uint8_t* qjl_bits, const float* qjl_rnorm, const uint16_t* qjl_S,
+                      int64_t T, int hkv, int d, int bits, uint64_t seed, const float* codebook,
+                      float scale, float* scores, void* stream) {
+  if (T < 0 || !d_ok(d) || !bits_ok(bits) || hq < 1 || hkv < 1 || hq % hkv != 0 ||
+      !std::isfinite(scale))
+    return RRQ_ERR_INVALID;
+  if (q == nullptr || !aligned(q, 16) || qjl_S == nullptr || !aligned(qjl_S, 16))
+    return RRQ_ERR_INVALID;
+  if (!arr_ok(codes, T, 16) || !arr_ok(norms, T, 4) || !arr_ok(qjl_bits, T, 16) ||
+      !arr_ok(qjl_rnorm, T, 4) || !arr_ok(scores, T, 16))
+    return RRQ_ERR_INVALID;
+  const int group = hq / hkv;
+  if (d != 128 || (group != 1 && group != 2 && group != 4 && group != 8)) return RRQ_ERR_UNSUPPORTED;
+  rrq::QjlScoreArgs a;
+  if (make_params(bits, codebook, seed, d, &a.p) != RRQ_OK) return RRQ_ERR_INVALID;
+  if (T == 0) return RRQ_OK;
+  a.q = static_cast<const __half*>(q);
+  a.codes = codes;
+  a.norms = norms;
+  a.bits = qjl_bits;
+  a.rnorm = qjl_rnorm;
+  a.S = reinterpret_cast<const __nv_bfloat16*>(qjl_S);
+  a.scores = scores;
+  a.T = T;
+  a.hq = hq;
+  a.hkv = hkv;
+  a.group = group;
+  a.scale = scale;
+  return status_of(rrq::launch_qk_scores_qjl(a, as_stream(stream)));
 }
 
 int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate,
