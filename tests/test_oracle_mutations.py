@@ -211,3 +211,31 @@ def test_mutation_q5_0_scale_from_unsigned_max(monkeypatch):
 
     monkeypatch.setattr(ogg, "block_decisions", bad)
     assert _fails(pins.test_ggml_hand_worked_blocks)
+
+
+def test_mutation_attention_values_decoded_with_the_key_rotation(monkeypatch):
+    """v̂ decoded with the key seed instead of the value seed."""
+    import oracle.attention as oatt
+    good = oatt.decode_attention
+
+    def bad(q, kp, kn, vp, vn, t_len, hkv, d, kb, vb, ks, vs, *a, **kw):
+        return good(q, kp, kn, vp, vn, t_len, hkv, d, kb, vb, ks, ks, *a, **kw)
+
+    monkeypatch.setattr(oatt, "decode_attention", bad)
+    assert _fails(pins.test_attention_single_token_returns_its_value)
+
+
+def test_mutation_attention_softmax_over_heads(monkeypatch):
+    """The softmax normalised over the query heads instead of the tokens."""
+    import oracle.attention as oatt
+
+    def bad(q, kp, kn, vp, vn, t_len, hkv, d, kb, vb, ks, vs, kl=None, vl=None, scale=1.0):
+        q = np.asarray(q, np.float64)
+        s = orrq.scores(q, kp, kn, t_len, hkv, d, kb, ks, kl, scale)
+        w = np.exp(s - s.max(axis=0, keepdims=True))
+        p = w / w.sum(axis=0, keepdims=True)
+        v_hat = orrq.decode_exact(vp, vn, vb, d, vs, vl).reshape(t_len, hkv, d)
+        return np.stack([p[h] @ v_hat[:, orrq.kv_group(h, q.shape[0], hkv), :] for h in range(q.shape[0])])
+
+    monkeypatch.setattr(oatt, "decode_attention", bad)
+    assert _fails(pins.test_attention_zero_query_is_the_mean_value_and_order_free)

@@ -16,7 +16,7 @@ import pytest
 import scipy.linalg
 import scipy.stats
 
-from oracle import codebook, ggml_blocks, hadamard, q4_0, qjl, rng, rrq, sphere
+from oracle import attention, codebook, ggml_blocks, hadamard, q4_0, qjl, rng, rrq, sphere
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -625,3 +625,55 @@ def test_qjl_unbiased_scores_average_to_the_true_inner_product():
     assert np.allclose(sc - mse_only,
                        np.stack([0.5 * qjl.estimate_residual_dot(rrq.rotate(q, 7)[h], s, enc.bits.reshape(t_len, hkv, 2)[:, g[h]],
                                                                   enc.rnorm.reshape(t_len, hkv)[:, g[h]]) for h in range(hq)]))
+
+
+
+# ----------------------------------------------------- attention over a quantised cache
+def _att_cache(t_len, hkv, d, seed_k, seed_v, rg):
+    k = rg.standard_normal((t_len * hkv, d)) * 1.5
+    v = rg.standard_normal((t_len * hkv, d)) * 0.8
+    ek = rrq.encode(k, 4, seed_k)
+    ev = rrq.encode(v, 4, seed_v)
+    return ek, ev
+
+
+def test_attention_single_token_returns_its_value():
+    rg = np.random.default_rng(40)
+    d, hkv, hq = 32, 2, 4
+    ek, ev = _att_cache(1, hkv, d, 3, 5, rg)
+    q = rg.standard_normal((hq, d))
+    out = attention.decode_attention(q, ek.packed, ek.norms, ev.packed, ev.norms, 1, hkv, d, 4, 4, 3, 5)
+    v_hat = rrq.decode_exact(ev.packed, ev.norms, 4, d, 5)
+    for h in range(hq):
+        assert np.allclose(out[h], v_hat[h // 2], rtol=0, atol=1e-12)
+
+
+def test_attention_zero_query_is_the_mean_value_and_order_free():
+    rg = np.random.default_rng(41)
+    d, hkv, hq, t_len = 32, 2, 2, 7
+    ek, ev = _att_cache(t_len, hkv, d, 3, 5, rg)
+    out = attention.decode_attention(np.zeros((hq, d)), ek.packed, ek.norms, ev.packed, ev.norms,
+                                     t_len, hkv, d, 4, 4, 3, 5)
+    v_hat = rrq.decode_exact(ev.packed, ev.norms, 4, d, 5).reshape(t_len, hkv, d)
+    assert np.allclose(out[0], v_hat[:, 0].mean(axis=0), atol=1e-12)
+    assert np.allclose(out[1], v_hat[:, 1].mean(axis=0), atol=1e-12)
+    q = rg.standard_normal((hq, d))
+    perm = rg.permutation(t_len)
+    rows = (perm[:, None] * hkv + np.arange(hkv)[None, :]).ravel()
+    a = attention.decode_attention(q, ek.packed, ek.norms, ev.packed, ev.norms, t_len, hkv, d, 4, 4, 3, 5)
+    b = attention.decode_attention(q, ek.packed[rows], ek.norms[rows], ev.packed[rows], ev.norms[rows],
+                                   t_len, hkv, d, 4, 4, 3, 5)
+    assert np.allclose(a, b, atol=1e-12)
+
+
+def test_attention_large_scale_picks_the_top_scoring_token():
+    rg = np.random.default_rng(42)
+    d, hkv, hq, t_len = 32, 1, 1, 9
+    ek, ev = _att_cache(t_len, hkv, d, 3, 5, rg)
+    q = rg.standard_normal((hq, d))
+    s = rrq.scores(q, ek.packed, ek.norms, t_len, hkv, d, 4, 3)
+    top = int(np.argmax(s[0]))
+    out = attention.decode_attention(q, ek.packed, ek.norms, ev.packed, ev.norms, t_len, hkv, d, 4, 4,
+                                     3, 5, scale=1e4)
+    v_hat = rrq.decode_exact(ev.packed, ev.norms, 4, d, 5)
+    assert np.allclose(out[0], v_hat[top], atol=1e-9)
