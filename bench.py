@@ -465,6 +465,22 @@ def extra_kernels(torch, dev, flush, reps, peak):
                         "frac_of_hbm": by / ms / 1e6 / peak}
     del codes, norms, cs, ns, scs
 
+    # one decode step of attention over a 4-bit K/V cache of the same shape
+    kt = torch.from_numpy(w.flat()).to(dev)
+    kc, kn_ = B.rrq_encode(kt, 4, 42)
+    vc, vn_ = B.rrq_encode(kt, 4, 43)  # values: the same tensor under another rotation
+    del kt
+    caches = [(kc, kn_, vc, vn_), (kc.clone(), kn_.clone(), vc.clone(), vn_.clone())]  # 2 x 142 MB
+    ao = torch.empty(32, 128, dtype=torch.float32, device=dev)
+    ms = time_loop(torch, stream, lambda i: B.rrq_attention_decode(
+        q, *caches[i % 2], 8, 128, 42, 43, scale=128 ** -0.5, out=ao), reps)
+    by = nkh * (64 + 4) * 2 + 32 * 128 * 4
+    out["attention_decode"] = {"workload": "32 q heads over [131072 tokens x 8 kv heads] d=128, "
+                                           "4-bit K and V codes",
+                               "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
+                               "frac_of_hbm": by / ms / 1e6 / peak}
+    del caches, kc, kn_, vc, vn_
+
     # unbiased scores on the same keys stored TurboQuant-style: 2-bit codes + QJL bits
     S = B.rrq_qjl_matrix(4242, 128, device=dev)
     k = torch.from_numpy(w.flat()).to(dev)

@@ -231,6 +231,33 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
                       float scale, float* scores, void* stream);
 
 /*
+ * rrq_attention_decode — one decode step of attention over a quantised K/V cache.
+ * "Attn-rot (TurboQuant lite) in llama.cpp" page, "What kind of beast is
+ * Attn-rot" (keys and values both quantised after a rotation);
+ * "Random-rotation quantization" page, "Three decoders, one rotation" (the MSE
+ * decoder is the one for KV-cache compression).  With g = ⌊h·hkv/hq⌋:
+ *     s[h][t] = scale · <q_h, k̂_{t,g}>         (as rrq_qk_scores, K codebook and seed),
+ *     p[h][t] = exp(s[h][t] − max_t s[h][·]) / Σ_t exp(s[h][t] − max_t s[h][·]),
+ *     out[h]  = Σ_t p[h][t] · v̂_{t,g}          (v̂ as rrq_decode, V codebook and seed).
+ * The values are summed in their rotated domain and rotated back once per head.
+ *   q        [hq × d] fp16
+ *   k_codes  [T·hkv × d/2] bytes (4-bit), row t·hkv + g;  k_norms [T·hkv] float
+ *   v_codes  [T·hkv × d/2] bytes (4-bit);                 v_norms [T·hkv] float
+ *   k_codebook, v_codebook: HOST float[16] or NULL (the default codebook)
+ *   out      [hq × d] float (output)
+ * d must be 128 and both codes 4-bit; hq a multiple of hkv with hq/hkv in
+ * {1, 2, 4, 8}; T ≥ 1.  Scores in fp16 pairs with fp32 partial sums (as
+ * rrq_qk_scores); softmax and the value sums in fp32.
+ * Errors: RRQ_ERR_INVALID, RRQ_ERR_UNSUPPORTED (d, bits, group size),
+ * RRQ_ERR_CUDA.
+ */
+int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
+                         const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,
+                         int k_bits, uint64_t k_seed, const float* k_codebook, int v_bits,
+                         uint64_t v_seed, const float* v_codebook, float scale, float* out,
+                         void* stream);
+
+/*
  * rrq_q4_0_rot — "Attn-rot" (TurboQuant lite): rotate, then q4_0.
  * "Attn-rot (TurboQuant lite) in llama.cpp" page: rotate K/V before an
  * ordinary block format, q4_0 first of all.  With y = Πx (rotate = 1) or

@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     LIB_PATH,
     RRQError,
     lib,
+    rrq_attention_decode,
     rrq_codebook,
     rrq_decode,
     rrq_drive_encode,

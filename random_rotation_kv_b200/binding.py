@@ -42,6 +42,8 @@ SIGNATURES = {
                              ctypes.c_float, _vp, _vp]),
     "rrq_qk_scores_qjl": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _vp, _c_i64, _int, _int, _int,
                                  _c_u64, _vp, ctypes.c_float, _vp, _vp]),
+    "rrq_attention_decode": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _c_i64, _int, _int, _int,
+                                    _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float, _vp, _vp]),
     "rrq_q4_0_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
     "rrq_q4_0_rot_decode": (_int, [_vp, _c_i64, _int, _c_u64, _int, _vp, _int, _vp]),
     "rrq_ggml_block_bytes": (_int, [_int]),
@@ -276,6 +278,37 @@ def rrq_qk_scores_qjl(q: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,
     _check(lib().rrq_qk_scores_qjl(_ptr(q), hq, _ptr(codes), _ptr(norms), _ptr(qjl_bits),
                                    _ptr(qjl_rnorm), _ptr(qjl_S), t_len, hkv, d, bits, seed, cb.ptr,
                                    float(scale), _ptr(out), _stream(q)), "rrq_qk_scores_qjl")
+    return out
+
+
+def rrq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.Tensor,
+                         v_codes: torch.Tensor, v_norms: torch.Tensor, hkv: int, d: int,
+                         k_seed: int, v_seed: int, k_bits: int = 4, v_bits: int = 4,
+                         k_codebook=None, v_codebook=None, scale: float = 1.0, out=None):
+    """One decode step of attention, out [hq, d] float32, of unrotated fp16 queries q [hq, d]
+    over a K/V cache of 4-bit codes + norms (rows t*hkv + g)."""
+    _dev_tensor(q, "q", (torch.float16,))
+    for t_, nm in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        _dev_tensor(t_, nm, (torch.uint8,))
+    for t_, nm in ((k_norms, "k_norms"), (v_norms, "v_norms")):
+        _dev_tensor(t_, nm, (torch.float32,))
+    hq = q.shape[0]
+    if q.shape != (hq, d):
+        raise ValueError("q must be [hq, d]")
+    rows = k_norms.numel()
+    if rows % hkv or v_norms.numel() != rows:
+        raise ValueError("norms must hold T*hkv values")
+    t_len = rows // hkv
+    if k_codes.numel() != rows * (d * k_bits // 8) or v_codes.numel() != rows * (d * v_bits // 8):
+        raise ValueError("codes / norms sizes disagree")
+    if out is None:
+        out = torch.empty(hq, d, dtype=torch.float32, device=q.device)
+    _dev_tensor(out, "out", (torch.float32,))
+    kc, vc = _HostFloats(k_codebook), _HostFloats(v_codebook)
+    _check(lib().rrq_attention_decode(_ptr(q), hq, _ptr(k_codes), _ptr(k_norms), _ptr(v_codes),
+                                      _ptr(v_norms), t_len, hkv, d, k_bits, k_seed, kc.ptr, v_bits,
+                                      v_seed, vc.ptr, float(scale), _ptr(out), _stream(q)),
+           "rrq_attention_decode")
     return out
 
 

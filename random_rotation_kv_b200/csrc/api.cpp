@@ -8,6 +8,7 @@
 #include <cstring>
 
 #include "rrq.h"
+#include "attention.h"
 #include "ggml_blocks.h"
 #include "scores_qjl.h"
 #include "rrq_params.h"
@@ -259,6 +260,40 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
   a.group = group;
   a.scale = scale;
   return status_of(rrq::launch_qk_scores_qjl(a, as_stream(stream)));
+}
+
+int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
+                         const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,
+                         int k_bits, uint64_t k_seed, const float* k_codebook, int v_bits,
+                         uint64_t v_seed, const float* v_codebook, float scale, float* out,
+                         void* stream) {
+  if (T < 1 || !d_ok(d) || !bits_ok(k_bits) || !bits_ok(v_bits) || hq < 1 || hkv < 1 ||
+      hq % hkv != 0 || !std::isfinite(scale))
+    return RRQ_ERR_INVALID;
+  if (q == nullptr || !aligned(q, 16) || out == nullptr || !aligned(out, 16)) return RRQ_ERR_INVALID;
+  if (!arr_ok(k_codes, T, 16) || !arr_ok(k_norms, T, 4) || !arr_ok(v_codes, T, 16) ||
+      !arr_ok(v_norms, T, 4))
+    return RRQ_ERR_INVALID;
+  const int group = hq / hkv;
+  if (d != 128 || k_bits != 4 || v_bits != 4 ||
+      (group != 1 && group != 2 && group != 4 && group != 8))
+    return RRQ_ERR_UNSUPPORTED;
+  rrq::AttnArgs a;
+  if (make_params(k_bits, k_codebook, k_seed, d, &a.pk) != RRQ_OK ||
+      make_params(v_bits, v_codebook, v_seed, d, &a.pv) != RRQ_OK)
+    return RRQ_ERR_INVALID;
+  a.q = static_cast<const __half*>(q);
+  a.k_codes = k_codes;
+  a.k_norms = k_norms;
+  a.v_codes = v_codes;
+  a.v_norms = v_norms;
+  a.out = out;
+  a.T = T;
+  a.hq = hq;
+  a.hkv = hkv;
+  a.group = group;
+  a.scale = scale;
+  return status_of(rrq::launch_attention_decode(a, as_stream(stream)));
 }
 
 int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate,
