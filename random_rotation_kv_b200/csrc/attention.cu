@@ -13,20 +13,25 @@
 //
 // Work split.  A cluster of C CTAs serves one kv head g and its GQA group of G
 // query heads; its warps take tiles of 32 consecutive tokens.  Per tile:
-//  A. one token per lane: the lane loads its K and V rows (64 B each, the next
-//     tile's while this one computes), scores the G heads with packed fp16 FMAs
-//     on a lane-replicated table of level pairs (as the score kernel), and the
-//     warp updates its running softmax state (max, sum) per head; the lane
-//     writes its V row and its weights w_h = p_h·ν^V/√d to the warp's buffer.
-//  B. four coordinates per lane: for each token of the tile the lane reads two
-//     V code bytes, looks each up in a lane-replicated table of fp32 level pairs
-//     and accumulates w_h times them into its fp32 partial sums (packed FMAs).
-// At the end the warps' states merge within the CTA, and the CTAs' within the
-// cluster through distributed shared memory: rank 0 reads every CTA's partial
-// sums, normalises, applies Πᵀ (a 128-point transform per head) and writes out.
+//  A. one token per lane: the lane loads its K row (64 B), scores the G heads
+//     with packed fp16 FMAs on a lane-replicated table of level pairs (as the
+//     score kernel), and the warp updates its running softmax state (max, sum)
+//     per head; the lane writes its weights w_h = p_h·ν^V/√d to the warp buffer.
+//  B. four coordinates per lane: the warp reads the tile's V rows (two bytes
+//     per lane per token, 64 contiguous bytes per token, all 32 loads in flight
+//     at once), looks each byte up in a table of fp32 level pairs (16 copies,
+//     one per lane of a half-warp) and accumulates w_h times them into fp32
+//     partial sums (packed FMAs).
+// At the end the warps' states merge within the CTA (shared-memory atomics after
+// a common rescaling), and the CTAs' within the cluster through distributed
+// shared memory: rank 0 reads every CTA's partial sums, normalises, applies Πᵀ
+// (a 128-point transform per head) and writes out.  16 warps and under 96 KB of
+// shared memory per CTA, so that 16-CTA clusters of every kv head are resident
+// together.
 #include <cooperative_groups.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "attention.h"
 #include "rrq_device.cuh"
@@ -38,48 +43,39 @@ namespace {
 
 constexpr int kAD = 128;
 constexpr int kAP = kAD / 2;
-constexpr int kAWarps = 8;
+constexpr int kAWarps = 16;
 constexpr int kAThreads = kAWarps * 32;
-constexpr int kVRow = 80;  // shared V row stride (64 code bytes, padded: conflict-free 16-byte stores)
 
 template <int G> struct ALayout {
   static constexpr int KTAB = 0;                               // [256][32] half2 (K level pairs)
-  static constexpr int VTAB = KTAB + 256 * 32 * 4;             // [256][32] float2 (V level pairs)
-  static constexpr int QH = VTAB + 256 * 32 * 8;               // [kAP][G] half2 q''
+  static constexpr int VTAB = KTAB + 256 * 32 * 4;             // [256][16] float2 (V level pairs)
+  static constexpr int QH = VTAB + 256 * 16 * 8;               // [kAP][G] half2 q''
   static constexpr int INV = QH + kAP * G * 4;                 // [G] 1/s
-  static constexpr int WARP = (INV + G * 4 + 15) / 16 * 16;    // per-warp buffers
-  static constexpr int VBUF = 32 * kVRow;                      // V rows of the tile
-  static constexpr int WBUF = 32 * G * 4;                      // weights [32][G]
-  static constexpr int WARP_BYTES = VBUF + WBUF;
+  static constexpr int WBUF = (INV + G * 4 + 15) / 16 * 16;    // per warp: weights [32][G]
+  static constexpr int WM = WBUF + kAWarps * 32 * G * 4;       // [kAWarps][G] warp maxima
   static constexpr int PART_FLOATS = 2 * G + G * kAD;         // [G] m, [G] l, [G][kAD] o
-  static constexpr int PART = WARP + kAWarps * WARP_BYTES;     // the CTA's partial state
+  static constexpr int PART = WM + kAWarps * G * 4;            // the CTA's partial state
   static constexpr int FIN = PART + PART_FLOATS * 4;           // rank 0: [G][kAD] sums, [G] denominators
   static constexpr int TOTAL = FIN + G * (kAD + 1) * 4;
-  // the warps' partial states, merged after the token loop, alias the level tables
-  static constexpr int WPART = 0;
-  static_assert(kAWarps * PART_FLOATS * 4 <= QH, "warp partials fit over the tables");
+  static_assert(TOTAL <= 96 * 1024, "two CTAs per SM, so 16-CTA clusters of 8 kv heads fit");
 };
 
-struct Row {
-  uint4 k[4], v[4];
+struct KRow {
+  uint4 k[4];
   float kn, vn;
 };
 
-__device__ __forceinline__ void load_rows(Row& r, const AttnArgs& a, int64_t t, int g) {
+__device__ __forceinline__ void load_krow(KRow& r, const AttnArgs& a, int64_t t, int g) {
   if (t < a.T) {
     const int64_t n = t * a.hkv + g;
     const uint4* kp = reinterpret_cast<const uint4*>(a.k_codes + n * 64);
-    const uint4* vp = reinterpret_cast<const uint4*>(a.v_codes + n * 64);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      r.k[i] = __ldcs(kp + i);
-      r.v[i] = __ldcs(vp + i);
-    }
+    for (int i = 0; i < 4; ++i) r.k[i] = __ldcs(kp + i);
     r.kn = __ldcs(a.k_norms + n);
     r.vn = __ldcs(a.v_norms + n);
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) r.k[i] = r.v[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < 4; ++i) r.k[i] = make_uint4(0u, 0u, 0u, 0u);
     r.kn = r.vn = 0.f;
   }
 }
@@ -118,17 +114,20 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   cg::cluster_group cluster = cg::this_cluster();
   const int C = int(cluster.num_blocks()), rank = int(cluster.block_rank());
   const int g = blockIdx.x / C;
-  uint8_t* wbase = smem + L::WARP + warp * L::WARP_BYTES;
-  uint8_t* vbuf = wbase;
-  float* wbuf = reinterpret_cast<float*>(wbase + L::VBUF);
+  float* wbuf = reinterpret_cast<float*>(smem + L::WBUF) + warp * 32 * G;
+  float* wmax = reinterpret_cast<float*>(smem + L::WM);
 
   // ---- level tables from the parameters alone
   for (int i = tid; i < 256 * 32; i += kAThreads) {
     const int e = i >> 5;
     const __half2 kv = __floats2half2_rn(a.pk.levels[e & 15], a.pk.levels[e >> 4]);
     ktab[i] = *reinterpret_cast<const uint32_t*>(&kv);
-    vtab[i] = make_float2(a.pv.levels[e & 15], a.pv.levels[e >> 4]);
   }
+  // 16 copies suffice for the fp32 pairs: a 64-bit shared load serves each half-warp
+  // in its own pass, so lanes l and l + 16 never meet in one
+  for (int i = tid; i < 256 * 16; i += kAThreads)
+    vtab[i] = make_float2(a.pv.levels[(i >> 4) & 15], a.pv.levels[i >> 8]);
+  for (int i = tid; i < L::PART_FLOATS; i += kAThreads) part[i] = 0.f;
   pdl_wait();  // from here on, global memory
 
   // ---- q' = H·D_K·q for the group's heads, scaled per head to |q''| ≤ 1
@@ -163,7 +162,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   const float kscale = a.scale * a.pk.inv_d;
   const float vscale = a.pv.inv_sqrt_d;
   const uint32_t* ktab_l = ktab + lane;
-  const float2* vtab_l = vtab + lane;
+  const float2* vtab_l = vtab + (lane & 15);
   float m_run[G], l_run[G];
   float2 o[G][2];  // coordinates 4·lane .. 4·lane+3 of each head's rotated-domain sum
 #pragma unroll
@@ -172,11 +171,19 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
     l_run[j] = 0.f;
     o[j][0] = o[j][1] = make_float2(0.f, 0.f);
   }
-  Row cur, nxt;
-  load_rows(cur, a, tile * 32 + lane, g);
   for (; tile < ntile; tile += stride) {
     const int64_t t = tile * 32 + lane;
-    load_rows(nxt, a, t + stride * 32, g);
+    KRow cur;
+    load_krow(cur, a, t, g);
+    // the tile's V code bytes for this lane's four coordinates, all in flight now
+    uint32_t vb[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int64_t tu = tile * 32 + u;
+      vb[u] = tu < a.T ? uint32_t(__ldcs(reinterpret_cast<const uint16_t*>(
+                             a.v_codes + (tu * a.hkv + g) * 64) + lane))
+                       : 0u;
+    }
     // A. scores of this lane's token
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur.k);
     float sc[G];
@@ -221,18 +228,15 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
       wbuf[lane * G + j] = pj * cur.vn * vscale;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(vbuf + lane * kVRow)[i] = cur.v[i];
-#pragma unroll
     for (int j = 0; j < G; ++j) {
       o[j][0] = make_float2(o[j][0].x * alpha[j], o[j][0].y * alpha[j]);
       o[j][1] = make_float2(o[j][1].x * alpha[j], o[j][1].y * alpha[j]);
     }
     __syncwarp();
     // B. weighted sum of the tile's V rows, four coordinates per lane
-#pragma unroll 4
+#pragma unroll
     for (int u = 0; u < 32; ++u) {
-      const uint32_t two = *reinterpret_cast<const uint16_t*>(vbuf + u * kVRow + 2 * lane);
-      const float2 c0 = vtab_l[(two & 255u) << 5], c1 = vtab_l[(two >> 8) << 5];
+      const float2 c0 = vtab_l[(vb[u] & 255u) << 4], c1 = vtab_l[(vb[u] >> 8) << 4];
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const float w = wbuf[u * G + j];
@@ -241,39 +245,29 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
       }
     }
     __syncwarp();
-    cur = nxt;
   }
 
-  // ---- merge the warps' states (the level tables are free now), then the CTAs'
-  __syncthreads();
-  float* wp = reinterpret_cast<float*>(smem + L::WPART) + warp * L::PART_FLOATS;
+  // ---- merge the warps' states: CTA maximum per head, then rescaled sums by
+  // shared-memory atomics; then the CTAs' states across the cluster
+  if (lane == 0) {
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    if (lane == 0) {
-      wp[j] = m_run[j];
-      wp[G + j] = l_run[j];
-    }
-    float* oj = wp + 2 * G + j * kAD + 4 * lane;
-    oj[0] = o[j][0].x;
-    oj[1] = o[j][0].y;
-    oj[2] = o[j][1].x;
-    oj[3] = o[j][1].y;
+    for (int jj = 0; jj < G; ++jj) wmax[warp * G + jj] = m_run[jj];
   }
   __syncthreads();
-  const float* wall = reinterpret_cast<const float*>(smem + L::WPART);
-  for (int idx = tid; idx < G * (kAD + 2); idx += kAThreads) {
-    const int j = idx / (kAD + 2), c = idx % (kAD + 2);
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
     float mx = -INFINITY;
-    for (int w = 0; w < kAWarps; ++w) mx = fmaxf(mx, wall[w * L::PART_FLOATS + j]);
-    float acc = 0.f;
-    for (int w = 0; w < kAWarps; ++w) {
-      const float* wpw = wall + w * L::PART_FLOATS;
-      const float f = mx == -INFINITY ? 0.f : __expf(wpw[j] - mx);
-      acc += f * (c < kAD ? wpw[2 * G + j * kAD + c] : (c == kAD ? wpw[G + j] : 0.f));
+    for (int w = 0; w < kAWarps; ++w) mx = fmaxf(mx, wmax[w * G + j]);
+    const float f = m_run[j] == -INFINITY ? 0.f : __expf(m_run[j] - mx);
+    float* oj = part + 2 * G + j * kAD + 4 * lane;
+    if (f > 0.f) {
+      atomicAdd(oj, f * o[j][0].x);
+      atomicAdd(oj + 1, f * o[j][0].y);
+      atomicAdd(oj + 2, f * o[j][1].x);
+      atomicAdd(oj + 3, f * o[j][1].y);
+      if (lane == 0) atomicAdd(part + G + j, f * l_run[j]);
     }
-    if (c < kAD) part[2 * G + j * kAD + c] = acc;
-    else if (c == kAD) part[G + j] = acc;
-    else part[j] = mx;
+    if (tid == 0) part[j] = mx;
   }
   cluster.sync();
   if (rank == 0) {
@@ -311,6 +305,31 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   }
 }
 
+// Cluster sizes found for (group size, device, hkv), a fixed table (no heap
+// memory); 0 = not yet known.  When the table is full a choice is simply
+// searched again on the next call.
+struct ClusterChoice {
+  int g, dev, hkv, c;
+};
+constexpr int kClusterChoices = 64;
+std::mutex g_cluster_mu;
+ClusterChoice g_cluster_choices[kClusterChoices];
+int g_cluster_count = 0;
+
+int cached_cluster_size(int g, int dev, int hkv) {
+  std::lock_guard<std::mutex> lock(g_cluster_mu);
+  for (int i = 0; i < g_cluster_count; ++i) {
+    const ClusterChoice& c = g_cluster_choices[i];
+    if (c.g == g && c.dev == dev && c.hkv == hkv) return c.c;
+  }
+  return 0;
+}
+
+void remember_cluster_size(int g, int dev, int hkv, int c) {
+  std::lock_guard<std::mutex> lock(g_cluster_mu);
+  if (g_cluster_count < kClusterChoices) g_cluster_choices[g_cluster_count++] = {g, dev, hkv, c};
+}
+
 template <int G>
 cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   auto k = attention_decode_kernel<G>;
@@ -321,30 +340,51 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
-  // cluster size: 16 CTAs per kv head when that many fit side by side, else 8, 4, ...
-  const int64_t ntile = (a.T + 31) / 32;
-  int C = 16;
-  while (C > 1 && int64_t(C / 2) * kAWarps >= ntile) C /= 2;  // no idle CTAs on short caches
+  // cluster size: the largest C ≤ 16 for which the clusters of every kv head can
+  // be resident together (one wave), found once per (device, hkv) by occupancy
+  // queries, and no larger than the cache needs
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int cmax = cached_cluster_size(G, dev, a.hkv);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
-  for (; C >= 1; C /= 2) {
-    cfg.gridDim = dim3(unsigned(a.hkv * C));
+  auto configure = [&](int c) {
+    cfg.gridDim = dim3(unsigned(a.hkv * c));
     cfg.blockDim = dim3(kAThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(C);
+    attr[0].val.clusterDim.x = unsigned(c);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(k), &cfg) == cudaSuccess &&
-        clusters > 0)
-      break;
-    (void)cudaGetLastError();
+  };
+  if (cmax == 0) {
+    int fallback = 0;
+    for (int c = 16; c >= 1; --c) {
+      configure(c);
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(k), &cfg) !=
+          cudaSuccess) {
+        (void)cudaGetLastError();
+        continue;
+      }
+      if (fallback == 0 && clusters > 0) fallback = c;  // the largest that runs at all
+      if (clusters >= a.hkv) {                            // every kv head at once
+        cmax = c;
+        break;
+      }
+    }
+    if (cmax == 0) cmax = fallback;
+    if (cmax == 0) return cudaErrorInvalidConfiguration;
+    remember_cluster_size(G, dev, a.hkv, cmax);
   }
-  if (C < 1) return cudaErrorInvalidConfiguration;
+  const int64_t ntile = (a.T + 31) / 32;
+  int C = cmax;
+  while (C > 1 && int64_t(C - 1) * kAWarps >= ntile) --C;  // no idle CTAs on short caches
+  configure(C);
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.numAttrs = 2;
