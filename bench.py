@@ -233,7 +233,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": workload_config({"sample_vectors_per_step": n_sample}),
+        "config": workload_config({"sample_vectors_per_step": n_sample,
+                                   "l2": "n/a (the CPU oracle on the host cores)"}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"first {n_sample} workload vectors per step, encode+decode"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -472,8 +473,10 @@ def extra_kernels(torch, dev, flush, reps, peak):
     del kt
     caches = [(kc, kn_, vc, vn_), (kc.clone(), kn_.clone(), vc.clone(), vn_.clone())]  # 2 x 142 MB
     ao = torch.empty(32, 128, dtype=torch.float32, device=dev)
+    ws = torch.zeros(B.rrq_attention_workspace_bytes(32, 8, 128, w.x.shape[0]), dtype=torch.uint8,
+                     device=dev)
     ms = time_loop(torch, stream, lambda i: B.rrq_attention_decode(
-        q, *caches[i % 2], 8, 128, 42, 43, scale=128 ** -0.5, out=ao), reps)
+        q, *caches[i % 2], 8, 128, 42, 43, scale=128 ** -0.5, out=ao, workspace=ws), reps)
     by = nkh * (64 + 4) * 2 + 32 * 128 * 4
     out["attention_decode"] = {"workload": "32 q heads over [131072 tokens x 8 kv heads] d=128, "
                                            "4-bit K and V codes",

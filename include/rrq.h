@@ -240,22 +240,33 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
  *     p[h][t] = exp(s[h][t] − max_t s[h][·]) / Σ_t exp(s[h][t] − max_t s[h][·]),
  *     out[h]  = Σ_t p[h][t] · v̂_{t,g}          (v̂ as rrq_decode, V codebook and seed).
  * The values are summed in their rotated domain and rotated back once per head.
- *   q        [hq × d] fp16
- *   k_codes  [T·hkv × d/2] bytes (4-bit), row t·hkv + g;  k_norms [T·hkv] float
- *   v_codes  [T·hkv × d/2] bytes (4-bit);                 v_norms [T·hkv] float
+ *   q          [hq × d] fp16
+ *   k_codes    [T·hkv × d/2] bytes (4-bit), row t·hkv + g;  k_norms [T·hkv] float
+ *   v_codes    [T·hkv × d/2] bytes (4-bit);                 v_norms [T·hkv] float
  *   k_codebook, v_codebook: HOST float[16] or NULL (the default codebook)
- *   out      [hq × d] float (output)
+ *   workspace  device scratch of workspace_bytes ≥ rrq_attention_workspace_bytes(
+ *              hq, hkv, d, T), 256-byte aligned, owned by the caller, and ZERO before
+ *              its first use: each call leaves its counters at zero again.  Calls
+ *              that share a workspace must not overlap on the GPU.
+ *   out        [hq × d] float (output)
  * d must be 128 and both codes 4-bit; hq a multiple of hkv with hq/hkv in
  * {1, 2, 4, 8}; T ≥ 1.  Scores in fp16 pairs with fp32 partial sums (as
  * rrq_qk_scores); softmax and the value sums in fp32.
- * Errors: RRQ_ERR_INVALID, RRQ_ERR_UNSUPPORTED (d, bits, group size),
- * RRQ_ERR_CUDA.
+ * Errors: RRQ_ERR_INVALID (incl. a workspace that is too small), RRQ_ERR_UNSUPPORTED
+ * (d, bits, group size), RRQ_ERR_CUDA.
  */
 int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
                          const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,
                          int k_bits, uint64_t k_seed, const float* k_codebook, int v_bits,
-                         uint64_t v_seed, const float* v_codebook, float scale, float* out,
-                         void* stream);
+                         uint64_t v_seed, const float* v_codebook, float scale, void* workspace,
+                         size_t workspace_bytes, float* out, void* stream);
+
+/*
+ * rrq_attention_workspace_bytes — the workspace rrq_attention_decode needs for
+ * (hq, hkv, d, T) on the current device (it depends on the SM count), or 0 for an
+ * invalid shape.  No CUDA work beyond reading the device's attributes.
+ */
+size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int64_t T);
 
 /*
  * rrq_q4_0_rot — "Attn-rot" (TurboQuant lite): rotate, then q4_0.

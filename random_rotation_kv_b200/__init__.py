@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     RRQError,
     lib,
     rrq_attention_decode,
+    rrq_attention_workspace_bytes,
     rrq_codebook,
     rrq_decode,
     rrq_drive_encode,

@@ -43,7 +43,9 @@ SIGNATURES = {
     "rrq_qk_scores_qjl": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _vp, _c_i64, _int, _int, _int,
                                  _c_u64, _vp, ctypes.c_float, _vp, _vp]),
     "rrq_attention_decode": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _c_i64, _int, _int, _int,
-                                    _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float, _vp, _vp]),
+                                    _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float, _vp,
+                                    ctypes.c_size_t, _vp, _vp]),
+    "rrq_attention_workspace_bytes": (ctypes.c_size_t, [_int, _int, _int, _c_i64]),
     "rrq_q4_0_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
     "rrq_q4_0_rot_decode": (_int, [_vp, _c_i64, _int, _c_u64, _int, _vp, _int, _vp]),
     "rrq_ggml_block_bytes": (_int, [_int]),
@@ -284,9 +286,14 @@ def rrq_qk_scores_qjl(q: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,
 def rrq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.Tensor,
                          v_codes: torch.Tensor, v_norms: torch.Tensor, hkv: int, d: int,
                          k_seed: int, v_seed: int, k_bits: int = 4, v_bits: int = 4,
-                         k_codebook=None, v_codebook=None, scale: float = 1.0, out=None):
+                         k_codebook=None, v_codebook=None, scale: float = 1.0, out=None,
+                         workspace=None):
     """One decode step of attention, out [hq, d] float32, of unrotated fp16 queries q [hq, d]
-    over a K/V cache of 4-bit codes + norms (rows t*hkv + g)."""
+    over a K/V cache of 4-bit codes + norms (rows t*hkv + g).
+
+    ``workspace``: a uint8 device tensor of at least rrq_attention_workspace_bytes(...)
+    bytes, zero before its first use (each call leaves it ready for the next); a zeroed
+    one is allocated when none is given."""
     _dev_tensor(q, "q", (torch.float16,))
     for t_, nm in ((k_codes, "k_codes"), (v_codes, "v_codes")):
         _dev_tensor(t_, nm, (torch.uint8,))
@@ -304,12 +311,22 @@ def rrq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.
     if out is None:
         out = torch.empty(hq, d, dtype=torch.float32, device=q.device)
     _dev_tensor(out, "out", (torch.float32,))
+    need = rrq_attention_workspace_bytes(hq, hkv, d, t_len)
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    _dev_tensor(workspace, "workspace", (torch.uint8,))
     kc, vc = _HostFloats(k_codebook), _HostFloats(v_codebook)
     _check(lib().rrq_attention_decode(_ptr(q), hq, _ptr(k_codes), _ptr(k_norms), _ptr(v_codes),
                                       _ptr(v_norms), t_len, hkv, d, k_bits, k_seed, kc.ptr, v_bits,
-                                      v_seed, vc.ptr, float(scale), _ptr(out), _stream(q)),
+                                      v_seed, vc.ptr, float(scale), _ptr(workspace),
+                                      workspace.numel(), _ptr(out), _stream(q)),
            "rrq_attention_decode")
     return out
+
+
+def rrq_attention_workspace_bytes(hq: int, hkv: int, d: int, t_len: int) -> int:
+    """Workspace bytes rrq_attention_decode needs on the current device."""
+    return int(lib().rrq_attention_workspace_bytes(hq, hkv, d, t_len))
 
 
 def rrq_q4_0_rot(x: torch.Tensor, seed: int, rotate: bool = True, out=None):

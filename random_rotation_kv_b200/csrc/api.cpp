@@ -262,11 +262,16 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
   return status_of(rrq::launch_qk_scores_qjl(a, as_stream(stream)));
 }
 
+size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int64_t T) {
+  if (T < 1 || !d_ok(d) || hq < 1 || hkv < 1 || hq % hkv != 0) return 0;
+  return rrq::attention_workspace_bytes(hq, hkv, T);
+}
+
 int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
                          const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,
                          int k_bits, uint64_t k_seed, const float* k_codebook, int v_bits,
-                         uint64_t v_seed, const float* v_codebook, float scale, float* out,
-                         void* stream) {
+                         uint64_t v_seed, const float* v_codebook, float scale, void* workspace,
+                         size_t workspace_bytes, float* out, void* stream) {
   if (T < 1 || !d_ok(d) || !bits_ok(k_bits) || !bits_ok(v_bits) || hq < 1 || hkv < 1 ||
       hq % hkv != 0 || !std::isfinite(scale))
     return RRQ_ERR_INVALID;
@@ -278,6 +283,9 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
   if (d != 128 || k_bits != 4 || v_bits != 4 ||
       (group != 1 && group != 2 && group != 4 && group != 8))
     return RRQ_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned(workspace, 256) ||
+      workspace_bytes < rrq::attention_workspace_bytes(hq, hkv, T))
+    return RRQ_ERR_INVALID;
   rrq::AttnArgs a;
   if (make_params(k_bits, k_codebook, k_seed, d, &a.pk) != RRQ_OK ||
       make_params(v_bits, v_codebook, v_seed, d, &a.pv) != RRQ_OK)
@@ -292,7 +300,11 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
   a.hq = hq;
   a.hkv = hkv;
   a.group = group;
+  a.splits = rrq::attention_splits(hkv, group, T);
   a.scale = scale;
+  a.counters = static_cast<unsigned*>(workspace);
+  a.states = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                      (size_t(hkv) * 4 + 255) / 256 * 256);
   return status_of(rrq::launch_attention_decode(a, as_stream(stream)));
 }
 

@@ -11,8 +11,9 @@
 //     out[h] = Σ_t p[h,t]·v̂_{t,g} = Πᵀ_V ( Σ_t p[h,t]·(ν^V_{t,g}/√d)·c_V[code^V_{t,g}] ),
 // so the values are summed in their rotated domain and rotated back once per head.
 //
-// Work split.  A cluster of C CTAs serves one kv head g and its GQA group of G
-// query heads; its warps take tiles of 32 consecutive tokens.  Per tile:
+// Work split.  The cache of kv head g is cut into S token ranges, one CTA each
+// (grid hkv × S, about two CTAs per SM); a CTA serves the GQA group of G query
+// heads of its kv head, and its warps take tiles of 32 consecutive tokens:
 //  A. one token per lane: the lane loads its K row (64 B), scores the G heads
 //     with packed fp16 FMAs on a lane-replicated table of level pairs (as the
 //     score kernel), and the warp updates its running softmax state (max, sum)
@@ -22,28 +23,23 @@
 //     at once), looks each byte up in a table of fp32 level pairs (16 copies,
 //     one per lane of a half-warp) and accumulates w_h times them into fp32
 //     partial sums (packed FMAs).
-// At the end the warps' states merge within the CTA (shared-memory atomics after
-// a common rescaling), and the CTAs' within the cluster through distributed
-// shared memory: rank 0 reads every CTA's partial sums, normalises, applies Πᵀ
-// (a 128-point transform per head) and writes out.  16 warps and under 96 KB of
-// shared memory per CTA, so that 16-CTA clusters of every kv head are resident
-// together.
-#include <cooperative_groups.h>
-
+// The warps' states merge within the CTA (shared-memory atomics after a common
+// rescaling); each CTA writes its state (max, sum, G×128 partial sums) to the
+// caller's workspace and counts itself in its kv head's counter there.  The
+// last CTA of a kv head merges the S states, applies Πᵀ (a 128-point transform
+// per head), writes the output and sets the counter back to zero.  No CTA waits
+// for another.
 #include <cmath>
-#include <mutex>
 
 #include "attention.h"
 #include "rrq_device.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace rrq {
 namespace {
 
 constexpr int kAD = 128;
 constexpr int kAP = kAD / 2;
-constexpr int kAWarps = 16;
+constexpr int kAWarps = 8;
 constexpr int kAThreads = kAWarps * 32;
 
 template <int G> struct ALayout {
@@ -55,9 +51,11 @@ template <int G> struct ALayout {
   static constexpr int WM = WBUF + kAWarps * 32 * G * 4;       // [kAWarps][G] warp maxima
   static constexpr int PART_FLOATS = 2 * G + G * kAD;         // [G] m, [G] l, [G][kAD] o
   static constexpr int PART = WM + kAWarps * G * 4;            // the CTA's partial state
-  static constexpr int FIN = PART + PART_FLOATS * 4;           // rank 0: [G][kAD] sums, [G] denominators
-  static constexpr int TOTAL = FIN + G * (kAD + 1) * 4;
-  static_assert(TOTAL <= 96 * 1024, "two CTAs per SM, so 16-CTA clusters of 8 kv heads fit");
+  static constexpr int FLAG = PART + PART_FLOATS * 4;          // "this CTA merges its kv head"
+  static constexpr int TOTAL = FLAG + 16;
+  static constexpr int FIN = KTAB;  // the last CTA's merged sums reuse the level tables
+  static_assert(G * (kAD + 1) * 4 <= VTAB, "merged sums fit over the K table");
+  static_assert(TOTAL <= 110 * 1024, "two CTAs per SM");
 };
 
 struct KRow {
@@ -99,8 +97,11 @@ __device__ __forceinline__ void fwht128(float (&v)[4], int lane) {
   }
 }
 
+// Two CTAs per SM (≤ 128 registers) where the group's accumulators allow it.
+template <int G> constexpr int attention_min_blocks() { return G <= 4 ? 2 : 1; }
+
 template <int G>
-__global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAThreads, attention_min_blocks<G>()) attention_decode_kernel(const AttnArgs a) {
   pdl_release();
   using L = ALayout<G>;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -110,10 +111,10 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   float* inv_s = reinterpret_cast<float*>(smem + L::INV);
   float* part = reinterpret_cast<float*>(smem + L::PART);
   float* fin = reinterpret_cast<float*>(smem + L::FIN);
+  int* last_flag = reinterpret_cast<int*>(smem + L::FLAG);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = int(cluster.num_blocks()), rank = int(cluster.block_rank());
-  const int g = blockIdx.x / C;
+  const int S = a.splits;
+  const int g = blockIdx.x / S, sidx = blockIdx.x % S;
   float* wbuf = reinterpret_cast<float*>(smem + L::WBUF) + warp * 32 * G;
   float* wmax = reinterpret_cast<float*>(smem + L::WM);
 
@@ -155,10 +156,10 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   }
   __syncthreads();
 
-  // ---- token tiles of kv head g (warp-major over the cluster's warps)
+  // ---- token tiles of kv head g (warp-major over the S CTAs' warps)
   const int64_t ntile = (a.T + 31) / 32;
-  const int64_t stride = int64_t(C) * kAWarps;
-  int64_t tile = int64_t(warp) * C + rank;
+  const int64_t stride = int64_t(S) * kAWarps;
+  int64_t tile = int64_t(warp) * S + sidx;
   const float kscale = a.scale * a.pk.inv_d;
   const float vscale = a.pv.inv_sqrt_d;
   const uint32_t* ktab_l = ktab + lane;
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   }
 
   // ---- merge the warps' states: CTA maximum per head, then rescaled sums by
-  // shared-memory atomics; then the CTAs' states across the cluster
+  // shared-memory atomics
   if (lane == 0) {
 #pragma unroll
     for (int jj = 0; jj < G; ++jj) wmax[warp * G + jj] = m_run[jj];
@@ -269,129 +270,78 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
     }
     if (tid == 0) part[j] = mx;
   }
-  cluster.sync();
-  if (rank == 0) {
-    for (int idx = tid; idx < G * (kAD + 1); idx += kAThreads) {
-      const int j = idx / (kAD + 1), c = idx % (kAD + 1);
-      float mx = -INFINITY;
-      for (int r = 0; r < C; ++r) mx = fmaxf(mx, cluster.map_shared_rank(part, r)[j]);
-      float acc = 0.f;
-      for (int r = 0; r < C; ++r) {
-        const float* pr = cluster.map_shared_rank(part, r);
-        const float f = mx == -INFINITY ? 0.f : __expf(pr[j] - mx);
-        acc += f * (c < kAD ? pr[2 * G + j * kAD + c] : pr[G + j]);
-      }
-      if (c < kAD) fin[j * kAD + c] = acc;  // Σ over every token of the rotated-domain sum
-      else fin[G * kAD + j] = acc;        // the softmax denominator
+  __syncthreads();
+
+  // ---- this CTA's state to the workspace; the kv head's last CTA merges them all
+  unsigned* counter = a.counters + g;
+  float* states = a.states + int64_t(g) * S * L::PART_FLOATS;
+  for (int i = tid; i < L::PART_FLOATS; i += kAThreads) __stcg(states + sidx * L::PART_FLOATS + i, part[i]);
+  __threadfence();  // the state is visible device-wide before the count says so
+  __syncthreads();
+  if (tid == 0) *last_flag = atomicAdd(counter, 1u) == unsigned(S - 1) ? 1 : 0;
+  __syncthreads();
+  if (*last_flag == 0) return;
+  __threadfence();
+  for (int idx = tid; idx < G * (kAD + 1); idx += kAThreads) {
+    const int j = idx / (kAD + 1), c = idx % (kAD + 1);
+    float mx = -INFINITY;
+    for (int r = 0; r < S; ++r) mx = fmaxf(mx, __ldcg(states + r * L::PART_FLOATS + j));
+    float acc = 0.f;
+    for (int r = 0; r < S; ++r) {
+      const float* pr = states + r * L::PART_FLOATS;
+      const float m = __ldcg(pr + j);
+      const float f = m == -INFINITY ? 0.f : __expf(m - mx);
+      acc += f * __ldcg(c < kAD ? pr + 2 * G + j * kAD + c : pr + G + j);
+    }
+    if (c < kAD) fin[j * kAD + c] = acc;  // Σ over every token of the rotated-domain sum
+    else fin[G * kAD + j] = acc;        // the softmax denominator
+  }
+  if (tid == 0) *counter = 0u;  // every CTA of this kv head has counted: ready for the next call
+  __syncthreads();
+  for (int j = warp; j < G; j += kAWarps) {
+    const float lsum = fin[G * kAD + j];
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = fin[j * kAD + lane * 4 + k] * inv;
+    fwht128(v, lane);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = lane * 4 + k;
+      const float y = v[k] * a.pv.inv_sqrt_d;
+      a.out[int64_t(g * G + j) * kAD + i] = sign_bit(a.pv.seed, i) ? -y : y;
     }
   }
-  cluster.sync();  // the other CTAs' shared memory stays alive until rank 0 has read it
-  if (rank == 0) {
-    __syncthreads();
-    for (int j = warp; j < G; j += kAWarps) {
-      const float lsum = fin[G * kAD + j];
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      float v[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = fin[j * kAD + lane * 4 + k] * inv;
-      fwht128(v, lane);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = lane * 4 + k;
-        const float y = v[k] * a.pv.inv_sqrt_d;
-        a.out[int64_t(g * G + j) * kAD + i] = sign_bit(a.pv.seed, i) ? -y : y;
-      }
-    }
-  }
-}
-
-// Cluster sizes found for (group size, device, hkv), a fixed table (no heap
-// memory); 0 = not yet known.  When the table is full a choice is simply
-// searched again on the next call.
-struct ClusterChoice {
-  int g, dev, hkv, c;
-};
-constexpr int kClusterChoices = 64;
-std::mutex g_cluster_mu;
-ClusterChoice g_cluster_choices[kClusterChoices];
-int g_cluster_count = 0;
-
-int cached_cluster_size(int g, int dev, int hkv) {
-  std::lock_guard<std::mutex> lock(g_cluster_mu);
-  for (int i = 0; i < g_cluster_count; ++i) {
-    const ClusterChoice& c = g_cluster_choices[i];
-    if (c.g == g && c.dev == dev && c.hkv == hkv) return c.c;
-  }
-  return 0;
-}
-
-void remember_cluster_size(int g, int dev, int hkv, int c) {
-  std::lock_guard<std::mutex> lock(g_cluster_mu);
-  if (g_cluster_count < kClusterChoices) g_cluster_choices[g_cluster_count++] = {g, dev, hkv, c};
 }
 
 template <int G>
 cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   auto k = attention_decode_kernel<G>;
   constexpr int smem = ALayout<G>::TOTAL;
-  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
-                           cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return e;
-  // cluster size: the largest C ≤ 16 for which the clusters of every kv head can
-  // be resident together (one wave), found once per (device, hkv) by occupancy
-  // queries, and no larger than the cache needs
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  int cmax = cached_cluster_size(G, dev, a.hkv);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  auto configure = [&](int c) {
-    cfg.gridDim = dim3(unsigned(a.hkv * c));
-    cfg.blockDim = dim3(kAThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(c);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  };
-  if (cmax == 0) {
-    int fallback = 0;
-    for (int c = 16; c >= 1; --c) {
-      configure(c);
-      int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(k), &cfg) !=
-          cudaSuccess) {
-        (void)cudaGetLastError();
-        continue;
-      }
-      if (fallback == 0 && clusters > 0) fallback = c;  // the largest that runs at all
-      if (clusters >= a.hkv) {                            // every kv head at once
-        cmax = c;
-        break;
-      }
-    }
-    if (cmax == 0) cmax = fallback;
-    if (cmax == 0) return cudaErrorInvalidConfiguration;
-    remember_cluster_size(G, dev, a.hkv, cmax);
-  }
-  const int64_t ntile = (a.T + 31) / 32;
-  int C = cmax;
-  while (C > 1 && int64_t(C - 1) * kAWarps >= ntile) --C;  // no idle CTAs on short caches
-  configure(C);
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k, a);
+  return launch_pdl(k, a.hkv * a.splits, kAThreads, smem, stream, a);
 }
 
 }  // namespace
+
+int attention_splits(int hkv, int group, int64_t T) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int per_sm = group <= 4 ? 2 : 1;  // the CTAs an SM holds (registers)
+  int64_t s = (int64_t(per_sm) * sms + hkv - 1) / hkv;
+  const int64_t ntile = (T + 31) / 32;
+  const int64_t most = (ntile + kAWarps - 1) / kAWarps;  // every CTA gets a tile per warp
+  if (s > most) s = most;
+  return int(s < 1 ? 1 : s);
+}
+
+size_t attention_workspace_bytes(int hq, int hkv, int64_t T) {
+  const int s = attention_splits(hkv, hq / hkv, T);
+  const size_t counters = (size_t(hkv) * 4 + 255) / 256 * 256;
+  return counters + size_t(hq) * s * (kAD + 2) * 4;
+}
 
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream) {
   switch (a.group) {

@@ -17,14 +17,22 @@ struct AttnArgs {
   const uint8_t* v_codes;   // [T·hkv × 64] 4-bit V codes
   const float* v_norms;     // [T·hkv]
   float* out;               // [hq × 128]
+  unsigned* counters;       // [hkv] in the workspace, zero between calls
+  float* states;            // [hkv × splits × G·130] in the workspace
   int64_t T;
-  int hq, hkv, group;
+  int hq, hkv, group, splits;
   float scale;
   QuantParams pk, pv;       // K and V codebooks and rotation seeds
 };
 
+// Token ranges per kv head for a cache of T tokens on the current device (as
+// many CTAs as the SMs hold: two each for groups up to 4, one for 8), and the
+// workspace bytes a call needs: hkv counters (padded to 256 bytes), then
+// hq × splits × 130 floats of partial states.
+int attention_splits(int hkv, int group, int64_t T);
+size_t attention_workspace_bytes(int hq, int hkv, int64_t T);
+
 // Asynchronous on `stream`; d = 128, 4-bit K and V codes, group ∈ {1, 2, 4, 8}.
-// Launched as clusters of up to 16 CTAs per kv head.
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace rrq

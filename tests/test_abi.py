@@ -118,11 +118,14 @@ def test_other_entry_points_validate():
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 96, 0, 1, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 128, 0, 3, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot_decode(P, 4, 128, 0, 1, P, 5, None) == B.RRQ_ERR_INVALID
-    # attention: 4-bit codes and d = 128 only; T must be at least 1
-    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 128, 2, 0, None, 4, 1, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
-    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 64, 4, 0, None, 4, 1, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
-    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 0, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, None) == B.RRQ_ERR_INVALID
-    assert lib.rrq_attention_decode(P, 32, P, P, P_MIS, P, 16, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, None) == B.RRQ_ERR_INVALID
+    # attention: 4-bit codes and d = 128 only; T must be at least 1; a big enough workspace
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 128, 2, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_UNSUPPORTED
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 64, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_UNSUPPORTED
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 0, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_attention_decode(P, 32, P, P, P_MIS, P, 16, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 16, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_attention_workspace_bytes(32, 8, 128, 1 << 17) > 0
+    assert lib.rrq_attention_workspace_bytes(30, 8, 128, 16) == 0
     # unbiased scores: d other than 128 and odd group sizes are unsupported; S must be given
     assert lib.rrq_qk_scores_qjl(P, 32, P, P, P, P, P, 16, 8, 64, 2, 0, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
     assert lib.rrq_qk_scores_qjl(P, 48, P, P, P, P, P, 16, 3, 128, 2, 0, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
