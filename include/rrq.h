@@ -72,6 +72,8 @@ extern "C" {
 #define RRQ_ERR_INVALID 1     /* bad argument, detected before any launch       */
 #define RRQ_ERR_CUDA 2        /* a CUDA launch or runtime call failed           */
 #define RRQ_ERR_UNSUPPORTED 3 /* valid request this build does not implement    */
+#define RRQ_ERR_SCRATCH 4     /* request larger than the fixed scratch of
+                                 rrq_attention_decode_noalloc                   */
 
 /* element types */
 #define RRQ_F32 0
@@ -260,6 +262,31 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
                          int k_bits, uint64_t k_seed, const float* k_codebook, int v_bits,
                          uint64_t v_seed, const float* v_codebook, float scale, void* workspace,
                          size_t workspace_bytes, float* out, void* stream);
+
+/*
+ * rrq_attention_decode_noalloc — rrq_attention_decode without a workspace argument
+ * and without allocating anything.  The pages have no counterpart: this entry is
+ * for callers that cannot allocate device memory at the point of the call, such
+ * as a serving loop whose memory is reserved up front by its own allocator (a
+ * cudaMalloc there would synchronise the device and fragment the pool) or code
+ * deep in a call chain that has no workspace to pass down.
+ * Its scratch is a fixed 4 MiB array inside the library's device image, so every
+ * GPU that loads the library holds those 4 MiB until the process exits.  Requests
+ * whose workspace (rrq_attention_workspace_bytes) exceeds 4 MiB are rejected with
+ * RRQ_ERR_SCRATCH before anything is launched.
+ * The first call on a device looks up the array's address on that device (once);
+ * make that first call before any stream capture.  Each call clears the array's
+ * counters on `stream` before its kernel runs.  All calls share the one array:
+ * calls whose GPU work overlaps (other streams, other host threads) race and
+ * give wrong results; calls ordered on one stream are safe.
+ * Arguments, outputs and the other errors as rrq_attention_decode.
+ */
+int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
+                                 const float* k_norms, const uint8_t* v_codes,
+                                 const float* v_norms, int64_t T, int hkv, int d, int k_bits,
+                                 uint64_t k_seed, const float* k_codebook, int v_bits,
+                                 uint64_t v_seed, const float* v_codebook, float scale,
+                                 float* out, void* stream);
 
 /*
  * rrq_attention_workspace_bytes — the workspace rrq_attention_decode needs for

@@ -17,7 +17,7 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librrq.so")
 
-RRQ_OK, RRQ_ERR_INVALID, RRQ_ERR_CUDA, RRQ_ERR_UNSUPPORTED = 0, 1, 2, 3
+RRQ_OK, RRQ_ERR_INVALID, RRQ_ERR_CUDA, RRQ_ERR_UNSUPPORTED, RRQ_ERR_SCRATCH = 0, 1, 2, 3, 4
 RRQ_F32, RRQ_F16, RRQ_BF16 = 0, 1, 2
 DTYPE_CODE = {torch.float32: RRQ_F32, torch.float16: RRQ_F16, torch.bfloat16: RRQ_BF16}
 # GGML block types (ggml's own type numbers), as in include/rrq.h
@@ -46,6 +46,9 @@ SIGNATURES = {
                                     _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float, _vp,
                                     ctypes.c_size_t, _vp, _vp]),
     "rrq_attention_workspace_bytes": (ctypes.c_size_t, [_int, _int, _int, _c_i64]),
+    "rrq_attention_decode_noalloc": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _c_i64, _int, _int,
+                                            _int, _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float,
+                                            _vp, _vp]),
     "rrq_q4_0_rot": (_int, [_vp, _int, _c_i64, _int, _c_u64, _int, _vp, _vp]),
     "rrq_q4_0_rot_decode": (_int, [_vp, _c_i64, _int, _c_u64, _int, _vp, _int, _vp]),
     "rrq_ggml_block_bytes": (_int, [_int]),

@@ -147,6 +147,9 @@ const char* rrq_strerror(int status) {
     case RRQ_ERR_INVALID: return "invalid argument (checked before launch; nothing was run)";
     case RRQ_ERR_CUDA: return "CUDA launch or runtime error";
     case RRQ_ERR_UNSUPPORTED: return "valid request that this build does not implement";
+    case RRQ_ERR_SCRATCH:
+      return "request needs more scratch than the 4 MiB of rrq_attention_decode_noalloc "
+             "(use rrq_attention_decode with a workspace)";
   }
   return "unknown status";
 }
@@ -260,6 +263,44 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
   a.group = group;
   a.scale = scale;
   return status_of(rrq::launch_qk_scores_qjl(a, as_stream(stream)));
+}
+
+int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
+                                 const float* k_norms, const uint8_t* v_codes,
+                                 const float* v_norms, int64_t T, int hkv, int d, int k_bits,
+                                 uint64_t k_seed, const float* k_codebook, int v_bits,
+                                 uint64_t v_seed, const float* v_codebook, float scale,
+                                 float* out, void* stream) {
+  if (T < 1 || !d_ok(d) || !bits_ok(k_bits) || !bits_ok(v_bits) || hq < 1 || hkv < 1 ||
+      hq % hkv != 0 || !std::isfinite(scale))
+    return RRQ_ERR_INVALID;
+  if (q == nullptr || !aligned(q, 16) || out == nullptr || !aligned(out, 16)) return RRQ_ERR_INVALID;
+  if (!arr_ok(k_codes, T, 16) || !arr_ok(k_norms, T, 4) || !arr_ok(v_codes, T, 16) ||
+      !arr_ok(v_norms, T, 4))
+    return RRQ_ERR_INVALID;
+  const int group = hq / hkv;
+  if (d != 128 || k_bits != 4 || v_bits != 4 ||
+      (group != 1 && group != 2 && group != 4 && group != 8))
+    return RRQ_ERR_UNSUPPORTED;
+  if (rrq::attention_workspace_bytes(hq, hkv, T) > rrq::kAttentionScratchBytes)
+    return RRQ_ERR_SCRATCH;
+  rrq::AttnArgs a;
+  if (make_params(k_bits, k_codebook, k_seed, d, &a.pk) != RRQ_OK ||
+      make_params(v_bits, v_codebook, v_seed, d, &a.pv) != RRQ_OK)
+    return RRQ_ERR_INVALID;
+  a.q = static_cast<const __half*>(q);
+  a.k_codes = k_codes;
+  a.k_norms = k_norms;
+  a.v_codes = v_codes;
+  a.v_norms = v_norms;
+  a.out = out;
+  a.T = T;
+  a.hq = hq;
+  a.hkv = hkv;
+  a.group = group;
+  a.splits = rrq::attention_splits(hkv, group, T);
+  a.scale = scale;
+  return status_of(rrq::launch_attention_decode_in_scratch(a, as_stream(stream)));
 }
 
 size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int64_t T) {

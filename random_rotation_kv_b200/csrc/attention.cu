@@ -30,6 +30,7 @@
 // per head), writes the output and sets the counter back to zero.  No CTA waits
 // for another.
 #include <cmath>
+#include <mutex>
 
 #include "attention.h"
 #include "rrq_device.cuh"
@@ -341,6 +342,47 @@ size_t attention_workspace_bytes(int hq, int hkv, int64_t T) {
   const int s = attention_splits(hkv, hq / hkv, T);
   const size_t counters = (size_t(hkv) * 4 + 255) / 256 * 256;
   return counters + size_t(hq) * s * (kAD + 2) * 4;
+}
+
+// ------------------------------------------------ allocation-free variant
+// Scratch of the allocation-free entry point: a fixed array in the library's own
+// device image, present on every GPU that loads the library until the process
+// exits.  Host code reaches it only through the address cudaGetSymbolAddress
+// reports for the current device (the array's name in host code is a stand-in).
+static __device__ __align__(256) uint8_t g_attention_scratch[kAttentionScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// The array's address on the current device, looked up once per device.
+cudaError_t attention_scratch(void** addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attention_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_attention_decode_in_scratch(AttnArgs a, cudaStream_t stream) {
+  void* base = nullptr;
+  cudaError_t e = attention_scratch(&base);
+  if (e != cudaSuccess) return e;
+  const size_t counters = (size_t(a.hkv) * 4 + 255) / 256 * 256;
+  // the counters must start at zero; the previous call's partial states need not
+  e = cudaMemsetAsync(base, 0, counters, stream);
+  if (e != cudaSuccess) return e;
+  a.counters = static_cast<unsigned*>(base);
+  a.states = reinterpret_cast<float*>(static_cast<uint8_t*>(base) + counters);
+  return launch_attention_decode(a, stream);
 }
 
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream) {

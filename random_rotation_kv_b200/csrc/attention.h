@@ -35,4 +35,10 @@ size_t attention_workspace_bytes(int hq, int hkv, int64_t T);
 // Asynchronous on `stream`; d = 128, 4-bit K and V codes, group ∈ {1, 2, 4, 8}.
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);
 
+// The same with the workspace in a fixed device array of the library
+// (kAttentionScratchBytes); a.counters / a.states are set here.  The caller has
+// checked attention_workspace_bytes(...) ≤ kAttentionScratchBytes.
+constexpr size_t kAttentionScratchBytes = size_t(4) << 20;
+cudaError_t launch_attention_decode_in_scratch(AttnArgs a, cudaStream_t stream);
+
 }  // namespace rrq

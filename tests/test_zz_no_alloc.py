@@ -1,0 +1,75 @@
+"""The allocation-free attention entry point, rrq_attention_decode_noalloc (needs a B200).
+
+Some callers cannot allocate device memory where they call the library (a serving
+loop whose memory an allocator of its own reserved up front, or code with no
+workspace to hand down); this entry point runs the attention kernel with its
+scratch in a fixed 4 MiB array inside the library.  The test calls it through the
+C ABI twice in a row, on the same inputs, and compares each output with the
+workspace entry point's within the attention tolerance (2e-3 of the largest value
+reconstruction, as in test_gpu_attention.py); it also checks that a request
+larger than the array is refused before anything runs.  This file is collected
+last, so that a run stopping at its first failure has run every other test.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from random_rotation_kv_b200 import binding as B
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+D = 128
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _noalloc(q, kc, kn, vc, vn, hkv, out, scale):
+    hq = q.shape[0]
+    t_len = kn.numel() // hkv
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return B.lib().rrq_attention_decode_noalloc(
+        _ptr(q), hq, _ptr(kc), _ptr(kn), _ptr(vc), _ptr(vn), t_len, hkv, D, 4, 42, None, 4, 43,
+        None, ctypes.c_float(scale), _ptr(out), stream)
+
+
+def test_noalloc_attention_matches_the_workspace_entry_twice():
+    rg = np.random.Generator(np.random.PCG64(2024))
+    t_len, hkv, hq = 20000, 8, 32
+    rows = t_len * hkv
+    kc = torch.from_numpy(rg.integers(0, 256, size=(rows, 64), dtype=np.uint8)).to(DEV)
+    vc = torch.from_numpy(rg.integers(0, 256, size=(rows, 64), dtype=np.uint8)).to(DEV)
+    kn = torch.from_numpy((np.exp(rg.standard_normal(rows) * 0.5) * 11.0).astype(np.float32)).to(DEV)
+    vn = torch.from_numpy((np.exp(rg.standard_normal(rows) * 0.5) * 9.0).astype(np.float32)).to(DEV)
+    q = torch.from_numpy(rg.standard_normal((hq, D)).astype(np.float16)).to(DEV)
+    scale = 1.0 / math.sqrt(D)
+    ref = B.rrq_attention_decode(q, kc, kn, vc, vn, hkv, D, 42, 43, scale=scale)
+    torch.cuda.synchronize()
+    bound = 2e-3 * float(vn.max()) * 2.7326
+    for _ in range(2):
+        out = torch.full((hq, D), float("nan"), dtype=torch.float32, device=DEV)
+        assert _noalloc(q, kc, kn, vc, vn, hkv, out, scale) == B.RRQ_OK
+        torch.cuda.synchronize()
+        err = torch.linalg.norm((out - ref).double(), dim=1)
+        assert torch.all(err <= bound), float(err.max())
+
+
+def test_noalloc_attention_refuses_requests_beyond_its_scratch():
+    # 8192 query heads of one kv head need far more than 4 MiB of partial states
+    hq, hkv, t_len = 8, 1, 64
+    need = B.rrq_attention_workspace_bytes(hq * 1024, hkv * 1024, D, t_len)
+    assert need > 4 << 20
+    kc = torch.zeros(t_len * hkv * 1024, 64, dtype=torch.uint8, device=DEV)
+    kn = torch.ones(t_len * hkv * 1024, dtype=torch.float32, device=DEV)
+    q = torch.zeros(hq * 1024, D, dtype=torch.float16, device=DEV)
+    out = torch.full((hq * 1024, D), 7.0, dtype=torch.float32, device=DEV)
+    assert _noalloc(q, kc, kn, kc, kn, hkv * 1024, out, 1.0) == B.RRQ_ERR_SCRATCH
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)  # nothing ran
