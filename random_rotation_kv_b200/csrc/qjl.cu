@@ -551,7 +551,8 @@ __global__ void __launch_bounds__(kQ2Threads, 1) qjl_batch_kernel(const __grid_c
     uint32_t words[NW];
 #pragma unroll
     for (int i = 0; i < NW; ++i) words[i] = 0u;
-    float rr = 0.f;
+    float2 rr2 = make_float2(0.f, 0.f);
+    const float2 k1x2 = make_float2(k1, k1), nk2x2 = make_float2(-k2, -k2);
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {  // 8 coordinates = one 16-byte chunk per part
       uint32_t hi[4], lo[4];
@@ -567,14 +568,13 @@ __global__ void __launch_bounds__(kQ2Threads, 1) qjl_batch_kernel(const __grid_c
         const uint32_t cy = __float_as_uint(ey0.y) + (sy > ey0.x ? 1u : 0u);
         put_code<B>(words, 2 * k, cx);
         put_code<B>(words, 2 * k + 1, cy);
-        const float r0 = fmaf(w[k].x, k1, -k2 * slev[cx]);
-        const float r1 = fmaf(w[k].y, k1, -k2 * slev[cy]);
-        rr = fmaf(r0, r0, fmaf(r1, r1, rr));
-        const __half2 h = __floats2half2_rn(r0, r1);
-        const float2 hf = __half22float2(h);
-        const __half2 l = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
-        hi[j] = valid ? *reinterpret_cast<const uint32_t*>(&h) : 0u;
-        lo[j] = valid ? *reinterpret_cast<const uint32_t*>(&l) : 0u;
+        // rows past n arrive zero-filled with ν = 0, so their residual is 0
+        const float2 r = fma2(w[k], k1x2, mul2(make_float2(slev[cx], slev[cy]), nk2x2));
+        rr2 = fma2(r, r, rr2);
+        const __half2 h = __float22half2_rn(r);
+        const __half2 l = __float22half2_rn(sub2(r, __half22float2(h)));
+        hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[j] = *reinterpret_cast<const uint32_t*>(&l);
       }
       const uint32_t off = cm_offset(gt, c);
       *reinterpret_cast<uint4*>(smem + Sm::A_OFF + (g * 2 + 0) * Sm::OPER + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1) qjl_batch_kernel(const __grid_c
       store_bytes<CB>(a.codes + vec * CB, words);
       a.norms[vec] = nu;
     }
-    const float rho = sqrtf(rr) / sc;  // ‖r‖ from the scaled residual
+    const float rho = sqrtf(rr2.x + rr2.y) / sc;  // ‖r‖ from the scaled residual
 
     // ---- V = R·Sᵀ on the tensor cores (one thread of the group issues)
     fence_proxy_async_smem();  // A tiles visible to the tensor cores
@@ -622,10 +622,12 @@ __global__ void __launch_bounds__(kQ2Threads, 1) qjl_batch_kernel(const __grid_c
       uint32_t v[32];
       tmem_ld32(tmem + (uint32_t((warp & 3) * 32) << 16) + uint32_t(cc * 32), v);
       tmem_ld_wait();
-      uint32_t bsum = 0;
+      // bit j = [v_j > 0] from the sign bits (an exact +0 only arises with r = 0,
+      // handled below; elsewhere it lies far inside the sign exemption band)
+      uint32_t neg = 0;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) bsum |= (__uint_as_float(v[j]) > 0.f ? 1u : 0u) << j;
-      bits[cc] = bsum;
+      for (int j = 31; j >= 0; --j) neg = (neg << 1) | (v[j] >> 31);
+      bits[cc] = rho > 0.f ? ~neg : 0u;
     }
     if (valid) {
       reinterpret_cast<uint4*>(a.qbits + vec * (D / 8))[0] = make_uint4(bits[0], bits[1], bits[2], bits[3]);
