@@ -71,7 +71,7 @@ extern "C" {
 #define RRQ_OK 0
 #define RRQ_ERR_INVALID 1     /* bad argument, detected before any launch       */
 #define RRQ_ERR_CUDA 2        /* a CUDA launch or runtime call failed           */
-#define RRQ_ERR_UNSUPPORTED 3 /* valid request this build does not implement    */
+#define RRQ_ERR_UNSUPPORTED 3 /* valid request the library does not implement  */
 #define RRQ_ERR_SCRATCH 4     /* request larger than the fixed scratch of
                                  rrq_attention_decode_noalloc                   */
 

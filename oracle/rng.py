@@ -17,7 +17,7 @@ is:
 
 Pins: ``splitmix64`` is pinned to the published first outputs for seed 1234567
 (tests/golden/splitmix64_vectors.txt).  The sign and Gaussian constructions on
-top of it are this build's own definition ("parity unpinned" against the pages,
+top of it are this library's own definition ("parity unpinned" against the pages,
 which name no generator); the Gaussian is pinned statistically (moments).
 """
 

@@ -146,7 +146,7 @@ const char* rrq_strerror(int status) {
     case RRQ_OK: return "ok";
     case RRQ_ERR_INVALID: return "invalid argument (checked before launch; nothing was run)";
     case RRQ_ERR_CUDA: return "CUDA launch or runtime error";
-    case RRQ_ERR_UNSUPPORTED: return "valid request that this build does not implement";
+    case RRQ_ERR_UNSUPPORTED: return "valid request that the library does not implement";
     case RRQ_ERR_SCRATCH:
       return "request needs more scratch than the 4 MiB of rrq_attention_decode_noalloc "
              "(use rrq_attention_decode with a workspace)";
