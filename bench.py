@@ -337,29 +337,56 @@ def run_gpu(args):
     dec_iso = time_kernel(torch, stream, flush, lambda: dec(0, 0), 20)
     x, out, codes0, norms0 = xs[0], outs[0], codes[0], norms[0]
 
-    # end to end through the public API: pinned host -> device -> encode -> decode -> host
+    # end to end through the public API: pinned host -> device -> encode -> decode -> host,
+    # every step copying its own input in and its result out.  Steps are pipelined
+    # over three streams and two buffer sets, so that step k's device-to-host copy,
+    # step k+1's kernels and step k+2's host-to-device copy overlap (PCIe carries
+    # both directions at once).
     x_pin = torch.from_numpy(x_host).pin_memory()
-    out_pin = torch.empty(N_VEC, D, dtype=torch.float16).pin_memory()
-    x_e2e = torch.empty_like(x)
+    out_pins = [torch.empty(N_VEC, D, dtype=torch.float16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    o_dev = [out, torch.empty_like(out)]
+    c_dev = [codes0, torch.empty_like(codes0)]
+    n_dev = [norms0, torch.empty_like(norms0)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {key: [torch.cuda.Event() for _ in range(2)] for key in ("in", "run", "out")}
+    issued = {key: [False, False] for key in ("run", "out")}
 
-    def e2e_step():
-        x_e2e.copy_(x_pin, non_blocking=True)
-        B.rrq_encode(x_e2e, BITS, 42, codes=codes0, norms=norms0)
-        B.rrq_decode(codes0, norms0, D, BITS, 42, out_dtype=torch.float16, out=out)
-        out_pin.copy_(out, non_blocking=True)
+    def e2e_step(k):
+        j = k % 2
+        with torch.cuda.stream(s_in):
+            if issued["run"][j]:
+                s_in.wait_event(ev["run"][j])  # the kernels of step k-2 have read x_dev[j]
+            x_dev[j].copy_(x_pin, non_blocking=True)
+            ev["in"][j].record(s_in)
+        stream.wait_event(ev["in"][j])
+        if issued["out"][j]:
+            stream.wait_event(ev["out"][j])  # step k-2's result has left o_dev[j]
+        B.rrq_encode(x_dev[j], BITS, 42, codes=c_dev[j], norms=n_dev[j])
+        B.rrq_decode(c_dev[j], n_dev[j], D, BITS, 42, out_dtype=torch.float16, out=o_dev[j])
+        ev["run"][j].record(stream)
+        issued["run"][j] = True
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["run"][j])
+            out_pins[j].copy_(o_dev[j], non_blocking=True)
+            ev["out"][j].record(s_out)
+        issued["out"][j] = True
 
-    for _ in range(3):
-        e2e_step()
+    for k in range(3):
+        e2e_step(k)
+    torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for k in range(args.e2e_steps):
+        e2e_step(k)
+    e1.record(s_out)
+    torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = job_throughput(world, N_VEC, args.e2e_steps, e2e_ms)
-    assert torch.equal(out_pin, out.cpu())
+    last = (args.e2e_steps - 1) % 2
+    assert torch.equal(out_pins[last], o_dev[last].cpu())
 
     if rank == 0:
         peak, peak_kind = peaks()
