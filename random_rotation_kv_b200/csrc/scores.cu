@@ -404,88 +404,97 @@ cudaError_t launch_scores_dbg(const ScoreArgs& a, cudaStream_t stream) {
   return cudaErrorInvalidValue;
 }
 
-// ------------------------------------------------ one lane per key-head
-// 4-bit codes, d = 64 or 128, GQA group G ∈ {1, 2, 4, 8}.  A work unit is 32
-// consecutive tokens of one kv head g: lane t owns key-head (t0 + t, g) and
-// computes its G scores alone.  The G rotated query heads of g sit in shared
-// memory pair-major ([g][pair][head] half2), so one broadcast load serves
-// every lane; each code byte is one byte-permute table lookup (level pair);
-// G packed fp16 FMAs per pair, folded to fp32 every 16 pairs.  A unit's codes
-// (32 rows of d/2 bytes, hkv rows apart) and norms stream through a per-warp
-// cp.async ring into padded rows; the warps split the units evenly.  Scores
-// leave as 128-byte rows (32 consecutive tokens of one head).
+// ------------------------------------------------ tensor-core tiles, 4-bit codes
+// 4-bit codes, d = 64 or 128, GQA group G ∈ {1, 2, 4, 8}.  For one kv head g
+// the scores of a 32-token unit are a [32 × d]·[d × G] product of the code
+// levels and the group's rotated queries, run as mma.sync m16n8k16 tiles
+// (fp16 operands, fp32 accumulation): tokens are M (two 16-row tiles), the
+// group's query heads are N (zero columns pad G to 8), d is K.
+//  * Because the dot product sums over coordinates, any assignment of code
+//    pairs to K positions serves, as long as the query operand uses the same
+//    one.  Thread quad position c owns code bytes [c·d/8, (c+1)·d/8) of a row
+//    (one 16- or 8-byte load per row), and in k-step kk its A-fragment columns
+//    2c, 2c+1 hold code byte 2kk of that slice and columns 2c+8, 2c+9 byte
+//    2kk+1.  Each byte becomes its fp16 level pair with one byte permute and
+//    one load from a lane-replicated table, which is the A register itself.
+//  * The B fragments (query pairs in the same order) are built once per CTA in
+//    shared memory, [g][j][lane] 16-byte words, so a unit loads them with
+//    d/32 conflict-free 16-byte loads.
+//  * A unit's codes (32 rows of d/2 bytes, hkv rows apart) and norms stream
+//    through a per-warp cp.async ring of unpadded rows; each 16-byte
+//    (8-byte) fragment load of a quarter (half) warp covers 128 contiguous
+//    bytes, so it is conflict-free.  The warps split the units evenly.
+//  * Epilogue: each accumulator is scaled by ν_t·scale/d and the head's
+//    power-of-two factor and stored; for a head, eight lanes write 32
+//    consecutive bytes.
 template <int D, int W>
-struct LaneScoreSmem {
+struct MmaScoreSmem {
   static constexpr int CB = D / 2;          // code bytes per key-head
-  static constexpr int RP = CB + 16;        // padded ring row
+  static constexpr int KK = CB / 8;         // k-steps of 16 coordinates
+  static constexpr int CW = CB / 16;        // words of a thread's row slice
   static constexpr int NS = 3;              // ring stages
-  static constexpr int STAGE = 32 * RP + 32 * 4;
+  static constexpr int STAGE = 32 * CB + 32 * 4;
   static constexpr int RING = NS * STAGE;   // per warp
   __host__ __device__ static constexpr size_t table() { return 256 * 64 * 4; }  // entry e at byte e·256 + lane·4
-  __host__ __device__ static size_t q(int hq) { return size_t(hq) * D * 2; }
+  __host__ __device__ static size_t bq(int hkv) { return size_t(hkv) * 32 * CB; }  // B fragments
   __host__ __device__ static size_t inv(int hq) { return (size_t(hq) * 4 + 15) / 16 * 16; }
   __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }  // prologue only (aliases rings)
   __host__ __device__ static constexpr size_t rings() { return size_t(W) * RING; }
-  // Plain layout: [table | q'' | inv | rings (qf aliased)].
-  __host__ __device__ static size_t total(int hq) {
-    return table() + q(hq) + inv(hq) + (qf(hq) > rings() ? qf(hq) : rings());
+  __host__ __device__ static size_t head(int hq, int hkv) { return bq(hkv) + inv(hq); }
+  // Plain layout: [table | B fragments | inv | rings (qf aliased)].
+  __host__ __device__ static size_t total(int hq, int hkv) {
+    return table() + head(hq, hkv) + (qf(hq) > rings() ? qf(hq) : rings());
   }
   // Folded layout, for a dynamic base at shared address kFoldBase: the table
   // sits at shared address 0x10000 so that the byte-permuted offset
-  // 0x10000 | byte·256 | lane·4 is the load address itself.  Below it: q'',
-  // inv and the first `front` rings; above it: the other rings (qf aliased).
+  // 0x10000 | byte·256 | lane·4 is the load address itself.  Below it: the B
+  // fragments, inv and the first `front` rings; above it: the other rings
+  // (qf aliased).
   static constexpr uint32_t kFoldBase = 0x400, kFoldTable = 0x10000;
-  __host__ __device__ static size_t fold_front_rings(int hq) {
-    const size_t start = (q(hq) + inv(hq) + 15) / 16 * 16;
+  __host__ __device__ static size_t fold_front_rings(int hq, int hkv) {
+    const size_t start = head(hq, hkv);
     const size_t room = kFoldTable - kFoldBase;
     const size_t n = start < room ? (room - start) / RING : 0;
     return n < size_t(W) ? n : size_t(W);
   }
-  __host__ __device__ static size_t fold_back(int hq) { return kFoldTable - kFoldBase + table(); }
-  __host__ __device__ static size_t fold_ring(int hq, int w) {
-    const size_t nf = fold_front_rings(hq);
-    return size_t(w) < nf ? (q(hq) + inv(hq) + 15) / 16 * 16 + size_t(w) * RING
-                          : fold_back(hq) + (size_t(w) - nf) * RING;
+  __host__ __device__ static size_t fold_back() { return kFoldTable - kFoldBase + table(); }
+  __host__ __device__ static size_t fold_ring(int hq, int hkv, int w) {
+    const size_t nf = fold_front_rings(hq, hkv);
+    return size_t(w) < nf ? head(hq, hkv) + size_t(w) * RING : fold_back() + (size_t(w) - nf) * RING;
   }
-  __host__ __device__ static size_t fold_total(int hq) {
-    const size_t back = (size_t(W) - fold_front_rings(hq)) * RING;
-    return fold_back(hq) + (qf(hq) > back ? qf(hq) : back);
+  __host__ __device__ static size_t fold_total(int hq, int hkv) {
+    const size_t back = (size_t(W) - fold_front_rings(hq, hkv)) * RING;
+    return head(hq, hkv) <= kFoldTable - kFoldBase ? fold_back() + (qf(hq) > back ? qf(hq) : back)
+                                                   : ~size_t(0);
   }
 };
 
-template <int G> struct QPairs;  // the G query half2 values of one code pair
-template <> struct QPairs<1> { uint32_t v[1]; };
-template <> struct QPairs<2> { uint32_t v[2]; };
-template <> struct QPairs<4> { uint32_t v[4]; };
-template <> struct QPairs<8> { uint32_t v[8]; };
-template <int G>
-__device__ __forceinline__ QPairs<G> load_qpairs(const uint32_t* q) {
-  QPairs<G> r;
-  if constexpr (G == 1) {
-    r.v[0] = q[0];
-  } else if constexpr (G == 2) {
-    const uint2 t = *reinterpret_cast<const uint2*>(q);
-    r.v[0] = t.x; r.v[1] = t.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < G / 4; ++i) {
-      const uint4 t = reinterpret_cast<const uint4*>(q)[i];
-      r.v[4 * i] = t.x; r.v[4 * i + 1] = t.y; r.v[4 * i + 2] = t.z; r.v[4 * i + 3] = t.w;
-    }
-  }
-  return r;
+// d += A·B for one m16n8k16 tile: fp16 A (row-major) and B (column-major)
+// fragments, fp32 accumulators.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ uint32_t word_of(const uint2& v, int i) { return i == 0 ? v.x : v.y; }
+
 template <int D, int G, int W, bool FOLD>
-__global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArgs a) {
   pdl_release();
-  using Sm = LaneScoreSmem<D, W>;
-  constexpr int P = D / 2, CB = Sm::CB, RP = Sm::RP, NS = Sm::NS;
+  using Sm = MmaScoreSmem<D, W>;
+  constexpr int CB = Sm::CB, KK = Sm::KK, NS = Sm::NS;
+  using Chunk = std::conditional_t<D == 128, uint4, uint2>;  // a thread's slice of a row
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const QuantParams& p = a.p;
   uint32_t* ptab;
-  uint32_t* qp;
+  uint4* bq;
   float* inv_s;
   float* qf;
   uint8_t* ring;
@@ -497,18 +506,18 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
         a.scores[i] = __int_as_float(0x7fc00000);
       return;
     }
-    qp = reinterpret_cast<uint32_t*>(smem);
-    inv_s = reinterpret_cast<float*>(smem + Sm::q(a.hq));
+    bq = reinterpret_cast<uint4*>(smem);
+    inv_s = reinterpret_cast<float*>(smem + Sm::bq(a.hkv));
     ptab = reinterpret_cast<uint32_t*>(smem + (Sm::kFoldTable - Sm::kFoldBase));
-    qf = reinterpret_cast<float*>(smem + Sm::fold_back(a.hq));
-    ring = smem + Sm::fold_ring(a.hq, warp);
+    qf = reinterpret_cast<float*>(smem + Sm::fold_back());
+    ring = smem + Sm::fold_ring(a.hq, a.hkv, warp);
   } else {
     ptab = reinterpret_cast<uint32_t*>(smem);
-    qp = reinterpret_cast<uint32_t*>(smem + Sm::table());  // [hkv][P][G] half2
-    inv_s = reinterpret_cast<float*>(smem + Sm::table() + Sm::q(a.hq));
-    uint8_t* work = smem + Sm::table() + Sm::q(a.hq) + Sm::inv(a.hq);
+    bq = reinterpret_cast<uint4*>(smem + Sm::table());
+    inv_s = reinterpret_cast<float*>(smem + Sm::table() + Sm::bq(a.hkv));
+    uint8_t* work = smem + Sm::table() + Sm::head(a.hq, a.hkv);
     qf = reinterpret_cast<float*>(work);  // prologue only
-    ring = work + warp * NS * Sm::STAGE;
+    ring = work + warp * Sm::RING;
   }
 
   for (int i = tid; i < 256 * 64; i += W * 32) {
@@ -519,10 +528,21 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
   pdl_wait();  // from here on, global memory
   rotate_queries<D>(a, qf, inv_s, warp, lane, W);
   __syncthreads();
-  for (int i = tid; i < a.hq * P; i += W * 32) {
-    const int h = i / P, pr = i - h * P;  // head h = g·G + j
-    const __half2 v = __floats2half2_rn(qf[h * D + 2 * pr], qf[h * D + 2 * pr + 1]);
-    qp[((h / G) * P + pr) * G + (h % G)] = *reinterpret_cast<const uint32_t*>(&v);
+  // B fragment word w = 2kk + hh of lane l (quad position c, column n): the
+  // rotated pair β = c·d/8 + 2kk + hh of head g·G + n, zero for n ≥ G.
+  {
+    uint32_t* bw = reinterpret_cast<uint32_t*>(bq);
+    for (int i = tid; i < a.hkv * 32 * 2 * KK; i += W * 32) {
+      const int comp = i & 3, l = (i >> 2) & 31, j = (i >> 7) % (KK / 2), g = (i >> 7) / (KK / 2);
+      const int w = 4 * j + comp, kk = w >> 1, hh = w & 1, c = l & 3, n = l >> 2;
+      const int beta = c * (CB / 4) + 2 * kk + hh;
+      __half2 v = __floats2half2_rn(0.f, 0.f);
+      if (n < G) {
+        const float* qh = qf + (g * G + n) * D;
+        v = __floats2half2_rn(qh[2 * beta], qh[2 * beta + 1]);
+      }
+      bw[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
   }
   __syncthreads();  // qf is dead: its space becomes the rings
 
@@ -535,6 +555,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
   // FOLD: byte 2 of the permute's second operand is the table's address bit 16
   const uint32_t lane4 = uint32_t(lane) * 4u | (FOLD ? Sm::kFoldTable : 0u);
   const float post = a.scale * p.inv_d;
+  const int qc = lane & 3, qr = lane >> 2;  // quad position, row in an 8-row group
 
   // Copy k of a unit moves chunk c = lane % CPR of row t = lane / CPR + k·(32 / CPR):
   // per-lane offsets are fixed, the unit adds one base.
@@ -542,7 +563,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
   const int lt = lane / CPR, lc = lane % CPR;
   const int64_t row_bytes = int64_t(a.hkv) * CB;  // global stride between tokens
   const int64_t lane_src = lt * row_bytes + lc * 16;
-  const uint32_t lane_dst = uint32_t(lt * RP + lc * 16);
+  const uint32_t lane_dst = uint32_t(lt * CB + lc * 16);
   auto issue = [&](int stage, int64_t u) {
     if (u < u_end) {
       const int g = int(u & (a.hkv - 1));
@@ -552,16 +573,16 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
       if (t0 + 32 <= a.T) {
 #pragma unroll
         for (int k = 0; k < CPR; ++k)
-          cp_async16(dst + k * (32 / CPR) * RP, src + k * (32 / CPR) * row_bytes, 16);
-        cp_async4(dst - lane_dst + 32 * RP + lane * 4, a.norms + (t0 + lane) * a.hkv + g, 4);
+          cp_async16(dst + k * (32 / CPR) * CB, src + k * (32 / CPR) * row_bytes, 16);
+        cp_async4(dst - lane_dst + 32 * CB + lane * 4, a.norms + (t0 + lane) * a.hkv + g, 4);
       } else {
 #pragma unroll
         for (int k = 0; k < CPR; ++k) {
           const bool ok = t0 + lt + k * (32 / CPR) < a.T;
-          cp_async16(dst + k * (32 / CPR) * RP, ok ? src + k * (32 / CPR) * row_bytes : a.codes, ok ? 16 : 0);
+          cp_async16(dst + k * (32 / CPR) * CB, ok ? src + k * (32 / CPR) * row_bytes : a.codes, ok ? 16 : 0);
         }
         const bool ok = t0 + lane < a.T;
-        cp_async4(dst - lane_dst + 32 * RP + lane * 4, a.norms + (ok ? (t0 + lane) * a.hkv + g : 0), ok ? 4 : 0);
+        cp_async4(dst - lane_dst + 32 * CB + lane * 4, a.norms + (ok ? (t0 + lane) * a.hkv + g : 0), ok ? 4 : 0);
       }
     }
     cp_async_commit();
@@ -569,61 +590,66 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
 #pragma unroll
   for (int k = 0; k < NS - 1; ++k) issue(k, u_begin + k);
 
+  auto level_pair = [&](uint32_t word, int pos) -> uint32_t {
+    uint32_t cv;
+    if constexpr (FOLD) {  // address 0x10000 | byte·256 | lane·4
+      const uint32_t addr = __byte_perm(word, lane4, 0x7604u | (pos << 4));
+      asm("ld.shared.b32 %0, [%1];" : "=r"(cv) : "r"(addr));
+    } else {
+      const uint32_t off = __byte_perm(word, lane4, 0x5504u | (pos << 4));
+      cv = *reinterpret_cast<const uint32_t*>(tab_bytes + off);
+    }
+    return cv;
+  };
+
   int stage = 0;
   for (int64_t u = u_begin; u < u_end; ++u) {
     cp_async_wait<NS - 2>();
     __syncwarp();
     const uint8_t* st = ring + stage * Sm::STAGE;
-    uint32_t cw[CB / 4];
+    // rows qr + 8m, m = 0..3: tile 0 holds m = 0, 1 and tile 1 m = 2, 3
+    Chunk cw[4];
+    float nu[4];
 #pragma unroll
-    for (int i = 0; i < CB / 16; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(st + lane * RP + 16 * i);
-      cw[4 * i] = v.x; cw[4 * i + 1] = v.y; cw[4 * i + 2] = v.z; cw[4 * i + 3] = v.w;
+    for (int m = 0; m < 4; ++m) {
+      cw[m] = *reinterpret_cast<const Chunk*>(st + (qr + 8 * m) * CB + qc * (CB / 4));
+      nu[m] = reinterpret_cast<const float*>(st + 32 * CB)[qr + 8 * m];
     }
-    const float nu = reinterpret_cast<const float*>(st + 32 * RP)[lane];
     __syncwarp();  // every lane has read this stage before it is refilled
     issue(stage == 0 ? NS - 1 : stage - 1, u + NS - 1);
     stage = (stage + 1 == NS) ? 0 : stage + 1;
 
     const int g = int(u & (a.hkv - 1));
-    const int64_t t = ((u >> lg_hkv) << 5) + lane;
-    const uint32_t* qg = qp + g * P * G;
-    float dot[G];
+    const int64_t t0 = (u >> lg_hkv) << 5;
+    uint4 bv[KK / 2];
 #pragma unroll
-    for (int j = 0; j < G; ++j) dot[j] = 0.f;
+    for (int j = 0; j < KK / 2; ++j) bv[j] = bq[(g * (KK / 2) + j) * 32 + lane];
+
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int blk = 0; blk < P; blk += 16) {
-      __half2 acc[G];
+    for (int kk = 0; kk < KK; ++kk) {
+      const int wi = kk >> 1, pos = 2 * (kk & 1);
+      const uint32_t b0 = word_of(bv[kk >> 1], pos), b1 = word_of(bv[kk >> 1], pos + 1);
 #pragma unroll
-      for (int j = 0; j < G; ++j) acc[j] = __float2half2_rn(0.f);
-#pragma unroll
-      for (int pr = blk; pr < blk + 16; ++pr) {
-        uint32_t cv;
-        if constexpr (FOLD) {  // address 0x10000 | byte·256 | lane·4
-          const uint32_t addr = __byte_perm(cw[pr >> 2], lane4, 0x7604u | ((pr & 3) << 4));
-          asm("ld.shared.b32 %0, [%1];" : "=r"(cv) : "r"(addr));
-        } else {
-          const uint32_t off = __byte_perm(cw[pr >> 2], lane4, 0x5504u | ((pr & 3) << 4));
-          cv = *reinterpret_cast<const uint32_t*>(tab_bytes + off);
-        }
-        const __half2 c = *reinterpret_cast<const __half2*>(&cv);
-        const QPairs<G> qv = load_qpairs<G>(qg + pr * G);
-#pragma unroll
-        for (int j = 0; j < G; ++j)
-          acc[j] = __hfma2(*reinterpret_cast<const __half2*>(&qv.v[j]), c, acc[j]);
-      }
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float2 f = __half22float2(acc[j]);
-        dot[j] += f.x + f.y;
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t lo = word_of(cw[2 * mt], wi), hi = word_of(cw[2 * mt + 1], wi);
+        mma_16816(acc[mt], level_pair(lo, pos), level_pair(hi, pos), level_pair(lo, pos + 1),
+                  level_pair(hi, pos + 1), b0, b1);
       }
     }
-    if (t < a.T) {
-      const float sc = nu * post;
-      float* out = a.scores + int64_t(g * G) * a.T + t;
-      const float* is = inv_s + g * G;
+
+    // accumulator i of tile mt: token row qr + 8·(i >> 1) + 16·mt, head 2·qc + (i & 1)
 #pragma unroll
-      for (int j = 0; j < G; ++j) out[j * a.T] = dot[j] * sc * is[j];
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * qc + e;
+      if (h < G) {
+        const float hs = post * inv_s[g * G + h];
+        float* out = a.scores + int64_t(g * G + h) * a.T + t0 + qr;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          if (t0 + qr + 8 * m < a.T) out[8 * m] = acc[m >> 1][2 * (m & 1) + e] * (nu[m] * hs);
+        }
+      }
     }
   }
   cp_async_wait<0>();
@@ -631,13 +657,13 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_lane_kernel(const ScoreAr
 
 template <int D, int G, int W>
 cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
-  using Sm = LaneScoreSmem<D, W>;
+  using Sm = MmaScoreSmem<D, W>;
   int dev = 0, reserved = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-  const bool fold = reserved == int(Sm::kFoldBase) && Sm::fold_total(a.hq) <= 227 * 1024;
-  auto k = fold ? qk_scores_lane_kernel<D, G, W, true> : qk_scores_lane_kernel<D, G, W, false>;
-  const size_t smem = fold ? Sm::fold_total(a.hq) : Sm::total(a.hq);
+  const bool fold = reserved == int(Sm::kFoldBase) && Sm::fold_total(a.hq, a.hkv) <= 227 * 1024;
+  auto k = fold ? qk_scores_mma_kernel<D, G, W, true> : qk_scores_mma_kernel<D, G, W, false>;
+  const size_t smem = fold ? Sm::fold_total(a.hq, a.hkv) : Sm::total(a.hq, a.hkv);
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
@@ -646,14 +672,14 @@ cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
   return launch_pdl(k, grid, W * 32, smem, stream, a);
 }
 
-// The lane-per-key-head kernel applies (4-bit codes, d ≤ 128, a power-of-two
-// group ≤ 8, and its shared memory fits with 16 or 8 warps); returns its warps or 0.
+// The tensor-core kernel applies (4-bit codes, d ≤ 128, a power-of-two group
+// ≤ 8, and its shared memory fits with 16 or 8 warps); returns its warps or 0.
 template <int D>
 int lane_score_warps(int bits, int hq, int hkv) {
   const int group = hq / hkv;
   if (bits != 4 || (D != 64 && D != 128) || group > 8 || (group & (group - 1))) return 0;
-  if (LaneScoreSmem<D, 16>::total(hq) <= 227 * 1024) return 16;
-  if (LaneScoreSmem<D, 8>::total(hq) <= 227 * 1024) return 8;
+  if (MmaScoreSmem<D, 16>::total(hq, hkv) <= 227 * 1024) return 16;
+  if (MmaScoreSmem<D, 8>::total(hq, hkv) <= 227 * 1024) return 8;
   return 0;
 }
 
