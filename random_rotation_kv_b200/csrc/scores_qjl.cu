@@ -12,14 +12,15 @@
 //
 // Work split.  A CTA serves one kv head g and its GQA group of G query heads,
 // so its prologue rotates only those G queries and projects them by S (G×d²
-// multiply-adds, S read from L2).  Both are kept as fp16 pairs, pair-major, each
-// head scaled by a power of two to |·| ≤ 1 (undone in fp32).  Warps then take
-// tiles of 32 consecutive tokens of that kv head, one token per lane: the lane
-// loads its code row, sign row, norm and residual norm (16-byte loads, the next
-// tile's while it works on this one), looks up each pair of codes in a
-// lane-replicated table of fp16 level pairs and each pair of sign bits in a
-// lane-replicated table of (±1, ±1), and accumulates both dot products for the
-// G heads with packed fp16 FMAs, folded into fp32 every 16 pairs.
+// multiply-adds, S read from L2).  Both are kept as fp16 pairs, each head
+// scaled by a power of two to |·| ≤ 1 (undone in fp32).  Warps then take
+// units of 32 consecutive tokens of that kv head, and each unit's two dot
+// products are mma.sync m16n8k16 tiles (fp16 operands, fp32 accumulation):
+// tokens are M, the group's heads N (zero columns pad G to 8), coordinates K.
+// Thread quad position c owns coordinate pairs [16c, 16c + 16) of its rows, so
+// it loads B code words and one sign word per row (the next unit's while it
+// works on this one); table lookups turn them into the A fragments: fp16
+// level pairs for the codes, (±1, ±1) pairs for a nibble of sign bits.
 #include <cmath>
 
 #include "rrq_device.cuh"
@@ -29,92 +30,179 @@ namespace rrq {
 namespace {
 
 constexpr int kSD = 128;              // head dimension served
-constexpr int kSP = kSD / 2;          // coordinate pairs
-constexpr int kSWarps = 8;
+constexpr int kSWarps = 16;
 constexpr int kSThreads = kSWarps * 32;
 
-template <int B, int G> struct QSLayout {
-  static constexpr int E = 1 << (2 * B);        // pair-table entries (two codes)
-  static constexpr int TAB = 0;                 // [E][32] half2 level pairs
-  static constexpr int SGN = TAB + E * 32 * 4;  // [4][32] half2 (±1, ±1)
-  static constexpr int QH = SGN + 4 * 32 * 4;   // [kSP][G] half2 q'' pairs
-  static constexpr int VH = QH + kSP * G * 4;   // [kSP][G] half2 v'' pairs
-  static constexpr int QF = VH + kSP * G * 4;   // [G][kSD] fp32 q' (prologue)
-  static constexpr int VF = QF + G * kSD * 4;   // [G][kSD] fp32 v (prologue)
-  static constexpr int SC = VF + G * kSD * 4;   // [G] 1/s_q, [G] 1/s_v, [G] max|v| bits
-  static constexpr int TOTAL = SC + 3 * G * 4;
+// Level table of the b-bit codes, lane-replicated, at a shared address aligned
+// to its size so that entry | lane column | base is one OR:
+//   b = 1: a code nibble (two coordinate pairs) → two half2, 16 entries × 256 B;
+//   b = 2: a code byte (two pairs) → two half2, 256 entries × 256 B;
+//   b = 3: six bits (one pair) → one half2, 64 entries × 128 B;
+//   b = 4: a code byte (one pair) → one half2, 256 entries × 256 B
+//     (the upper half of each entry is unused: the byte permute places the
+//     byte at bits 8..15).
+template <int B> struct LevelTable {
+  static constexpr uint32_t kEntries = B == 1 ? 16 : B == 3 ? 64 : 256;
+  static constexpr uint32_t kStride = B == 3 ? 128 : 256;
+  static constexpr uint32_t kBytes = kEntries * kStride;
+  static constexpr bool kTwoPairs = B <= 2;  // an entry holds pairs 2kk and 2kk+1
 };
 
-// Bits [o, o + n) of a little-endian word array (o, n compile-time after unrolling).
-template <int NW>
-__device__ __forceinline__ uint32_t bit_field(const uint32_t (&w)[NW], int o, int n) {
-  const int wi = o >> 5, sh = o & 31;
-  const uint32_t lo = w[wi];
-  const uint32_t hi = (wi + 1 < NW) ? w[wi + 1] : 0u;
-  const uint32_t v = sh + n <= 32 ? (lo >> sh) : __funnelshift_r(lo, hi, sh);
-  return v & ((1u << n) - 1u);
+// Shared memory, as offsets from the dynamic base at shared address `base`
+// (the host computes it for the device's reserved shared memory; the kernel
+// checks it):
+//   sgn  sign-nibble table, 16 entries × 256 B, 4 KB-aligned;
+//   bf   B fragments of q'' and v'', [2][4][32] × 16 B;
+//   qf   q' and v in fp32 (prologue), [2][G][128];
+//   sc   1/s_q, 1/s_v and max|v| bits per head;
+//   tab  the level table, aligned to its size.
+struct QjlLayout {
+  uint32_t sgn, bf, qf, sc, tab, total;
+};
+template <int B, int G>
+__host__ __device__ constexpr QjlLayout qjl_layout(uint32_t base) {
+  const uint32_t tb = LevelTable<B>::kBytes;
+  const uint32_t sgn = (base + 4095u) / 4096u * 4096u;
+  const uint32_t bf = sgn + 4096u;
+  const uint32_t qf = bf + 2u * 4u * 32u * 16u;
+  const uint32_t sc = qf + 2u * G * kSD * 4u;
+  const uint32_t end = (sc + 3u * G * 4u + 15u) / 16u * 16u;
+  const uint32_t tab = (end + tb - 1u) / tb * tb;
+  return QjlLayout{sgn - base, bf - base, qf - base, sc - base, tab - base, tab + tb - base};
 }
 
-template <int B>
-struct KeyRow {
-  static constexpr int NW = 4 * B;  // code words (16·B bytes)
-  uint32_t c[NW];
-  uint32_t s[4];  // sign bits
+// The slice of one key row that quad position c owns: coordinate pairs
+// [16c, 16c + 16), i.e. code words [B·c, B·c + B) and sign word c.
+template <int B> struct RowSlice {
+  uint32_t c[B];
+  uint32_t s;
   float nu, rho;
 };
 
 template <int B>
-__device__ __forceinline__ void load_row(KeyRow<B>& r, const QjlScoreArgs& a, int64_t t, int g) {
+__device__ __forceinline__ void load_slice(RowSlice<B>& r, const QjlScoreArgs& a, int64_t t, int g,
+                                           int qc) {
   if (t < a.T) {
     const int64_t n = t * a.hkv + g;
-    const uint4* cp = reinterpret_cast<const uint4*>(a.codes + n * (16 * B));
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(a.codes + n * (16 * B)) + B * qc;
+    if constexpr (B == 4) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(cw));
+      r.c[0] = v.x; r.c[1] = v.y; r.c[2] = v.z; r.c[3] = v.w;
+    } else if constexpr (B == 2) {
+      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(cw));
+      r.c[0] = v.x; r.c[1] = v.y;
+    } else {
 #pragma unroll
-    for (int k = 0; k < B; ++k) {
-      const uint4 v = __ldcs(cp + k);
-      r.c[4 * k] = v.x; r.c[4 * k + 1] = v.y; r.c[4 * k + 2] = v.z; r.c[4 * k + 3] = v.w;
+      for (int k = 0; k < B; ++k) r.c[k] = __ldcs(cw + k);
     }
-    const uint4 sv = __ldcs(reinterpret_cast<const uint4*>(a.bits + n * 16));
-    r.s[0] = sv.x; r.s[1] = sv.y; r.s[2] = sv.z; r.s[3] = sv.w;
+    r.s = __ldcs(reinterpret_cast<const uint32_t*>(a.bits + n * 16) + qc);
     r.nu = __ldcs(a.norms + n);
     r.rho = __ldcs(a.rnorm + n);
   } else {
 #pragma unroll
-    for (int k = 0; k < KeyRow<B>::NW; ++k) r.c[k] = 0u;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) r.s[k] = 0u;
+    for (int k = 0; k < B; ++k) r.c[k] = 0u;
+    r.s = 0u;
     r.nu = 0.f;
     r.rho = 0.f;
   }
 }
 
+// Table address of nibble kk of w: (nibble << 8) | col (kk compile-time after unrolling).
+__device__ __forceinline__ uint32_t nibble_addr(uint32_t w, int kk, uint32_t col) {
+  const uint32_t t = kk <= 2 ? (w << (8 - 4 * kk)) : (w >> (4 * kk - 8));
+  return (t & 0xF00u) | col;
+}
+
+__device__ __forceinline__ uint2 lds2(uint32_t addr) {
+  uint2 v;
+  asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds1(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// d += A·B for one m16n8k16 tile: fp16 A (row-major) and B (column-major)
+// fragments, fp32 accumulators.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Level pairs of coordinate pairs 2kk (x) and 2kk + 1 (y) of a row slice.
+template <int B>
+__device__ __forceinline__ uint2 level_pairs(const uint32_t (&c)[B], int kk, uint32_t col) {
+  if constexpr (B == 1) {
+    return lds2(nibble_addr(c[0], kk, col));
+  } else if constexpr (B == 2) {
+    return lds2(__byte_perm(c[kk >> 2], col, 0x7604u | ((kk & 3) << 4)));
+  } else if constexpr (B == 4) {
+    const uint32_t w = c[kk >> 1], pos = 2 * (kk & 1);
+    return make_uint2(lds1(__byte_perm(w, col, 0x7604u | (pos << 4))),
+                      lds1(__byte_perm(w, col, 0x7604u | ((pos + 1) << 4))));
+  } else {  // B == 3: six bits per pair, possibly across a word boundary
+    uint32_t e[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int o = 6 * (2 * kk + hh), wi = o >> 5, sh = o & 31;
+      const uint32_t v = sh + 6 <= 32 ? (c[wi] >> sh) : __funnelshift_r(c[wi], c[wi + 1], sh);
+      e[hh] = lds1(((v & 63u) << 7) | col);
+    }
+    return make_uint2(e[0], e[1]);
+  }
+}
+
 template <int B, int G>
-__global__ void __launch_bounds__(kSThreads) qk_scores_qjl_kernel(const QjlScoreArgs a) {
+__global__ void __launch_bounds__(kSThreads, 1) qk_scores_qjl_kernel(const QjlScoreArgs a, uint32_t base) {
   pdl_release();
-  using L = QSLayout<B, G>;
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::TAB);
-  uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + L::SGN);
-  __half2* qh = reinterpret_cast<__half2*>(smem + L::QH);
-  __half2* vh = reinterpret_cast<__half2*>(smem + L::VH);
-  float* qf = reinterpret_cast<float*>(smem + L::QF);
-  float* vf = reinterpret_cast<float*>(smem + L::VF);
-  float* inv_sq = reinterpret_cast<float*>(smem + L::SC);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = blockIdx.x % a.hkv;
+  const QjlLayout lay = qjl_layout<B, G>(base);
+  if (smem_addr(smem) != base) {
+    // not the layout the launch assumed: mark this CTA's scores as invalid
+    pdl_wait();
+    const int cpg = gridDim.x / a.hkv;
+    for (int64_t t = int64_t(blockIdx.x / a.hkv) * kSThreads + tid; t < a.T; t += int64_t(cpg) * kSThreads)
+      for (int j = 0; j < G; ++j) a.scores[int64_t(g * G + j) * a.T + t] = __int_as_float(0x7fc00000);
+    return;
+  }
+  uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + lay.sgn);
+  uint32_t* bf = reinterpret_cast<uint32_t*>(smem + lay.bf);
+  float* qf = reinterpret_cast<float*>(smem + lay.qf);
+  float* vf = qf + G * kSD;
+  float* inv_sq = reinterpret_cast<float*>(smem + lay.sc);
   float* inv_sv = inv_sq + G;
   unsigned* vmax = reinterpret_cast<unsigned*>(inv_sv + G);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem + lay.tab);
   const QuantParams& p = a.p;
-  const int g = blockIdx.x % a.hkv;
 
   // ---- tables from the parameters alone
-  for (int i = tid; i < L::E * 32; i += kSThreads) {
-    const int e = i >> 5;
-    const __half2 v = __floats2half2_rn(p.levels[e & ((1 << B) - 1)], p.levels[e >> B]);
+  using LT = LevelTable<B>;
+  constexpr uint32_t M = (1u << B) - 1u;
+  for (uint32_t i = tid; i < LT::kBytes / 4; i += kSThreads) {
+    const uint32_t e = i / (LT::kStride / 4), wv = i % (LT::kStride / 4);
+    float lo, hi;
+    if constexpr (LT::kTwoPairs) {  // word wv = 2·lane + hh: pair hh of the entry
+      const uint32_t pr = (e >> (4 * B / 2 * (wv & 1))) & ((1u << (2 * B)) - 1u);
+      lo = p.levels[pr & M];
+      hi = p.levels[pr >> B];
+    } else {
+      lo = p.levels[e & M];
+      hi = p.levels[e >> B];
+    }
+    const __half2 v = __floats2half2_rn(lo, hi);
     tab[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
-  if (tid < 128) {
-    const int e = tid >> 5;
-    const __half2 v = __floats2half2_rn((e & 1) ? 1.f : -1.f, (e & 2) ? 1.f : -1.f);
-    sgn[tid] = *reinterpret_cast<const uint32_t*>(&v);
+  for (uint32_t i = tid; i < 1024; i += kSThreads) {  // sign nibble → (±1, ±1), (±1, ±1)
+    const uint32_t e = i >> 6, pr = (e >> (2 * (i & 1))) & 3u;
+    const __half2 v = __floats2half2_rn((pr & 1u) ? 1.f : -1.f, (pr & 2u) ? 1.f : -1.f);
+    sgn[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
   if (tid < G) vmax[tid] = 0u;
   pdl_wait();  // from here on, global memory
@@ -144,19 +232,8 @@ __global__ void __launch_bounds__(kSThreads) qk_scores_qjl_kernel(const QjlScore
 #pragma unroll
       for (int k = 0; k < 4; ++k) v[k] = fmaf(v[k], sg, __shfl_xor_sync(kFull, v[k], m));
     }
-    float mx = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) mx = fmaxf(mx, fabsf(v[k]));
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-    int ex = 0;
-    frexpf(mx, &ex);
-    const float s = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
 #pragma unroll
     for (int k = 0; k < 4; ++k) qf[j * kSD + lane * 4 + k] = v[k];
-    qh[(2 * lane) * G + j] = __floats2half2_rn(v[0] * s, v[1] * s);
-    qh[(2 * lane + 1) * G + j] = __floats2half2_rn(v[2] * s, v[3] * s);
-    if (lane == 0) inv_sq[j] = 1.f / s;
   }
   __syncthreads();
 
@@ -180,81 +257,120 @@ __global__ void __launch_bounds__(kSThreads) qk_scores_qjl_kernel(const QjlScore
     vf[o] = acc;
     atomicMax(&vmax[j], __float_as_uint(fabsf(acc)));
   }
+  if (warp < G) {  // max|q'| of head `warp`
+    float mx = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx = fmaxf(mx, fabsf(qf[warp * kSD + lane * 4 + k]));
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+    if (lane == 0) {
+      int ex = 0;
+      frexpf(mx, &ex);  // mx = f·2^ex, 0.5 ≤ f < 1
+      inv_sq[warp] = mx > 0.f ? ldexpf(1.f, ex) : 1.f;
+    }
+  }
   __syncthreads();
-  for (int o = tid; o < G * kSP; o += kSThreads) {
-    const int j = o / kSP, pr = o % kSP;
-    const float mx = __uint_as_float(vmax[j]);
+  if (tid < G) {
+    const float mx = __uint_as_float(vmax[tid]);
     int ex = 0;
     frexpf(mx, &ex);
-    const float s = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
-    vh[pr * G + j] = __floats2half2_rn(vf[j * kSD + 2 * pr] * s, vf[j * kSD + 2 * pr + 1] * s);
-    if (pr == 0) inv_sv[j] = 1.f / s;
+    inv_sv[tid] = mx > 0.f ? ldexpf(1.f, ex) : 1.f;
+  }
+  __syncthreads();
+  // B fragment word w = 2kk + hh of lane l (quad position c, column n): the
+  // pair β = 16c + 2kk + hh of head n's q'' (part 0) or v'' (part 1), zero for n ≥ G.
+  for (int i = tid; i < 2 * 4 * 32 * 4; i += kSThreads) {
+    const int comp = i & 3, l = (i >> 2) & 31, j = (i >> 7) & 3, part = i >> 9;
+    const int w = 4 * j + comp, kk = w >> 1, hh = w & 1, c = l & 3, n = l >> 2;
+    const int beta = 16 * c + 2 * kk + hh;
+    __half2 v = __floats2half2_rn(0.f, 0.f);
+    if (n < G) {
+      const float* src = (part ? vf : qf) + n * kSD;
+      const float s = 1.f / (part ? inv_sv[n] : inv_sq[n]);  // a power of two
+      v = __floats2half2_rn(src[2 * beta] * s, src[2 * beta + 1] * s);
+    }
+    bf[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
   __syncthreads();
 
-  // ---- tiles of 32 tokens of kv head g, one token per lane
+  const int qc = lane & 3, qr = lane >> 2;  // quad position, row in an 8-row group
+  uint32_t bq[16], bv[16];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 x = reinterpret_cast<const uint4*>(bf)[j * 32 + lane];
+    const uint4 y = reinterpret_cast<const uint4*>(bf)[(4 + j) * 32 + lane];
+    bq[4 * j] = x.x; bq[4 * j + 1] = x.y; bq[4 * j + 2] = x.z; bq[4 * j + 3] = x.w;
+    bv[4 * j] = y.x; bv[4 * j + 1] = y.y; bv[4 * j + 2] = y.z; bv[4 * j + 3] = y.w;
+  }
+  // per accumulator column e (head 2·qc + e): scale·inv_d/s_q and scale·cq/s_v
+  const float cq = sqrtf(0.5f * float(M_PI)) / (float(kSD) * sqrtf(float(kSD)));
+  float km[2], ks[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * qc + e;
+    km[e] = h < G ? a.scale * p.inv_d * inv_sq[h] : 0.f;
+    ks[e] = h < G ? a.scale * cq * inv_sv[h] : 0.f;
+  }
+  const uint32_t col_t = (base + lay.tab) | uint32_t(lane) * (LT::kTwoPairs ? 8u : 4u);
+  const uint32_t col_s = (base + lay.sgn) | uint32_t(lane) * 8u;
+
+  // ---- units of 32 tokens of kv head g; rows qr + 8m (m = 0..3) per thread
   const int cpg = gridDim.x / a.hkv;
   const int64_t ntile = (a.T + 31) / 32;
   const int64_t stride = int64_t(cpg) * kSWarps;
   int64_t tile = int64_t(warp) * cpg + blockIdx.x / a.hkv;  // warp-major: equal tiles per CTA
-  const float cq = sqrtf(0.5f * float(M_PI)) / (float(kSD) * sqrtf(float(kSD)));
-  const uint32_t* tab_l = tab + lane;
-  const uint32_t* sgn_l = sgn + lane;
-  KeyRow<B> cur, nxt;
-  load_row<B>(cur, a, tile * 32 + lane, g);
+  RowSlice<B> cur[4], nxt[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) load_slice<B>(cur[m], a, tile * 32 + qr + 8 * m, g, qc);
   for (; tile < ntile; tile += stride) {
-    const int64_t t = tile * 32 + lane;
-    load_row<B>(nxt, a, t + stride * 32, g);
-    float accm[G], accq[G];
+    const int64_t t0 = tile * 32;
 #pragma unroll
-    for (int j = 0; j < G; ++j) accm[j] = accq[j] = 0.f;
+    for (int m = 0; m < 4; ++m) load_slice<B>(nxt[m], a, t0 + stride * 32 + qr + 8 * m, g, qc);
+    float am[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float as[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int f = 0; f < kSP / 16; ++f) {
-      __half2 hm[G], hs[G];
+    for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-      for (int j = 0; j < G; ++j) hm[j] = hs[j] = __float2half2_rn(0.f);
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint2 lo = level_pairs<B>(cur[2 * mt].c, kk, col_t);
+        const uint2 hi = level_pairs<B>(cur[2 * mt + 1].c, kk, col_t);
+        mma16816(am[mt], lo.x, hi.x, lo.y, hi.y, bq[2 * kk], bq[2 * kk + 1]);
+        const uint2 slo = lds2(nibble_addr(cur[2 * mt].s, kk, col_s));
+        const uint2 shi = lds2(nibble_addr(cur[2 * mt + 1].s, kk, col_s));
+        mma16816(as[mt], slo.x, shi.x, slo.y, shi.y, bv[2 * kk], bv[2 * kk + 1]);
+      }
+    }
+    // accumulator i of tile mt: row qr + 8·(i >> 1) + 16·mt, head 2·qc + (i & 1)
 #pragma unroll
-      for (int pp = 0; pp < 16; ++pp) {
-        const int pr = f * 16 + pp;
-        const uint32_t e = bit_field(cur.c, 2 * B * pr, 2 * B);
-        const uint32_t sb = (cur.s[pr >> 4] >> ((2 * pr) & 31)) & 3u;
-        const uint32_t cw = tab_l[e << 5], sw = sgn_l[sb << 5];
-        const __half2 c2 = *reinterpret_cast<const __half2*>(&cw);
-        const __half2 s2 = *reinterpret_cast<const __half2*>(&sw);
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * qc + e;
+      if (h < G) {
+        float* out = a.scores + int64_t(g * G + h) * a.T + t0 + qr;
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          hm[j] = __hfma2(qh[pr * G + j], c2, hm[j]);
-          hs[j] = __hfma2(vh[pr * G + j], s2, hs[j]);
+        for (int m = 0; m < 4; ++m) {
+          const float v = fmaf(cur[m].nu * km[e], am[m >> 1][2 * (m & 1) + e],
+                               cur[m].rho * ks[e] * as[m >> 1][2 * (m & 1) + e]);
+          if (t0 + qr + 8 * m < a.T) out[8 * m] = v;
         }
       }
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float2 m2 = __half22float2(hm[j]), s2 = __half22float2(hs[j]);
-        accm[j] += m2.x + m2.y;
-        accq[j] += s2.x + s2.y;
-      }
     }
-    if (t < a.T) {
-      const float mse = cur.nu * p.inv_d, res = cur.rho * cq;
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float sc = a.scale * (mse * inv_sq[j] * accm[j] + res * inv_sv[j] * accq[j]);
-        a.scores[int64_t(g * G + j) * a.T + t] = sc;
-      }
-    }
-    cur = nxt;
+    for (int m = 0; m < 4; ++m) cur[m] = nxt[m];
   }
 }
 
 template <int B, int G>
 cudaError_t launch_bg(const QjlScoreArgs& a, cudaStream_t stream) {
   auto k = qk_scores_qjl_kernel<B, G>;
-  constexpr int smem = QSLayout<B, G>::TOTAL;
-  if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-  }
+  int dev = 0, reserved = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  const uint32_t base = uint32_t(reserved);
+  const QjlLayout lay = qjl_layout<B, G>(base);
+  const int smem = int(lay.total);
+  const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
   const int64_t ntile = (a.T + 31) / 32;
   const int resident = grid_for(reinterpret_cast<const void*>(k), kSThreads, smem, int64_t(1) << 40);
   int64_t cpg = resident / a.hkv;
@@ -262,7 +378,7 @@ cudaError_t launch_bg(const QjlScoreArgs& a, cudaStream_t stream) {
   if (cpg > need) cpg = need;
   if (cpg < 1) cpg = 1;
   const int grid = int(cpg * a.hkv);
-  return launch_pdl(k, grid, kSThreads, smem, stream, a);
+  return launch_pdl(k, grid, kSThreads, size_t(smem), stream, a, base);
 }
 
 template <int B>
