@@ -39,45 +39,54 @@ namespace rrq {
 namespace {
 
 constexpr int kAD = 128;
-constexpr int kAP = kAD / 2;
-constexpr int kAWarps = 8;
+constexpr int kAWarps = 16;
 constexpr int kAThreads = kAWarps * 32;
+constexpr int kWRow = 40;  // fp16 weights per head row of a warp's transpose buffer (padded)
 
+// Shared memory, as offsets from the dynamic base at shared address kBase (the
+// launch checks the device's reserved shared memory; the kernel checks the
+// address).  The two level tables sit at 64 KB-aligned addresses so that a byte
+// permute of a code byte and the lane column (byte·256 | lane·4 | table) is the
+// load address itself.
 template <int G> struct ALayout {
-  static constexpr int KTAB = 0;                               // [256][32] half2 (K level pairs)
-  static constexpr int VTAB = KTAB + 256 * 32 * 4;             // [256][16] float2 (V level pairs)
-  static constexpr int QH = VTAB + 256 * 16 * 8;               // [kAP][G] half2 q''
-  static constexpr int INV = QH + kAP * G * 4;                 // [G] 1/s
-  static constexpr int WBUF = (INV + G * 4 + 15) / 16 * 16;    // per warp: weights [32][G]
-  static constexpr int WM = WBUF + kAWarps * 32 * G * 4;       // [kAWarps][G] warp maxima
-  static constexpr int PART_FLOATS = 2 * G + G * kAD;         // [G] m, [G] l, [G][kAD] o
-  static constexpr int PART = WM + kAWarps * G * 4;            // the CTA's partial state
-  static constexpr int FLAG = PART + PART_FLOATS * 4;          // "this CTA merges its kv head"
-  static constexpr int TOTAL = FLAG + 16;
-  static constexpr int FIN = KTAB;  // the last CTA's merged sums reuse the level tables
-  static_assert(G * (kAD + 1) * 4 <= VTAB, "merged sums fit over the K table");
-  static_assert(TOTAL <= 110 * 1024, "two CTAs per SM");
+  static constexpr uint32_t kBase = 0x400;
+  static constexpr uint32_t KTAB = 0x10000 - kBase;              // [256][64] half2, K level pairs
+  static constexpr uint32_t VTAB = 0x20000 - kBase;              // [256][64] half2, V level pairs
+  static constexpr uint32_t BF = 0;                              // [4][32] uint4 B fragments of q''
+  static constexpr uint32_t QF = BF + 4 * 32 * 16;               // [G][kAD] fp32 q' (prologue)
+  static constexpr uint32_t INV = QF + G * kAD * 4;              // [G] 1/s
+  static constexpr uint32_t WBUF = (INV + G * 4 + 15) / 16 * 16; // per warp: [8][kWRow] fp16 weights
+  static constexpr uint32_t WM = WBUF + kAWarps * 8 * kWRow * 2; // [kAWarps][G] warp maxima
+  static constexpr int PART_FLOATS = 2 * G + G * kAD;           // [G] m, [G] l, [G][kAD] o
+  static constexpr uint32_t PART = WM + kAWarps * G * 4;         // the CTA's partial state
+  static constexpr uint32_t FLAG = PART + PART_FLOATS * 4;       // "this CTA merges its kv head"
+  static constexpr uint32_t FIN = (FLAG + 16 + 15) / 16 * 16;    // the merging CTA's sums [G][kAD + 1]
+  static constexpr uint32_t END = FIN + G * (kAD + 1) * 4;
+  static constexpr uint32_t TOTAL = VTAB + 256 * 256;
+  static_assert(END <= KTAB, "the small buffers fit below the K table");
+  static_assert(TOTAL <= 227 * 1024, "shared memory");
 };
 
-struct KRow {
-  uint4 k[4];
-  float kn, vn;
-};
-
-__device__ __forceinline__ void load_krow(KRow& r, const AttnArgs& a, int64_t t, int g) {
-  if (t < a.T) {
-    const int64_t n = t * a.hkv + g;
-    const uint4* kp = reinterpret_cast<const uint4*>(a.k_codes + n * 64);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) r.k[i] = __ldcs(kp + i);
-    r.kn = __ldcs(a.k_norms + n);
-    r.vn = __ldcs(a.v_norms + n);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) r.k[i] = make_uint4(0u, 0u, 0u, 0u);
-    r.kn = r.vn = 0.f;
-  }
+// d += A·B for one m16n8k16 tile: fp16 A (row-major) and B (column-major)
+// fragments, fp32 accumulators.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+
+// Level pair of code byte `pos` of w: one load at byte·256 | col.
+__device__ __forceinline__ uint32_t pair_at(uint32_t w, int pos, uint32_t col) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(__byte_perm(w, col, 0x7604u | (pos << 4))));
+  return v;
+}
+__device__ __forceinline__ uint32_t word4(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ uint32_t word2(const uint2& v, int i) { return i == 0 ? v.x : v.y; }
 
 // 128-point unnormalised Walsh–Hadamard transform of v (4 values per lane, lane-major).
 __device__ __forceinline__ void fwht128(float (&v)[4], int lane) {
@@ -98,37 +107,56 @@ __device__ __forceinline__ void fwht128(float (&v)[4], int lane) {
   }
 }
 
-// Two CTAs per SM (≤ 128 registers) where the group's accumulators allow it.
-template <int G> constexpr int attention_min_blocks() { return G <= 4 ? 2 : 1; }
-
+// Per 32-token tile of kv head g, in each warp (qr = lane / 4, qc = lane % 4):
+//  A. scores S[32 tokens × 8] = levels(K codes)·q'' as in the score kernel:
+//     rows qr + 8m (m = 0..3) are the thread's tokens, its code slice is bytes
+//     [16qc, 16qc + 16), columns 2qc, 2qc + 1 its heads.
+//  B. the online softmax per head on those fragments (max and sum over the
+//     tile by shuffles across the 8 lanes of equal qc); the weights
+//     w = p·ν^V/√d go to the warp's transpose buffer as fp16 [head][token].
+//  C. O^T[128 × 8] += levels(V codes)^T·W^T: coordinates are M, heads N,
+//     tokens K.  Row qr of m-tile mt is coordinate 2(8qr + mt) and row qr + 8
+//     coordinate 2(8qr + mt) + 1, so both come from V byte 8qr + mt; for the
+//     token pair of a fragment column the two bytes' level pairs are looked up
+//     and regrouped per coordinate with two byte permutes.  The output
+//     columns are the same heads 2qc, 2qc + 1 as the score columns, so the
+//     softmax rescaling touches only the thread's own accumulators.
 template <int G>
-__global__ void __launch_bounds__(kAThreads, attention_min_blocks<G>()) attention_decode_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const AttnArgs a) {
   pdl_release();
   using L = ALayout<G>;
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* ktab = reinterpret_cast<uint32_t*>(smem + L::KTAB);
-  float2* vtab = reinterpret_cast<float2*>(smem + L::VTAB);
-  __half2* qh = reinterpret_cast<__half2*>(smem + L::QH);
-  float* inv_s = reinterpret_cast<float*>(smem + L::INV);
-  float* part = reinterpret_cast<float*>(smem + L::PART);
-  float* fin = reinterpret_cast<float*>(smem + L::FIN);
-  int* last_flag = reinterpret_cast<int*>(smem + L::FLAG);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.splits;
   const int g = blockIdx.x / S, sidx = blockIdx.x % S;
-  float* wbuf = reinterpret_cast<float*>(smem + L::WBUF) + warp * 32 * G;
-  float* wmax = reinterpret_cast<float*>(smem + L::WM);
-
-  // ---- level tables from the parameters alone
-  for (int i = tid; i < 256 * 32; i += kAThreads) {
-    const int e = i >> 5;
-    const __half2 kv = __floats2half2_rn(a.pk.levels[e & 15], a.pk.levels[e >> 4]);
-    ktab[i] = *reinterpret_cast<const uint32_t*>(&kv);
+  if (smem_addr(smem) != L::kBase) {
+    // not the layout the launch assumed: this CTA's kv head gets NaN outputs
+    pdl_wait();
+    if (sidx == 0)
+      for (int i = tid; i < G * kAD; i += kAThreads) a.out[int64_t(g * G) * kAD + i] = __int_as_float(0x7fc00000);
+    return;
   }
-  // 16 copies suffice for the fp32 pairs: a 64-bit shared load serves each half-warp
-  // in its own pass, so lanes l and l + 16 never meet in one
-  for (int i = tid; i < 256 * 16; i += kAThreads)
-    vtab[i] = make_float2(a.pv.levels[(i >> 4) & 15], a.pv.levels[i >> 8]);
+  uint32_t* ktab = reinterpret_cast<uint32_t*>(smem + L::KTAB);
+  uint32_t* vtab = reinterpret_cast<uint32_t*>(smem + L::VTAB);
+  uint32_t* bf = reinterpret_cast<uint32_t*>(smem + L::BF);
+  float* qf = reinterpret_cast<float*>(smem + L::QF);
+  float* inv_s = reinterpret_cast<float*>(smem + L::INV);
+  __half* wbuf = reinterpret_cast<__half*>(smem + L::WBUF) + warp * 8 * kWRow;
+  float* wmax = reinterpret_cast<float*>(smem + L::WM);
+  float* part = reinterpret_cast<float*>(smem + L::PART);
+  int* last_flag = reinterpret_cast<int*>(smem + L::FLAG);
+  float* fin = reinterpret_cast<float*>(smem + L::FIN);
+
+  // ---- level tables from the parameters alone: entry e at e·256 + lane·4
+  for (int i = tid; i < 256 * 64; i += kAThreads) {
+    const int e = i >> 6;
+    const __half2 kv = __floats2half2_rn(a.pk.levels[e & 15], a.pk.levels[e >> 4]);
+    const __half2 vv = __floats2half2_rn(a.pv.levels[e & 15], a.pv.levels[e >> 4]);
+    ktab[i] = *reinterpret_cast<const uint32_t*>(&kv);
+    vtab[i] = *reinterpret_cast<const uint32_t*>(&vv);
+  }
+  // weight rows of the padding heads (G..7) stay zero
+  for (int i = lane; i < 8 * kWRow; i += 32) wbuf[i] = __float2half_rn(0.f);
   for (int i = tid; i < L::PART_FLOATS; i += kAThreads) part[i] = 0.f;
   pdl_wait();  // from here on, global memory
 
@@ -151,125 +179,160 @@ __global__ void __launch_bounds__(kAThreads, attention_min_blocks<G>()) attentio
     int ex = 0;
     frexpf(mx, &ex);
     const float s = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
-    qh[(2 * lane) * G + j] = __floats2half2_rn(v[0] * s, v[1] * s);
-    qh[(2 * lane + 1) * G + j] = __floats2half2_rn(v[2] * s, v[3] * s);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qf[j * kAD + lane * 4 + k] = v[k] * s;
     if (lane == 0) inv_s[j] = 1.f / s;
   }
   __syncthreads();
+  // B fragment word w = 2kk + hh of lane l (quad position c, column n): the
+  // pair β = 16c + 2kk + hh of head n's q'', zero for n ≥ G.
+  for (int i = tid; i < 4 * 32 * 4; i += kAThreads) {
+    const int comp = i & 3, l = (i >> 2) & 31, j = i >> 7;
+    const int w = 4 * j + comp, kk = w >> 1, hh = w & 1, c = l & 3, n = l >> 2;
+    const int beta = 16 * c + 2 * kk + hh;
+    __half2 v = __floats2half2_rn(0.f, 0.f);
+    if (n < G) v = __floats2half2_rn(qf[n * kAD + 2 * beta], qf[n * kAD + 2 * beta + 1]);
+    bf[i] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  __syncthreads();
+
+  const int qc = lane & 3, qr = lane >> 2;
+  // this lane's B fragment words, read per k-step (registers are the scarce resource)
+  const uint2* bq = reinterpret_cast<const uint2*>(bf) + lane * 2;
+  const float vscale = a.pv.inv_sqrt_d;
+  float kse[2];  // scale·inv_d/s of heads 2qc + e
+#pragma unroll
+  for (int e = 0; e < 2; ++e) kse[e] = 2 * qc + e < G ? a.scale * a.pk.inv_d * inv_s[2 * qc + e] : 0.f;
+  const uint32_t kcol = 0x10000u | uint32_t(lane) * 4u;
+  const uint32_t vcol = 0x20000u | uint32_t(lane) * 4u;
 
   // ---- token tiles of kv head g (warp-major over the S CTAs' warps)
   const int64_t ntile = (a.T + 31) / 32;
   const int64_t stride = int64_t(S) * kAWarps;
-  int64_t tile = int64_t(warp) * S + sidx;
-  const float kscale = a.scale * a.pk.inv_d;
-  const float vscale = a.pv.inv_sqrt_d;
-  const uint32_t* ktab_l = ktab + lane;
-  const float2* vtab_l = vtab + (lane & 15);
-  float m_run[G], l_run[G];
-  float2 o[G][2];  // coordinates 4·lane .. 4·lane+3 of each head's rotated-domain sum
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  float o[8][4];
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    m_run[j] = -INFINITY;
-    l_run[j] = 0.f;
-    o[j][0] = o[j][1] = make_float2(0.f, 0.f);
-  }
-  for (; tile < ntile; tile += stride) {
-    const int64_t t = tile * 32 + lane;
-    KRow cur;
-    load_krow(cur, a, t, g);
-    // the tile's V code bytes for this lane's four coordinates, all in flight now
-    uint32_t vb[32];
+  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  for (int64_t tile = int64_t(warp) * S + sidx; tile < ntile; tile += stride) {
+    const int64_t t0 = tile * 32;
+    // K slices of tokens qr + 8m, V bytes [8qr, 8qr + 8) of tokens 2qc + {0, 1, 8, 9} + 16ks
+    uint4 kc[4];
+    uint2 vc[2][4];
+    float kn[4], vn[4];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int64_t tu = tile * 32 + u;
-      vb[u] = tu < a.T ? uint32_t(__ldcs(reinterpret_cast<const uint16_t*>(
-                             a.v_codes + (tu * a.hkv + g) * 64) + lane))
-                       : 0u;
+    for (int m = 0; m < 4; ++m) {
+      const int64_t t = t0 + qr + 8 * m;
+      const bool ok = t < a.T;
+      const int64_t n = ok ? t * a.hkv + g : 0;
+      kc[m] = ok ? __ldcs(reinterpret_cast<const uint4*>(a.k_codes + n * 64) + qc) : make_uint4(0u, 0u, 0u, 0u);
+      kn[m] = ok ? __ldcs(a.k_norms + n) : 0.f;
+      vn[m] = ok ? __ldcs(a.v_norms + n) : 0.f;
     }
-    // A. scores of this lane's token
-    const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur.k);
-    float sc[G];
 #pragma unroll
-    for (int j = 0; j < G; ++j) sc[j] = 0.f;
+    for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
-    for (int f = 0; f < kAP / 16; ++f) {
-      __half2 hs[G];
-#pragma unroll
-      for (int j = 0; j < G; ++j) hs[j] = __float2half2_rn(0.f);
-#pragma unroll
-      for (int pp = 0; pp < 16; ++pp) {
-        const int pr = f * 16 + pp;
-        const uint32_t byte = (kw[pr >> 2] >> (8 * (pr & 3))) & 255u;
-        const uint32_t cw = ktab_l[byte << 5];
-        const __half2 c2 = *reinterpret_cast<const __half2*>(&cw);
-#pragma unroll
-        for (int j = 0; j < G; ++j) hs[j] = __hfma2(qh[pr * G + j], c2, hs[j]);
+      for (int j = 0; j < 4; ++j) {
+        const int64_t t = t0 + 16 * ks + 2 * qc + (j & 1) + 8 * (j >> 1);
+        const bool ok = t < a.T;
+        vc[ks][j] = ok ? __ldcs(reinterpret_cast<const uint2*>(a.v_codes + (t * a.hkv + g) * 64) + qr)
+                       : make_uint2(0u, 0u);
       }
+
+    // A. scores
+    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float2 s2 = __half22float2(hs[j]);
-        sc[j] += s2.x + s2.y;
+    for (int kk = 0; kk < 8; ++kk) {
+      const int wi = kk >> 1, pos = 2 * (kk & 1);
+      const uint2 b = bq[(kk >> 1) * 64 + (kk & 1)];  // words 2kk, 2kk + 1 of the lane's fragment
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t lo = word4(kc[2 * mt], wi), hi = word4(kc[2 * mt + 1], wi);
+        mma16816(sacc[mt], pair_at(lo, pos, kcol), pair_at(hi, pos, kcol), pair_at(lo, pos + 1, kcol),
+                 pair_at(hi, pos + 1, kcol), b.x, b.y);
       }
     }
-    const bool valid = t < a.T;
-    float alpha[G];
+
+    // B. online softmax per head; weights to the transpose buffer
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-      const float s = valid ? kscale * cur.kn * inv_s[j] * sc[j] : -INFINITY;
-      float mt = s;
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * qc + e;
+      float s[4];
+      float mt = -INFINITY;
 #pragma unroll
-      for (int m = 16; m > 0; m >>= 1) mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, m));
-      const float mn = fmaxf(m_run[j], mt);  // finite: the tile holds a valid token
-      alpha[j] = __expf(m_run[j] - mn);
-      const float pj = valid ? __expf(s - mn) : 0.f;
-      float ps = pj;
+      for (int m = 0; m < 4; ++m) {
+        const bool ok = t0 + qr + 8 * m < a.T;
+        s[m] = ok ? kse[e] * kn[m] * sacc[m >> 1][2 * (m & 1) + e] : -INFINITY;
+        mt = fmaxf(mt, s[m]);
+      }
 #pragma unroll
-      for (int m = 16; m > 0; m >>= 1) ps += __shfl_xor_sync(kFull, ps, m);
-      l_run[j] = l_run[j] * alpha[j] + ps;
-      m_run[j] = mn;
-      wbuf[lane * G + j] = pj * cur.vn * vscale;
-    }
+      for (int sh = 4; sh < 32; sh <<= 1) mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, sh));
+      const float mn = fmaxf(m_run[e], mt);  // finite: the tile holds a valid token
+      const float alpha = __expf(m_run[e] - mn);
+      float ps = 0.f;
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-      o[j][0] = make_float2(o[j][0].x * alpha[j], o[j][0].y * alpha[j]);
-      o[j][1] = make_float2(o[j][1].x * alpha[j], o[j][1].y * alpha[j]);
-    }
-    __syncwarp();
-    // B. weighted sum of the tile's V rows, four coordinates per lane
+      for (int m = 0; m < 4; ++m) {
+        const float p = __expf(s[m] - mn);  // 0 for a token past T
+        ps += p;
+        if (h < G) wbuf[h * kWRow + qr + 8 * m] = __float2half_rn(p * vn[m] * vscale);
+      }
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const float2 c0 = vtab_l[(vb[u] & 255u) << 4], c1 = vtab_l[(vb[u] >> 8) << 4];
+      for (int sh = 4; sh < 32; sh <<= 1) ps += __shfl_xor_sync(kFull, ps, sh);
+      l_run[e] = l_run[e] * alpha + ps;
+      m_run[e] = mn;
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float w = wbuf[u * G + j];
-        o[j][0] = __ffma2_rn(c0, make_float2(w, w), o[j][0]);
-        o[j][1] = __ffma2_rn(c1, make_float2(w, w), o[j][1]);
+      for (int mt2 = 0; mt2 < 8; ++mt2) {
+        o[mt2][e] *= alpha;
+        o[mt2][2 + e] *= alpha;
       }
     }
     __syncwarp();
+
+    // C. O^T += levels(V)^T · W^T
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      const uint32_t* wr = reinterpret_cast<const uint32_t*>(wbuf + qr * kWRow + 16 * ks + 2 * qc);
+      const uint32_t b0 = wr[0], b1 = wr[4];  // tokens 16ks + 2qc, +1 and +8, +9 of head qr
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int wi = mt >> 2, pos = mt & 3;
+        const uint32_t p0 = pair_at(word2(vc[ks][0], wi), pos, vcol);  // token 2qc
+        const uint32_t p1 = pair_at(word2(vc[ks][1], wi), pos, vcol);  // token 2qc + 1
+        const uint32_t p8 = pair_at(word2(vc[ks][2], wi), pos, vcol);  // token 2qc + 8
+        const uint32_t p9 = pair_at(word2(vc[ks][3], wi), pos, vcol);  // token 2qc + 9
+        mma16816(o[mt], __byte_perm(p0, p1, 0x5410u), __byte_perm(p0, p1, 0x7632u),
+                 __byte_perm(p8, p9, 0x5410u), __byte_perm(p8, p9, 0x7632u), b0, b1);
+      }
+    }
+    __syncwarp();  // the buffer is read before the next tile writes it
   }
 
   // ---- merge the warps' states: CTA maximum per head, then rescaled sums by
-  // shared-memory atomics
-  if (lane == 0) {
+  // shared-memory atomics.  Accumulator o[mt][i]: coordinate 16qr + 2mt + (i >> 1),
+  // head 2qc + (i & 1).
+  if (qr == 0) {
 #pragma unroll
-    for (int jj = 0; jj < G; ++jj) wmax[warp * G + jj] = m_run[jj];
+    for (int e = 0; e < 2; ++e)
+      if (2 * qc + e < G) wmax[warp * G + 2 * qc + e] = m_run[e];
   }
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    float mx = -INFINITY;
-    for (int w = 0; w < kAWarps; ++w) mx = fmaxf(mx, wmax[w * G + j]);
-    const float f = m_run[j] == -INFINITY ? 0.f : __expf(m_run[j] - mx);
-    float* oj = part + 2 * G + j * kAD + 4 * lane;
-    if (f > 0.f) {
-      atomicAdd(oj, f * o[j][0].x);
-      atomicAdd(oj + 1, f * o[j][0].y);
-      atomicAdd(oj + 2, f * o[j][1].x);
-      atomicAdd(oj + 3, f * o[j][1].y);
-      if (lane == 0) atomicAdd(part + G + j, f * l_run[j]);
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * qc + e;
+    if (h < G) {
+      float mx = -INFINITY;
+      for (int w = 0; w < kAWarps; ++w) mx = fmaxf(mx, wmax[w * G + h]);
+      const float f = m_run[e] == -INFINITY ? 0.f : __expf(m_run[e] - mx);
+      float* oh = part + 2 * G + h * kAD + 16 * qr;
+      if (f > 0.f) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          atomicAdd(oh + 2 * mt, f * o[mt][e]);
+          atomicAdd(oh + 2 * mt + 1, f * o[mt][2 + e]);
+        }
+        if (qr == 0) atomicAdd(part + G + h, f * l_run[e]);
+      }
+      if (warp == 0 && qr == 0) part[h] = mx;
     }
-    if (tid == 0) part[j] = mx;
   }
   __syncthreads();
 
@@ -318,9 +381,14 @@ __global__ void __launch_bounds__(kAThreads, attention_min_blocks<G>()) attentio
 template <int G>
 cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
   auto k = attention_decode_kernel<G>;
+  int dev = 0, reserved = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
+  if (uint32_t(reserved) != ALayout<G>::kBase) return cudaErrorNotSupported;
   constexpr int smem = ALayout<G>::TOTAL;
-  const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, a.hkv * a.splits, kAThreads, smem, stream, a);
 }
@@ -330,8 +398,8 @@ cudaError_t launch_g(const AttnArgs& a, cudaStream_t stream) {
 int attention_splits(int hkv, int group, int64_t T) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int per_sm = group <= 4 ? 2 : 1;  // the CTAs an SM holds (registers)
-  int64_t s = (int64_t(per_sm) * sms + hkv - 1) / hkv;
+  (void)group;  // one CTA per SM for every group
+  int64_t s = (int64_t(sms) + hkv - 1) / hkv;
   const int64_t ntile = (T + 31) / 32;
   const int64_t most = (ntile + kAWarps - 1) / kAWarps;  // every CTA gets a tile per warp
   if (s > most) s = most;

@@ -63,19 +63,22 @@ def test_attention_parity_on_oracle_encoded_cache(hq, hkv, t_len):
 
 def test_attention_special_cases():
     """One token returns its value; a zero query averages the values; a large scale
-    picks the top-scoring token's value."""
+    picks the top-scoring token's value.  The weighted sum runs on fp16 levels and
+    weights (fp32 accumulation), so the value checks use the reconstruction
+    tolerance, 2e-3 of the largest |v̂|."""
     rg = np.random.Generator(np.random.PCG64(5))
     hq, hkv = 4, 2
     kp, kn, vp, vn = _cache(rg, 1, hkv, 7, 8)
     q = rg.standard_normal((hq, D)).astype(np.float16)
     got, _ = _check(q, kp, kn, vp, vn, 1, hkv, 7, 8, 1.0, "one token")
     v_hat = orc.decode_exact(vp, vn, 4, D, 8)
-    assert np.allclose(got, v_hat[np.arange(hq) // 2], atol=1e-4 * np.abs(v_hat).max())
+    # fp16 level and weight operands: within the reconstruction tolerance (2e-3 relative)
+    assert np.allclose(got, v_hat[np.arange(hq) // 2], atol=2e-3 * np.abs(v_hat).max())
     t_len = 300
     kp, kn, vp, vn = _cache(rg, t_len, hkv, 7, 8)
     got, _ = _check(np.zeros((hq, D), np.float16), kp, kn, vp, vn, t_len, hkv, 7, 8, 1.0, "zero query")
     v_hat = orc.decode_exact(vp, vn, 4, D, 8).reshape(t_len, hkv, D)
-    assert np.allclose(got[0], v_hat[:, 0].mean(axis=0), atol=1e-4)
+    assert np.allclose(got[0], v_hat[:, 0].mean(axis=0), atol=2e-3 * np.abs(v_hat[:, 0]).max())
     q = rg.standard_normal((hq, D)).astype(np.float16)
     _check(q, kp, kn, vp, vn, t_len, hkv, 7, 8, 50.0, "large scale")
 
