@@ -348,9 +348,13 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   __threadfence();
   for (int idx = tid; idx < G * (kAD + 1); idx += kAThreads) {
     const int j = idx / (kAD + 1), c = idx % (kAD + 1);
+    // unrolled so that each batch of loads is in flight at once (the order of
+    // the additions is unchanged)
     float mx = -INFINITY;
+#pragma unroll 8
     for (int r = 0; r < S; ++r) mx = fmaxf(mx, __ldcg(states + r * L::PART_FLOATS + j));
     float acc = 0.f;
+#pragma unroll 8
     for (int r = 0; r < S; ++r) {
       const float* pr = states + r * L::PART_FLOATS;
       const float m = __ldcg(pr + j);
