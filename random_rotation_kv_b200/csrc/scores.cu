@@ -656,7 +656,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
 }
 
 template <int D, int G, int W>
-cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
+cudaError_t launch_scores_mma_w(const ScoreArgs& a, cudaStream_t stream) {
   using Sm = MmaScoreSmem<D, W>;
   int dev = 0, reserved = 0;
   cudaGetDevice(&dev);
@@ -675,7 +675,7 @@ cudaError_t launch_scores_lane_w(const ScoreArgs& a, cudaStream_t stream) {
 // The tensor-core kernel applies (4-bit codes, d ≤ 128, a power-of-two group
 // ≤ 8, and its shared memory fits with 16 or 8 warps); returns its warps or 0.
 template <int D>
-int lane_score_warps(int bits, int hq, int hkv) {
+int mma_score_warps(int bits, int hq, int hkv) {
   const int group = hq / hkv;
   if (bits != 4 || (D != 64 && D != 128) || group > 8 || (group & (group - 1))) return 0;
   if (MmaScoreSmem<D, 16>::total(hq, hkv) <= 227 * 1024) return 16;
@@ -684,18 +684,18 @@ int lane_score_warps(int bits, int hq, int hkv) {
 }
 
 template <int D, int G>
-cudaError_t launch_scores_lane_g(const ScoreArgs& a, cudaStream_t stream) {
-  if (lane_score_warps<D>(4, a.hq, a.hkv) == 16) return launch_scores_lane_w<D, G, 16>(a, stream);
-  return launch_scores_lane_w<D, G, 8>(a, stream);
+cudaError_t launch_scores_mma_g(const ScoreArgs& a, cudaStream_t stream) {
+  if (mma_score_warps<D>(4, a.hq, a.hkv) == 16) return launch_scores_mma_w<D, G, 16>(a, stream);
+  return launch_scores_mma_w<D, G, 8>(a, stream);
 }
 
 template <int D>
-cudaError_t launch_scores_lane(const ScoreArgs& a, cudaStream_t stream) {
+cudaError_t launch_scores_mma(const ScoreArgs& a, cudaStream_t stream) {
   switch (a.group) {
-    case 1: return launch_scores_lane_g<D, 1>(a, stream);
-    case 2: return launch_scores_lane_g<D, 2>(a, stream);
-    case 4: return launch_scores_lane_g<D, 4>(a, stream);
-    case 8: return launch_scores_lane_g<D, 8>(a, stream);
+    case 1: return launch_scores_mma_g<D, 1>(a, stream);
+    case 2: return launch_scores_mma_g<D, 2>(a, stream);
+    case 4: return launch_scores_mma_g<D, 4>(a, stream);
+    case 8: return launch_scores_mma_g<D, 8>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -703,7 +703,7 @@ cudaError_t launch_scores_lane(const ScoreArgs& a, cudaStream_t stream) {
 template <int D, int B>
 cudaError_t launch_scores_db(const ScoreArgs& a, cudaStream_t stream) {
   if constexpr (B == 4 && D <= 128) {
-    if (lane_score_warps<D>(B, a.hq, a.hkv) > 0) return launch_scores_lane<D>(a, stream);
+    if (mma_score_warps<D>(B, a.hq, a.hkv) > 0) return launch_scores_mma<D>(a, stream);
   }
   switch (a.group) {
     case 1: return launch_scores_dbg<D, B, 1>(a, stream);
@@ -741,8 +741,8 @@ bool qk_scores_supported(int d, int bits, int hq, int hkv) {
   }
   (void)hb;
   if (w > 0) return true;  // a warp's head block is fixed: head blocks divide the warps
-  if (d == 64) return lane_score_warps<64>(bits, hq, hkv) > 0;
-  if (d == 128) return lane_score_warps<128>(bits, hq, hkv) > 0;
+  if (d == 64) return mma_score_warps<64>(bits, hq, hkv) > 0;
+  if (d == 128) return mma_score_warps<128>(bits, hq, hkv) > 0;
   return false;
 }
 
