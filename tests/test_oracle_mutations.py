@@ -239,3 +239,49 @@ def test_mutation_attention_softmax_over_heads(monkeypatch):
 
     monkeypatch.setattr(oatt, "decode_attention", bad)
     assert _fails(pins.test_attention_zero_query_is_the_mean_value_and_order_free)
+
+
+def _unbiased_with(residual_query, group_of):
+    """scores_unbiased with the residual term's query and kv group replaced."""
+
+    def bad(q, packed, norms, qjl_bits, rnorm, t_len, hkv, d, bits, seed, s_matrix, levels=None,
+            scale=1.0):
+        q = np.asarray(q, np.float64)
+        hq = q.shape[0]
+        out = orrq.scores(q, packed, norms, t_len, hkv, d, bits, seed, levels, scale)
+        qr = residual_query(q, seed)
+        qb = np.asarray(qjl_bits, dtype=np.uint8).reshape(t_len, hkv, d // 8)
+        rn = np.asarray(rnorm, np.float64).reshape(t_len, hkv)
+        for h in range(hq):
+            g = group_of(h, hq, hkv)
+            out[h] += scale * oqjl.estimate_residual_dot(qr[h], s_matrix, qb[:, g, :], rn[:, g])
+        return out
+
+    return bad
+
+
+def test_mutation_unbiased_residual_with_the_unrotated_query(monkeypatch):
+    """The QJL term dotted with S·q instead of S·Πq (the sketch lives in the rotated domain)."""
+    monkeypatch.setattr(oqjl, "scores_unbiased", _unbiased_with(lambda q, seed: q, orrq.kv_group))
+    assert _fails(pins.test_qjl_unbiased_scores_average_to_the_true_inner_product)
+
+
+def test_mutation_unbiased_residual_with_the_wrong_kv_group(monkeypatch):
+    """The QJL term of head h taken from kv head h mod Hkv instead of ⌊h·Hkv/Hq⌋."""
+    monkeypatch.setattr(oqjl, "scores_unbiased",
+                        _unbiased_with(orrq.rotate, lambda h, hq, hkv: h % hkv))
+    assert _fails(pins.test_qjl_unbiased_scores_average_to_the_true_inner_product)
+
+
+def test_mutation_unbiased_residual_subtracted(monkeypatch):
+    """The residual estimate subtracted instead of added."""
+    monkeypatch.setattr(oqjl, "scores_unbiased",
+                        _unbiased_with(lambda q, seed: -orrq.rotate(q, seed), orrq.kv_group))
+    assert _fails(pins.test_qjl_unbiased_scores_average_to_the_true_inner_product)
+
+
+def test_unbiased_harness_unmutated_passes(monkeypatch):
+    """Control: the harness above with the right query and group passes the pin, so the
+    three failures come from the planted slips alone."""
+    monkeypatch.setattr(oqjl, "scores_unbiased", _unbiased_with(orrq.rotate, orrq.kv_group))
+    assert not _fails(pins.test_qjl_unbiased_scores_average_to_the_true_inner_product)
