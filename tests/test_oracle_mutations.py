@@ -285,3 +285,46 @@ def test_unbiased_harness_unmutated_passes(monkeypatch):
     three failures come from the planted slips alone."""
     monkeypatch.setattr(oqjl, "scores_unbiased", _unbiased_with(orrq.rotate, orrq.kv_group))
     assert not _fails(pins.test_qjl_unbiased_scores_average_to_the_true_inner_product)
+
+
+def _attention_with(group_of, use_scale, key_seed_of):
+    """decode_attention with the kv group map, the score scale or the key rotation seed replaced."""
+
+    def bad(q, kp, kn, vp, vn, t_len, hkv, d, kb, vb, ks, vs, kl=None, vl=None, scale=1.0):
+        q = np.asarray(q, np.float64)
+        hq = q.shape[0]
+        s = orrq.scores(q, kp, kn, t_len, hkv, d, kb, key_seed_of(ks, vs), kl, scale if use_scale else 1.0)
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        p = w / w.sum(axis=1, keepdims=True)
+        v_hat = orrq.decode_exact(vp, vn, vb, d, vs, vl).reshape(t_len, hkv, d)
+        return np.stack([p[h] @ v_hat[:, group_of(h, hq, hkv), :] for h in range(hq)])
+
+    return bad
+
+
+_ATT_PINS = (lambda: pins.test_attention_single_token_returns_its_value(),
+             lambda: pins.test_attention_zero_query_is_the_mean_value_and_order_free(),
+             lambda: pins.test_attention_large_scale_picks_the_top_scoring_token())
+
+
+def _any_pin_fails():
+    return any(_fails(p) for p in _ATT_PINS)
+
+
+@pytest.mark.parametrize("slip", ["group", "scale", "key_seed"])
+def test_mutation_attention_slips(monkeypatch, slip):
+    """Head h reading kv head h mod Hkv; the score scale dropped; the scores taken
+    under the value rotation instead of the key rotation."""
+    import oracle.attention as oatt
+    group_of = (lambda h, hq, hkv: h % hkv) if slip == "group" else orrq.kv_group
+    key_seed_of = (lambda ks, vs: vs) if slip == "key_seed" else (lambda ks, vs: ks)
+    monkeypatch.setattr(oatt, "decode_attention", _attention_with(group_of, slip != "scale", key_seed_of))
+    assert _any_pin_fails()
+
+
+def test_attention_harness_unmutated_passes(monkeypatch):
+    """Control: the harness with the right map, scale and seed passes every attention pin."""
+    import oracle.attention as oatt
+    monkeypatch.setattr(oatt, "decode_attention",
+                        _attention_with(orrq.kv_group, True, lambda ks, vs: ks))
+    assert not _any_pin_fails()
