@@ -328,3 +328,65 @@ def test_attention_harness_unmutated_passes(monkeypatch):
     monkeypatch.setattr(oatt, "decode_attention",
                         _attention_with(orrq.kv_group, True, lambda ks, vs: ks))
     assert not _any_pin_fails()
+
+
+# ---------------------------------------------------------------- DRIVE
+def _drive_encode_with(sign_rule, stored_factor):
+    """drive_encode with the sign rule or the stored scale factor replaced."""
+    import oracle.sphere as osp
+
+    def bad(x, seed, unbiased):
+        x = np.asarray(x, np.float64)
+        d = x.shape[-1]
+        rx = orrq.rotate(x, seed)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            s = osp.drive_scale_unbiased(x, rx) if unbiased else osp.drive_scale_biased(rx)
+        s = np.where(np.sum(np.abs(rx), axis=-1) > 0, s, 0.0)
+        signs = sign_rule(rx).astype(np.int64)
+        stored = (s * stored_factor(d)).astype(np.float32)
+        return osp.DriveEncoded(signs, orrq.pack_codes(signs, 1), s, stored, rx)
+
+    return bad
+
+
+def test_mutation_drive_biased_scale_with_the_two_norm(monkeypatch):
+    """S = ‖R(x)‖₂/d instead of ‖R(x)‖₁/d."""
+    import oracle.sphere as osp
+    monkeypatch.setattr(osp, "drive_scale_biased",
+                        lambda rx: np.linalg.norm(np.asarray(rx, np.float64), axis=-1) / np.shape(rx)[-1])
+    assert _fails(pins.test_drive_biased_scale_is_mse_optimal, 16)
+
+
+def test_mutation_drive_unbiased_scale_with_the_two_norm(monkeypatch):
+    """S = ‖x‖₂²/‖R(x)‖₂ instead of ‖x‖₂²/‖R(x)‖₁."""
+    import oracle.sphere as osp
+
+    def bad(x, rx):
+        x, rx = np.asarray(x, np.float64), np.asarray(rx, np.float64)
+        return np.sum(x * x, axis=-1) / np.linalg.norm(rx, axis=-1)
+
+    monkeypatch.setattr(osp, "drive_scale_unbiased", bad)
+    assert _fails(pins.test_drive_unbiased_scale, 8)
+
+
+def test_mutation_drive_zero_takes_plus_one(monkeypatch):
+    """sign(0) = +1 in the encoder (the decoder and the b-bit rule keep −1)."""
+    import oracle.sphere as osp
+    monkeypatch.setattr(osp, "drive_encode", _drive_encode_with(lambda rx: rx >= 0, math.sqrt))
+    assert _fails(pins.test_drive_zero_coordinates_take_the_minus_one_sign)
+
+
+def test_mutation_drive_stored_without_sqrt_d(monkeypatch):
+    """The stored per-vector value S instead of S·√d."""
+    import oracle.sphere as osp
+    monkeypatch.setattr(osp, "drive_encode", _drive_encode_with(lambda rx: rx > 0, lambda d: 1.0))
+    assert _fails(pins.test_drive_encode_through_the_one_bit_decoder, False)
+
+
+def test_drive_harness_unmutated_passes(monkeypatch):
+    """Control: the encoder harness with the right sign rule and factor passes both pins."""
+    import oracle.sphere as osp
+    monkeypatch.setattr(osp, "drive_encode", _drive_encode_with(lambda rx: rx > 0, math.sqrt))
+    assert not _fails(pins.test_drive_zero_coordinates_take_the_minus_one_sign)
+    assert not _fails(pins.test_drive_encode_through_the_one_bit_decoder, False)
+    assert not _fails(pins.test_drive_encode_through_the_one_bit_decoder, True)
