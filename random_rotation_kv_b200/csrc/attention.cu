@@ -11,18 +11,14 @@
 //     out[h] = Σ_t p[h,t]·v̂_{t,g} = Πᵀ_V ( Σ_t p[h,t]·(ν^V_{t,g}/√d)·c_V[code^V_{t,g}] ),
 // so the values are summed in their rotated domain and rotated back once per head.
 //
-// Work split.  The cache of kv head g is cut into S token ranges, one CTA each
-// (grid hkv × S, about two CTAs per SM); a CTA serves the GQA group of G query
-// heads of its kv head, and its warps take tiles of 32 consecutive tokens:
-//  A. one token per lane: the lane loads its K row (64 B), scores the G heads
-//     with packed fp16 FMAs on a lane-replicated table of level pairs (as the
-//     score kernel), and the warp updates its running softmax state (max, sum)
-//     per head; the lane writes its weights w_h = p_h·ν^V/√d to the warp buffer.
-//  B. four coordinates per lane: the warp reads the tile's V rows (two bytes
-//     per lane per token, 64 contiguous bytes per token, all 32 loads in flight
-//     at once), looks each byte up in a table of fp32 level pairs (16 copies,
-//     one per lane of a half-warp) and accumulates w_h times them into fp32
-//     partial sums (packed FMAs).
+// Work split.  The cache of kv head g is cut into S token ranges, one 16-warp
+// CTA each (grid hkv × S, one CTA per SM); a CTA serves the GQA group of G query
+// heads of its kv head, and its warps take tiles of 32 consecutive tokens.  Both
+// contractions of a tile run as mma.sync m16n8k16 tiles (fp16 operands, fp32
+// accumulation; the group padded to 8 columns), their A fragments looked up from
+// lane-replicated tables of level pairs; the online softmax runs on the score
+// fragments, and the weights w = p·ν^V/√d reach the value product through a
+// per-warp transpose buffer (attention_decode_kernel says how).
 // The warps' states merge within the CTA (shared-memory atomics after a common
 // rescaling); each CTA writes its state (max, sum, G×128 partial sums) to the
 // caller's workspace and counts itself in its kv head's counter there.  The

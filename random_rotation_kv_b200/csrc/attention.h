@@ -26,7 +26,7 @@ struct AttnArgs {
 };
 
 // Token ranges per kv head for a cache of T tokens on the current device (as
-// many CTAs as the SMs hold: two each for groups up to 4, one for 8), and the
+// many CTAs as the device has SMs, one each), and the
 // workspace bytes a call needs: hkv counters (padded to 256 bytes), then
 // hq × splits × 130 floats of partial states.
 int attention_splits(int hkv, int group, int64_t T);

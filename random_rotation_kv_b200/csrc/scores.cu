@@ -6,6 +6,10 @@
 //     s[h][t] = scale · (ν_{t,g}/d) · Σ_i q'_{h,i} · c[code_{t,g,i}],  g = ⌊h·hkv/hq⌋,
 // which equals scale·<q_h, x̂_{t,g}> without ever forming x̂.
 //
+// 4-bit codes at d ≤ 128 with a power-of-two group ≤ 8 (the KV-cache case) take
+// the tensor-core kernel further down (qk_scores_mma_kernel); the rest of this
+// header describes the general kernel, for every other width and d.
+//
 // Layout.  Each lane owns 32 consecutive coordinates of a key-head row
 // (d/32 lanes per key-head; KPW = 1024/d key-heads per warp iteration).  A
 // lane's GQA group of GQ query heads is fixed for the whole kernel, so its
