@@ -196,8 +196,10 @@ int rrq_drive_encode(const void* x, int x_dtype, int64_t n, int d, uint64_t seed
  *   codes   [T·hkv × d·bits/8] bytes, row t·hkv + g;  norms [T·hkv] float
  *   scores  [hq × T] float (output)
  * hq must be a multiple of hkv with hq/hkv in {1, 2, 4, 8}.
- * Accuracy: products in fp16 pairs with fp32 partial sums; the error is far
- * below 1e-3·‖q‖·‖x̂‖ for bits ≤ 4.
+ * Accuracy: fp16 query values (each head scaled by a power of two) times fp16
+ * levels, summed in fp32 (tensor-core tiles for 4-bit codes at d ≤ 128, fp16 pairs
+ * with fp32 partial sums otherwise); the error is far below 1e-3·‖q‖·‖x̂‖ for
+ * bits ≤ 4.
  * Errors: RRQ_ERR_INVALID, RRQ_ERR_UNSUPPORTED (group size), RRQ_ERR_CUDA.
  */
 int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norms, int64_t T,
@@ -222,8 +224,8 @@ int rrq_qk_scores(const void* q, int hq, const uint8_t* codes, const float* norm
  *   qjl_S      bf16 [d × d] (the S given to rrq_encode)
  *   scores     [hq × T] float (output)
  * d must be 128; hq a multiple of hkv with hq/hkv in {1, 2, 4, 8}.
- * Accuracy: both dot products in fp16 pairs with fp32 partial sums (every 32
- * products), each head's query and projected query scaled by a power of two.
+ * Accuracy: both dot products as fp16 × fp16 products summed in fp32 (tensor-core
+ * tiles), each head's query and projected query scaled by a power of two.
  * Errors: RRQ_ERR_INVALID, RRQ_ERR_UNSUPPORTED (d other than 128, group size),
  * RRQ_ERR_CUDA.
  */
@@ -252,10 +254,12 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
  *              that share a workspace must not overlap on the GPU.
  *   out        [hq × d] float (output)
  * d must be 128 and both codes 4-bit; hq a multiple of hkv with hq/hkv in
- * {1, 2, 4, 8}; T ≥ 1.  Scores in fp16 pairs with fp32 partial sums (as
- * rrq_qk_scores); softmax and the value sums in fp32.
+ * {1, 2, 4, 8}; T ≥ 1.  Scores as rrq_qk_scores (fp16 operands, fp32 sums);
+ * softmax in fp32; the value sums take fp16 levels and fp16 weights p·ν/√d with
+ * fp32 accumulation (within 2e-3 of the largest reconstruction).
  * Errors: RRQ_ERR_INVALID (incl. a workspace that is too small), RRQ_ERR_UNSUPPORTED
- * (d, bits, group size), RRQ_ERR_CUDA.
+ * (d, bits, group size, or a device whose per-block reserved shared memory is not
+ * the 1 KB the kernel's shared layout assumes), RRQ_ERR_CUDA.
  */
 int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
                          const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,

@@ -300,7 +300,8 @@ int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
   a.group = group;
   a.splits = rrq::attention_splits(hkv, group, T);
   a.scale = scale;
-  return status_of(rrq::launch_attention_decode_in_scratch(a, as_stream(stream)));
+  const cudaError_t e = rrq::launch_attention_decode_in_scratch(a, as_stream(stream));
+  return e == cudaErrorNotSupported ? RRQ_ERR_UNSUPPORTED : status_of(e);
 }
 
 size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int64_t T) {
@@ -346,7 +347,8 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
   a.counters = static_cast<unsigned*>(workspace);
   a.states = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                       (size_t(hkv) * 4 + 255) / 256 * 256);
-  return status_of(rrq::launch_attention_decode(a, as_stream(stream)));
+  const cudaError_t e = rrq::launch_attention_decode(a, as_stream(stream));
+  return e == cudaErrorNotSupported ? RRQ_ERR_UNSUPPORTED : status_of(e);
 }
 
 int rrq_q4_0_rot(const void* x, int x_dtype, int64_t n, int d, uint64_t seed, int rotate,
