@@ -399,7 +399,9 @@ int attention_splits(int hkv, int group, int64_t T) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   (void)group;  // one CTA per SM for every group
-  int64_t s = (int64_t(sms) + hkv - 1) / hkv;
+  // rounded down: one CTA more than the SMs hold would run as a second wave and
+  // double the kernel's time
+  int64_t s = int64_t(sms) / hkv;
   const int64_t ntile = (T + 31) / 32;
   const int64_t most = (ntile + kAWarps - 1) / kAWarps;  // every CTA gets a tile per warp
   if (s > most) s = most;
