@@ -145,3 +145,22 @@ def test_other_entry_points_validate():
     assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 100, 0, 0, P, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_drive_encode(P, B.RRQ_F16, 4, 128, 0, 1, P, P_MIS, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_drive_encode(ctypes.c_void_p(None), B.RRQ_F16, 0, 128, 0, 1, P, P, None) == B.RRQ_OK
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 1), (16, 2), (32, 32), (64, 8)])
+def test_attention_splits_fill_the_sms_in_one_wave(hq, hkv):
+    """The token ranges per kv head that rrq_attention_workspace_bytes implies: one CTA
+    per SM, rounded down so that hkv × ranges never exceeds the SM count (148 on this
+    part, and the library's default when no device is visible); a range per 16 tiles
+    of 32 tokens at most; at least one."""
+    lib = B.lib()
+    sms = 148
+    counters = (hkv * 4 + 255) // 256 * 256
+    for t_len in (1, 100, 4096, 1 << 17, 1 << 20):
+        ws = lib.rrq_attention_workspace_bytes(hq, hkv, 128, t_len)
+        per_range = hq * 130 * 4
+        assert (ws - counters) % per_range == 0
+        s = (ws - counters) // per_range
+        ntile = (t_len + 31) // 32
+        assert s == max(1, min(sms // hkv, (ntile + 15) // 16))
+        assert s * hkv <= max(sms, hkv)
