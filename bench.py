@@ -198,15 +198,46 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def cpu_baseline(x_flat: np.ndarray, budget_s: float = 12.0):
-    """The oracle as it stands on a bounded sample of the workload."""
-    n0 = 8192
-    t0 = oracle_step_time(x_flat[:n0])
-    n = int(min(x_flat.shape[0], max(n0, n0 * budget_s / max(t0, 1e-3) / 2)))
-    t = oracle_step_time(x_flat[:n])
-    return {"value": n / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    """The oracle as it stands on a bounded sample of the workload, timed twice: with
+    its BLAS on every core this process may use, and pinned to one thread.  About
+    budget_s seconds of wall time each."""
+    from threadpoolctl import threadpool_limits
+    cores = host_cores()
+    out = {}
+    for label, threads in (("all", cores), ("one", 1)):
+        with threadpool_limits(limits=threads):
+            n0 = 2048
+            t0 = oracle_step_time(x_flat[:n0])
+            n = int(min(x_flat.shape[0], max(n0, n0 * budget_s / max(t0, 1e-3) / 2)))
+            t = oracle_step_time(x_flat[:n])
+            out[label] = (n, t, min(threads, blas_threads()))
+    n, t, used = out["all"]
+    n1, t1, _ = out["one"]
+    return {"value": n / t, "unit": UNIT, "cores": used, "kind": "oracle",
             "sample": f"first {n} of the {x_flat.shape[0]} workload vectors, encode+decode, "
-                      f"numpy fp64 (dense rotation matrix), {t:.2f} s wall"}
+                      f"numpy fp64 (dense rotation matrix), {t:.2f} s wall, BLAS on {used} threads",
+            "cpu_model": cpu_model(), "host_cores": cores,
+            "single_thread": {"value": n1 / t1, "unit": UNIT, "cores": 1,
+                              "sample": f"first {n1} workload vectors, {t1:.2f} s wall, BLAS on 1 thread"}}
 
 
 # ------------------------------------------------------------ reference
@@ -236,7 +267,8 @@ def run_reference(args):
         "config": workload_config({"sample_vectors_per_step": n_sample,
                                    "l2": "n/a (the CPU oracle on the host cores)"}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"first {n_sample} workload vectors per step, encode+decode"},
+                         "sample": f"first {n_sample} workload vectors per step, encode+decode",
+                         "cpu_model": cpu_model(), "host_cores": host_cores()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -419,7 +451,20 @@ def run_gpu(args):
             "clocks": clocks,
         }
         if world == 1 and not args.no_extras:
-            line["kernels"] = extra_kernels(torch, dev, flush, 50, peak)
+            sel = set(args.extras.split(",")) if args.extras else None
+            line["kernels"] = extra_kernels(torch, dev, flush, 50, peak, sel)
+            if sel is None or "reports" in sel:
+                c_r, n_r = B.rrq_encode(xs[0], BITS, 42)
+                x_r = B.rrq_decode(c_r, n_r, D, BITS, 42, out_dtype=torch.float32)
+                kv_err = float(((x_r.double() - xs[0].double()) ** 2).sum())
+                line["reports"] = {
+                    "pr1": quality_reports(torch, dev),
+                    "kv_headline": {"nmse": kv_err / float((xs[0].double() ** 2).sum()),
+                                    "lloyd_max_distortion_D_b": lloyd_max_distortion(
+                                        B.rrq_codebook(BITS))},
+                    "attnrot_q4_0": {k: line["kernels"]["q4_0_rot"][k] for k in (
+                        "mse_rotated", "mse_unrotated", "mse_rotated_over_unrotated")}
+                    if "q4_0_rot" in line["kernels"] else None}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(x_host)
         print(json.dumps(line), flush=True)
@@ -458,7 +503,91 @@ def time_kernel(torch, stream, flush, fn, reps):
     return sum(e0.elapsed_time(e1) for e0, e1 in evs) / reps
 
 
-def extra_kernels(torch, dev, flush, reps, peak):
+def lloyd_max_distortion(levels) -> float:
+    """E[(X − Q(X))²] for X ~ N(0,1) under nearest-level quantisation with `levels`
+    (ascending), summed in closed form over the cells between midpoints."""
+    import math
+    lv = [float(c) for c in levels]
+    edges = [-math.inf] + [(lv[i] + lv[i + 1]) / 2 for i in range(len(lv) - 1)] + [math.inf]
+
+    def phi(x):
+        return 0.0 if math.isinf(x) else math.exp(-x * x / 2) / math.sqrt(2 * math.pi)
+
+    def cdf(x):
+        return 0.5 * (1 + math.erf(x / math.sqrt(2))) if not math.isinf(x) else (0.0 if x < 0 else 1.0)
+
+    def xphi(x):
+        return 0.0 if math.isinf(x) else x * phi(x)
+
+    tot = 0.0
+    for c, a, b in zip(lv, edges[:-1], edges[1:]):
+        mass = cdf(b) - cdf(a)
+        tot += mass * (1 + c * c) - (xphi(b) - xphi(a)) - 2 * c * (phi(a) - phi(b))
+    return tot
+
+
+def quality_reports(torch, dev):
+    """Reconstruction error of the GPU path on the PR1 workload (4096 fp32 vectors,
+    d = 128, three outlier channels x20, b = 2): MSE per coordinate, NMSE against the
+    Lloyd-Max distortion D_2 of N(0,1), and the NMSE of the same codebook applied
+    without the rotation.  The unrotated figure runs on the same kernels: encoding
+    Πᵀx with the rotating encoder quantises the coordinates of x itself (Π·Πᵀx = x),
+    and the decoder's Πᵀ is an isometry, so ‖decode − Πᵀx‖ is the unrotated error."""
+    from random_rotation_kv_b200 import binding as B
+    from random_rotation_kv_b200 import workloads as W
+    w = W.pr1()
+    x = torch.from_numpy(w.flat()).to(dev)
+    d, bits = w.d, w.bits
+
+    def nmse_of(v):
+        codes, norms = B.rrq_encode(v, bits, 42)
+        vh = B.rrq_decode(codes, norms, d, bits, 42, out_dtype=torch.float32)
+        err = float(((vh.double() - v.double()) ** 2).sum())
+        return err, err / float((v.double() ** 2).sum())
+
+    err, nmse = nmse_of(x)
+    _, nmse_u = nmse_of(B.rrq_rotate(x, 42, inverse=True))
+    d_b = lloyd_max_distortion(B.rrq_codebook(bits))
+    return {"workload": "PR1: 4096 fp32 vectors d=128, N(0,1) with channels {3,47,111} x20, b=2",
+            "mse": err / x.numel(), "nmse": nmse, "lloyd_max_distortion_D_b": d_b,
+            "nmse_over_D_b": nmse / d_b, "unrotated_nmse": nmse_u,
+            "unrotated_over_rotated_nmse": nmse_u / nmse}
+
+
+def scores_sweep(torch, dev, reps, peak):
+    """rrq_qk_scores over d in {64, 128, 256, 512} x b in {1, 2, 3, 4}: 32 query heads
+    against 131072 tokens x 8 kv heads, keys with the KV-cache distribution.  Each
+    case rotates over enough copies of its cache to exceed L2 (at least 3, and at
+    least 384 MB in all).  Bytes per key-head: d·b/8 code bytes + 4 norm bytes
+    + 4 scores of 4 bytes."""
+    from random_rotation_kv_b200 import binding as B
+    from random_rotation_kv_b200 import workloads as W
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for d in (64, 128, 256, 512):
+        w = W.scores(d=d)
+        t_len = w.x.shape[0]
+        k = torch.from_numpy(w.flat()).to(dev)
+        q = torch.from_numpy(w.extra["q"]).to(dev)
+        for bits in (1, 2, 3, 4):
+            codes, norms = B.rrq_encode(k, bits, 42)
+            per_copy = codes.numel() + 4 * norms.numel() + 32 * t_len * 4
+            copies = max(3, -(-(384 << 20) // per_copy))
+            cs = [(codes, norms)] + [(codes.clone(), norms.clone()) for _ in range(copies - 1)]
+            sc = [torch.empty(32, t_len, dtype=torch.float32, device=dev) for _ in range(copies)]
+            ms = time_loop(torch, stream, lambda i: B.rrq_qk_scores(
+                q, *cs[i % copies], 8, d, bits, 42, out=sc[i % copies]), reps)
+            nkh = t_len * 8
+            by = nkh * (d * bits // 8 + 4 + 16)
+            rows.append({"d": d, "bits": bits, "us": 1e3 * ms, "gbs": by / ms / 1e6,
+                         "frac_of_hbm": by / ms / 1e6 / peak, "copies": copies})
+            del cs, sc, codes, norms
+        del k
+    return {"workload": "32 q heads x [131072 tokens x 8 kv heads], KV distribution, scale 1",
+            "rows": rows}
+
+
+def extra_kernels(torch, dev, flush, reps, peak, sel=None):
     """Other hot-path kernels on their own workloads (not part of the headline step),
     each timed as `reps` back-to-back launches whose inputs exceed L2 (the 1M-vector
     inputs are 268 MB; the scores rotate over 3 copies of its 71 MB cache)."""
@@ -474,125 +603,150 @@ def extra_kernels(torch, dev, flush, reps, peak):
     tc_peak = float(mp["bf16_tflops"]) if mp else 1590.0
     out = {}
 
-    # workload 5: scores of 32 query heads against 131072 tokens x 8 KV heads, 4-bit codes
+    def want(name):
+        return sel is None or name in sel
+
     w = W.scores()
-    k = torch.from_numpy(w.flat()).to(dev)
-    codes, norms = B.rrq_encode(k, 4, 42)
-    del k
     q = torch.from_numpy(w.extra["q"]).to(dev)
-    cs = [codes] + [codes.clone() for _ in range(2)]
-    ns = [norms] + [norms.clone() for _ in range(2)]
-    scs = [torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev) for _ in range(3)]
-    ms = time_loop(torch, stream,
-                   lambda k: B.rrq_qk_scores(q, cs[k % 3], ns[k % 3], 8, 128, 4, 42, out=scs[k % 3]),
-                   reps)
     nkh = w.x.shape[0] * 8
-    by = nkh * (64 + 4) + 32 * w.x.shape[0] * 4
-    out["qk_scores"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128 b=4",
-                        "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
-                        "frac_of_hbm": by / ms / 1e6 / peak}
-    del codes, norms, cs, ns, scs
 
-    # one decode step of attention over a 4-bit K/V cache of the same shape
-    kt = torch.from_numpy(w.flat()).to(dev)
-    kc, kn_ = B.rrq_encode(kt, 4, 42)
-    vc, vn_ = B.rrq_encode(kt, 4, 43)  # values: the same tensor under another rotation
-    del kt
-    caches = [(kc, kn_, vc, vn_), (kc.clone(), kn_.clone(), vc.clone(), vn_.clone())]  # 2 x 142 MB
-    ao = torch.empty(32, 128, dtype=torch.float32, device=dev)
-    ws = torch.zeros(B.rrq_attention_workspace_bytes(32, 8, 128, w.x.shape[0]), dtype=torch.uint8,
-                     device=dev)
-    ms = time_loop(torch, stream, lambda i: B.rrq_attention_decode(
-        q, *caches[i % 2], 8, 128, 42, 43, scale=128 ** -0.5, out=ao, workspace=ws), reps)
-    by = nkh * (64 + 4) * 2 + 32 * 128 * 4
-    out["attention_decode"] = {"workload": "32 q heads over [131072 tokens x 8 kv heads] d=128, "
-                                           "4-bit K and V codes",
-                               "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
-                               "frac_of_hbm": by / ms / 1e6 / peak}
-    del caches, kc, kn_, vc, vn_
-
-    # unbiased scores on the same keys stored TurboQuant-style: 2-bit codes + QJL bits
-    S = B.rrq_qjl_matrix(4242, 128, device=dev)
-    k = torch.from_numpy(w.flat()).to(dev)
-    sets = []
-    for _ in range(3):  # 3 copies of 56 MB: larger than L2 in rotation
-        c2, n2, b2, r2 = B.rrq_encode(k, 2, 42, qjl_S=S)
-        sets.append((c2, n2, b2, r2))
-    del k
-    sc = [torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev) for _ in range(3)]
-    ms = time_loop(torch, stream, lambda i: B.rrq_qk_scores_qjl(
-        q, *sets[i % 3], S, 8, 128, 2, 42, out=sc[i % 3]), reps)
-    by = nkh * (32 + 4 + 16 + 4) + 32 * w.x.shape[0] * 4
-    out["qk_scores_qjl"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128, "
-                                        "2-bit codes + QJL bits (unbiased)",
+    # workload 5: scores of 32 query heads against 131072 tokens x 8 KV heads, 4-bit codes
+    if want("qk_scores"):
+        k = torch.from_numpy(w.flat()).to(dev)
+        codes, norms = B.rrq_encode(k, 4, 42)
+        del k
+        cs = [codes] + [codes.clone() for _ in range(2)]
+        ns = [norms] + [norms.clone() for _ in range(2)]
+        scs = [torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev) for _ in range(3)]
+        ms = time_loop(torch, stream,
+                       lambda k: B.rrq_qk_scores(q, cs[k % 3], ns[k % 3], 8, 128, 4, 42, out=scs[k % 3]),
+                       reps)
+        by = nkh * (64 + 4) + 32 * w.x.shape[0] * 4
+        out["qk_scores"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128 b=4",
                             "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
                             "frac_of_hbm": by / ms / 1e6 / peak}
-    del sets, sc
+        del codes, norms, cs, ns, scs
+
+        # one decode step of attention over a 4-bit K/V cache of the same shape
+    if want("attention_decode"):
+        kt = torch.from_numpy(w.flat()).to(dev)
+        kc, kn_ = B.rrq_encode(kt, 4, 42)
+        vc, vn_ = B.rrq_encode(kt, 4, 43)  # values: the same tensor under another rotation
+        del kt
+        caches = [(kc, kn_, vc, vn_), (kc.clone(), kn_.clone(), vc.clone(), vn_.clone())]  # 2 x 142 MB
+        ao = torch.empty(32, 128, dtype=torch.float32, device=dev)
+        ws = torch.zeros(B.rrq_attention_workspace_bytes(32, 8, 128, w.x.shape[0]), dtype=torch.uint8,
+                         device=dev)
+        ms = time_loop(torch, stream, lambda i: B.rrq_attention_decode(
+            q, *caches[i % 2], 8, 128, 42, 43, scale=128 ** -0.5, out=ao, workspace=ws), reps)
+        by = nkh * (64 + 4) * 2 + 32 * 128 * 4
+        out["attention_decode"] = {"workload": "32 q heads over [131072 tokens x 8 kv heads] d=128, "
+                                               "4-bit K and V codes",
+                                   "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
+                                   "frac_of_hbm": by / ms / 1e6 / peak}
+        del caches, kc, kn_, vc, vn_
+
+        # unbiased scores on the same keys stored TurboQuant-style: 2-bit codes + QJL bits
+    if want("qk_scores_qjl"):
+        S = B.rrq_qjl_matrix(4242, 128, device=dev)
+        k = torch.from_numpy(w.flat()).to(dev)
+        sets = []
+        for _ in range(3):  # 3 copies of 56 MB: larger than L2 in rotation
+            c2, n2, b2, r2 = B.rrq_encode(k, 2, 42, qjl_S=S)
+            sets.append((c2, n2, b2, r2))
+        del k
+        sc = [torch.empty(32, w.x.shape[0], dtype=torch.float32, device=dev) for _ in range(3)]
+        ms = time_loop(torch, stream, lambda i: B.rrq_qk_scores_qjl(
+            q, *sets[i % 3], S, 8, 128, 2, 42, out=sc[i % 3]), reps)
+        by = nkh * (32 + 4 + 16 + 4) + 32 * w.x.shape[0] * 4
+        out["qk_scores_qjl"] = {"workload": "32 q heads x [131072 tokens x 8 kv heads] d=128, "
+                                            "2-bit codes + QJL bits (unbiased)",
+                                "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
+                                "frac_of_hbm": by / ms / 1e6 / peak}
+        del sets, sc
+
+    if want("qk_scores_sweep"):
+        out["qk_scores_sweep"] = scores_sweep(torch, dev, reps, peak)
+
+    if want("q4_0_rot") or want("ggml") or want("drive_1bit"):
+        w = W.attnrot()
+        x = torch.from_numpy(w.flat()).to(dev)
+        n = x.shape[0]
 
     # workload 3: rotate-then-q4_0, 1,048,576 fp16 vectors
-    w = W.attnrot()
-    x = torch.from_numpy(w.flat()).to(dev)
-    n = x.shape[0]
-    blk = torch.empty(n, 72, dtype=torch.uint8, device=dev)
-    xo = torch.empty_like(x)
-    ms_e = time_loop(torch, stream, lambda k: B.rrq_q4_0_rot(x, 42, out=blk), reps)
-    ms_d = time_loop(torch, stream, lambda k: B.rrq_q4_0_rot_decode(blk, 128, 42, out=xo), reps)
-    by = n * (256 + 72)
-    out["q4_0_rot"] = {"workload": "fp16 [131072 x 8 x 128], rotate + q4_0", "encode_us": 1e3 * ms_e,
-                       "decode_us": 1e3 * ms_d, "encode_gbs": by / ms_e / 1e6,
-                       "decode_gbs": by / ms_d / 1e6, "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
-                       "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
-    del blk, xo
+    if want("q4_0_rot"):
+        blk = torch.empty(n, 72, dtype=torch.uint8, device=dev)
+        xo = torch.empty_like(x)
+        ms_e = time_loop(torch, stream, lambda k: B.rrq_q4_0_rot(x, 42, out=blk), reps)
+        ms_d = time_loop(torch, stream, lambda k: B.rrq_q4_0_rot_decode(blk, 128, 42, out=xo), reps)
+        by = n * (256 + 72)
+        # reconstruction MSE over all 1,048,576 vectors, rotated and unrotated q4_0
+        mse = {}
+        for rot in (True, False):
+            bq = B.rrq_q4_0_rot(x, 42, rotate=rot)
+            xq = B.rrq_q4_0_rot_decode(bq, 128, 42, rotate=rot, out_dtype=torch.float32)
+            mse[rot] = float(((xq.double() - x.double()) ** 2).mean())
+            del bq, xq
+        out["q4_0_rot"] = {"workload": "fp16 [131072 x 8 x 128], rotate + q4_0", "encode_us": 1e3 * ms_e,
+                           "decode_us": 1e3 * ms_d, "encode_gbs": by / ms_e / 1e6,
+                           "decode_gbs": by / ms_d / 1e6, "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
+                           "decode_frac_of_hbm": by / ms_d / 1e6 / peak,
+                           "mse_rotated": mse[True], "mse_unrotated": mse[False],
+                           "mse_rotated_over_unrotated": mse[True] / mse[False]}
+        del blk, xo
 
     # the other GGML block types on the same vectors (rotate, then blocks of 32)
-    for fmt in ("q4_1", "q5_0", "q5_1", "q8_0"):
-        per = 4 * B.rrq_ggml_block_bytes(fmt)
-        gb = torch.empty(n, per, dtype=torch.uint8, device=dev)
+    if want("ggml"):
+        for fmt in ("q4_1", "q5_0", "q5_1", "q8_0"):
+            per = 4 * B.rrq_ggml_block_bytes(fmt)
+            gb = torch.empty(n, per, dtype=torch.uint8, device=dev)
+            xo = torch.empty_like(x)
+            ms_e = time_loop(torch, stream, lambda k: B.rrq_ggml_rot(x, 42, fmt, out=gb), reps)
+            ms_d = time_loop(torch, stream, lambda k: B.rrq_ggml_rot_decode(gb, 128, 42, fmt, out=xo), reps)
+            by = n * (256 + per)
+            out[f"{fmt}_rot"] = {"workload": f"fp16 [131072 x 8 x 128], rotate + {fmt}",
+                                 "encode_us": 1e3 * ms_e, "decode_us": 1e3 * ms_d,
+                                 "encode_gbs": by / ms_e / 1e6, "decode_gbs": by / ms_d / 1e6,
+                                 "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
+                                 "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
+            del gb, xo
+
+    # DRIVE one-bit encode (unbiased scale) of the same vectors, and the
+    # one-bit decode back to fp16
+    if want("drive_1bit"):
+        dc = torch.empty(n, 16, dtype=torch.uint8, device=dev)
+        ds = torch.empty(n, dtype=torch.float32, device=dev)
         xo = torch.empty_like(x)
-        ms_e = time_loop(torch, stream, lambda k: B.rrq_ggml_rot(x, 42, fmt, out=gb), reps)
-        ms_d = time_loop(torch, stream, lambda k: B.rrq_ggml_rot_decode(gb, 128, 42, fmt, out=xo), reps)
-        by = n * (256 + per)
-        out[f"{fmt}_rot"] = {"workload": f"fp16 [131072 x 8 x 128], rotate + {fmt}",
+        ms_e = time_loop(torch, stream,
+                         lambda k: B.rrq_drive_encode(x, 42, True, codes=dc, scales=ds), reps)
+        ms_d = time_loop(torch, stream, lambda k: B.rrq_decode(
+            dc, ds, 128, 1, 42, codebook=[-1.0, 1.0], out=xo), reps)
+        by = n * (256 + 16 + 4)
+        out["drive_1bit"] = {"workload": "fp16 [131072 x 8 x 128], DRIVE sign + unbiased scale",
                              "encode_us": 1e3 * ms_e, "decode_us": 1e3 * ms_d,
                              "encode_gbs": by / ms_e / 1e6, "decode_gbs": by / ms_d / 1e6,
                              "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
                              "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
-        del gb, xo
-
-    # DRIVE one-bit encode (unbiased scale) of the same vectors, and the
-    # one-bit decode back to fp16
-    dc = torch.empty(n, 16, dtype=torch.uint8, device=dev)
-    ds = torch.empty(n, dtype=torch.float32, device=dev)
-    xo = torch.empty_like(x)
-    ms_e = time_loop(torch, stream,
-                     lambda k: B.rrq_drive_encode(x, 42, True, codes=dc, scales=ds), reps)
-    ms_d = time_loop(torch, stream, lambda k: B.rrq_decode(
-        dc, ds, 128, 1, 42, codebook=[-1.0, 1.0], out=xo), reps)
-    by = n * (256 + 16 + 4)
-    out["drive_1bit"] = {"workload": "fp16 [131072 x 8 x 128], DRIVE sign + unbiased scale",
-                         "encode_us": 1e3 * ms_e, "decode_us": 1e3 * ms_d,
-                         "encode_gbs": by / ms_e / 1e6, "decode_gbs": by / ms_d / 1e6,
-                         "encode_frac_of_hbm": by / ms_e / 1e6 / peak,
-                         "decode_frac_of_hbm": by / ms_d / 1e6 / peak}
-    del x, dc, ds, xo
+        del dc, ds, xo
 
     # workload 4: 2-bit codes + QJL sketch, 1,048,576 bf16 vectors (tcgen05 projection)
-    w = W.turbo()
-    x = torch.from_numpy(w.flat()).to(dev).to(torch.bfloat16)
-    n = x.shape[0]
-    S = B.rrq_qjl_matrix(4242, 128, device=dev)
-    cq = torch.empty(n, 32, dtype=torch.uint8, device=dev)
-    nq = torch.empty(n, dtype=torch.float32, device=dev)
-    qb = torch.empty(n, 16, dtype=torch.uint8, device=dev)
-    rq = torch.empty(n, dtype=torch.float32, device=dev)
-    ms = time_loop(torch, stream, lambda k: B.rrq_encode(
-        x, 2, 42, codes=cq, norms=nq, qjl_S=S, qjl_bits=qb, qjl_rnorm=rq), reps)
-    by = n * (256 + 32 + 4 + 16 + 4)
-    flops = n * 2 * 2 * 128 * 128  # two fp16 MMA passes (residual split r_hi + r_lo)
-    out["encode_qjl"] = {"workload": "bf16 [1048576 x 128], b=2 + QJL (2 fp16 MMA passes per tile)",
-                         "us": 1e3 * ms, "gbs": by / ms / 1e6, "frac_of_hbm": by / ms / 1e6 / peak,
-                         "tensor_tflops": flops / ms / 1e9,
-                         "frac_of_tensor_peak": flops / ms / 1e9 / tc_peak}
+    if want("encode_qjl"):
+        w = W.turbo()
+        x = torch.from_numpy(w.flat()).to(dev).to(torch.bfloat16)
+        n = x.shape[0]
+        S = B.rrq_qjl_matrix(4242, 128, device=dev)
+        cq = torch.empty(n, 32, dtype=torch.uint8, device=dev)
+        nq = torch.empty(n, dtype=torch.float32, device=dev)
+        qb = torch.empty(n, 16, dtype=torch.uint8, device=dev)
+        rq = torch.empty(n, dtype=torch.float32, device=dev)
+        ms = time_loop(torch, stream, lambda k: B.rrq_encode(
+            x, 2, 42, codes=cq, norms=nq, qjl_S=S, qjl_bits=qb, qjl_rnorm=rq), reps)
+        by = n * (256 + 32 + 4 + 16 + 4)
+        flops = n * 2 * 2 * 128 * 128  # two fp16 MMA passes (residual split r_hi + r_lo)
+        out["encode_qjl"] = {"workload": "bf16 [1048576 x 128], b=2 + QJL (2 fp16 MMA passes per tile)",
+                             "us": 1e3 * ms, "gbs": by / ms / 1e6, "frac_of_hbm": by / ms / 1e6 / peak,
+                             "tensor_tflops": flops / ms / 1e9,
+                             "frac_of_tensor_peak": flops / ms / 1e9 / tc_peak}
     return out
 
 
@@ -613,6 +767,10 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip timing the other kernels (scores, q4_0, QJL) on their workloads")
+    ap.add_argument("--extras", default="",
+                    help="comma-separated subset of the other kernels and reports (qk_scores, "
+                         "attention_decode, qk_scores_qjl, qk_scores_sweep, q4_0_rot, ggml, "
+                         "drive_1bit, encode_qjl, reports); default all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps, always
     if args.impl == "reference":

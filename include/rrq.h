@@ -255,8 +255,11 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
  *   out        [hq × d] float (output)
  * d must be 128 and both codes 4-bit; hq a multiple of hkv with hq/hkv in
  * {1, 2, 4, 8}; T ≥ 1.  Scores as rrq_qk_scores (fp16 operands, fp32 sums);
- * softmax in fp32; the value sums take fp16 levels and fp16 weights p·ν/√d with
- * fp32 accumulation (within 2e-3 of the largest reconstruction).
+ * softmax in fp32.  The value sums take fp16 levels and fp16 weights with fp32
+ * accumulation; the weights are p·ν relative to the largest p·ν of the head
+ * (exponent and log2 ν added before the one exponential), so any finite value
+ * norm keeps its precision: per head the output is within 2e-3·Σ_t p_t·‖v̂_t‖ of
+ * the exact softmax-weighted sum of the reconstructions.
  * Errors: RRQ_ERR_INVALID (incl. a workspace that is too small), RRQ_ERR_UNSUPPORTED
  * (d, bits, group size, or a device whose per-block reserved shared memory is not
  * the 1 KB the kernel's shared layout assumes), RRQ_ERR_CUDA.
@@ -278,8 +281,10 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
  * GPU that loads the library holds those 4 MiB until the process exits.  Requests
  * whose workspace (rrq_attention_workspace_bytes) exceeds 4 MiB are rejected with
  * RRQ_ERR_SCRATCH before anything is launched.
- * The first call on a device looks up the array's address on that device (once);
- * make that first call before any stream capture.  Each call clears the array's
+ * The first call on a device looks up the array's address on that device (once)
+ * and keeps it for the life of the process; make that first call before any
+ * stream capture.  A cudaDeviceReset() of that device invalidates the kept
+ * address: do not call this entry on a device after resetting it.  Each call clears the array's
  * counters on `stream` before its kernel runs.  All calls share the one array:
  * calls whose GPU work overlaps (other streams, other host threads) race and
  * give wrong results; calls ordered on one stream are safe.

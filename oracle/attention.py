@@ -28,8 +28,9 @@ from .rrq import as_f64
 
 def decode_attention(q, k_packed, k_norms, v_packed, v_norms, t_len: int, hkv: int, d: int,
                      k_bits: int, v_bits: int, k_seed: int, v_seed: int, k_levels=None,
-                     v_levels=None, scale: float = 1.0) -> np.ndarray:
-    """out [Hq, d] float64.  Cache rows are n = t·Hkv + g for both K and V."""
+                     v_levels=None, scale: float = 1.0, return_weights: bool = False):
+    """out [Hq, d] float64.  Cache rows are n = t·Hkv + g for both K and V.
+    With return_weights, also the softmax weights p [Hq, T]."""
     q = as_f64(q)
     hq = q.shape[0]
     s = rrq.scores(q, k_packed, k_norms, t_len, hkv, d, k_bits, k_seed, k_levels, scale)
@@ -41,4 +42,4 @@ def decode_attention(q, k_packed, k_norms, v_packed, v_norms, t_len: int, hkv: i
     for h in range(hq):
         g = rrq.kv_group(h, hq, hkv)
         out[h] = p[h] @ v_hat[:, g, :]
-    return out
+    return (out, p) if return_weights else out

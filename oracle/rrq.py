@@ -11,7 +11,7 @@
   nearest of 2^b centroids and reconstructs with Πᵀ; the inner-product decoder
   recovers <q, x> from <Πq, code(Πx)> and a normalising scalar.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * per-vector scale is ν = ‖x‖₂ of the input, stored as fp32; the normalised
   coordinate is u = √d·(Πx)_i / ν, which is about N(0,1);

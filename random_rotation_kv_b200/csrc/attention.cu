@@ -17,8 +17,17 @@
 // contractions of a tile run as mma.sync m16n8k16 tiles (fp16 operands, fp32
 // accumulation; the group padded to 8 columns), their A fragments looked up from
 // lane-replicated tables of level pairs; the online softmax runs on the score
-// fragments, and the weights w = p·ν^V/√d reach the value product through a
+// fragments in base 2, and the value weights reach the value product through a
 // per-warp transpose buffer (attention_decode_kernel says how).
+//
+// Range of the value weights.  The value product takes fp16 weights.  Rather
+// than p·ν^V (which flushes to zero for small value norms and overflows for
+// large ones), a weight is 2^(z − M + kWBias) with z = s·log2(e) + log2(ν^V) and
+// M the running maximum of z: the token with the largest p·ν^V weighs
+// 2^kWBias, no weight overflows, and only terms below 2^-(24 + kWBias) of the
+// largest one flush, at any scale of the value norms.  The softmax denominator
+// Σ 2^(s·log2(e) − m) keeps its own running maximum m, in fp32; the two meet
+// once, in the final factor 2^(M − m − kWBias)/Σ.
 // The warps' states merge within the CTA (shared-memory atomics after a common
 // rescaling); each CTA writes its state (max, sum, G×128 partial sums) to the
 // caller's workspace and counts itself in its kv head's counter there.  The
@@ -38,6 +47,20 @@ constexpr int kAD = 128;
 constexpr int kAWarps = 16;
 constexpr int kAThreads = kAWarps * 32;
 constexpr int kWRow = 40;  // fp16 weights per head row of a warp's transpose buffer (padded)
+constexpr float kWBias = 14.f;  // log2 of the largest value weight (fp16 holds up to 65504)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x and log2(x) (the SFU approximations; relative error about 2^-22).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Shared memory, as offsets from the dynamic base at shared address kBase (the
 // launch checks the device's reserved shared memory; the kernel checks the
@@ -52,12 +75,12 @@ template <int G> struct ALayout {
   static constexpr uint32_t QF = BF + 4 * 32 * 16;               // [G][kAD] fp32 q' (prologue)
   static constexpr uint32_t INV = QF + G * kAD * 4;              // [G] 1/s
   static constexpr uint32_t WBUF = (INV + G * 4 + 15) / 16 * 16; // per warp: [8][kWRow] fp16 weights
-  static constexpr uint32_t WM = WBUF + kAWarps * 8 * kWRow * 2; // [kAWarps][G] warp maxima
-  static constexpr int PART_FLOATS = 2 * G + G * kAD;           // [G] m, [G] l, [G][kAD] o
-  static constexpr uint32_t PART = WM + kAWarps * G * 4;         // the CTA's partial state
+  static constexpr uint32_t WM = WBUF + kAWarps * 8 * kWRow * 2; // [kAWarps][2G] warp maxima m, M
+  static constexpr int PART_FLOATS = 3 * G + G * kAD;           // [G] m, [G] l, [G] M, [G][kAD] o
+  static constexpr uint32_t PART = WM + kAWarps * 2 * G * 4;     // the CTA's partial state
   static constexpr uint32_t FLAG = PART + PART_FLOATS * 4;       // "this CTA merges its kv head"
-  static constexpr uint32_t FIN = (FLAG + 16 + 15) / 16 * 16;    // the merging CTA's sums [G][kAD + 1]
-  static constexpr uint32_t END = FIN + G * (kAD + 1) * 4;
+  static constexpr uint32_t FIN = (FLAG + 16 + 15) / 16 * 16;    // the merging CTA's sums [G][kAD], [G] l, [G] M − m
+  static constexpr uint32_t END = FIN + G * (kAD + 2) * 4;
   static constexpr uint32_t TOTAL = VTAB + 256 * 256;
   static_assert(END <= KTAB, "the small buffers fit below the K table");
   static_assert(TOTAL <= 227 * 1024, "shared memory");
@@ -107,9 +130,9 @@ __device__ __forceinline__ void fwht128(float (&v)[4], int lane) {
 //  A. scores S[32 tokens × 8] = levels(K codes)·q'' as in the score kernel:
 //     rows qr + 8m (m = 0..3) are the thread's tokens, its code slice is bytes
 //     [16qc, 16qc + 16), columns 2qc, 2qc + 1 its heads.
-//  B. the online softmax per head on those fragments (max and sum over the
-//     tile by shuffles across the 8 lanes of equal qc); the weights
-//     w = p·ν^V/√d go to the warp's transpose buffer as fp16 [head][token].
+//  B. the online softmax per head on those fragments (maxima and sum over the
+//     tile by shuffles across the 8 lanes of equal qc); the value weights
+//     2^(z − M + kWBias) go to the warp's transpose buffer as fp16 [head][token].
 //  C. O^T[128 × 8] += levels(V codes)^T·W^T: coordinates are M, heads N,
 //     tokens K.  Row qr of m-tile mt is coordinate 2(8qr + mt) and row qr + 8
 //     coordinate 2(8qr + mt) + 1, so both come from V byte 8qr + mt; for the
@@ -195,17 +218,18 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   const int qc = lane & 3, qr = lane >> 2;
   // this lane's B fragment words, read per k-step (registers are the scarce resource)
   const uint2* bq = reinterpret_cast<const uint2*>(bf) + lane * 2;
-  const float vscale = a.pv.inv_sqrt_d;
-  float kse[2];  // scale·inv_d/s of heads 2qc + e
+  float kse[2];  // log2(e)·scale·inv_d/s of heads 2qc + e: scores in base 2
 #pragma unroll
-  for (int e = 0; e < 2; ++e) kse[e] = 2 * qc + e < G ? a.scale * a.pk.inv_d * inv_s[2 * qc + e] : 0.f;
+  for (int e = 0; e < 2; ++e)
+    kse[e] = 2 * qc + e < G ? kLog2e * a.scale * a.pk.inv_d * inv_s[2 * qc + e] : 0.f;
   const uint32_t kcol = 0x10000u | uint32_t(lane) * 4u;
   const uint32_t vcol = 0x20000u | uint32_t(lane) * 4u;
 
   // ---- token tiles of kv head g (warp-major over the S CTAs' warps)
   const int64_t ntile = (a.T + 31) / 32;
   const int64_t stride = int64_t(S) * kAWarps;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  // per head: score maximum m, denominator l, maximum M of z = s + log2 ν^V
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f}, M_run[2] = {-INFINITY, -INFINITY};
   float o[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
@@ -248,37 +272,50 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
       }
     }
 
-    // B. online softmax per head; weights to the transpose buffer
+    // B. online softmax per head (base 2); value weights to the transpose buffer
+    float lv[4];  // log2 ν^V: −inf for a zero norm and for a token past T
+#pragma unroll
+    for (int m = 0; m < 4; ++m) lv[m] = lg2(vn[m]);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int h = 2 * qc + e;
-      float s[4];
-      float mt = -INFINITY;
+      float s[4], z[4];
+      float mt = -INFINITY, zt = -INFINITY;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const bool ok = t0 + qr + 8 * m < a.T;
         s[m] = ok ? kse[e] * kn[m] * sacc[m >> 1][2 * (m & 1) + e] : -INFINITY;
+        z[m] = s[m] + lv[m];
         mt = fmaxf(mt, s[m]);
+        zt = fmaxf(zt, z[m]);
       }
 #pragma unroll
-      for (int sh = 4; sh < 32; sh <<= 1) mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, sh));
+      for (int sh = 4; sh < 32; sh <<= 1) {
+        mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, sh));
+        zt = fmaxf(zt, __shfl_xor_sync(kFull, zt, sh));
+      }
       const float mn = fmaxf(m_run[e], mt);  // finite: the tile holds a valid token
-      const float alpha = __expf(m_run[e] - mn);
+      const float zn = fmaxf(M_run[e], zt);  // −inf while every value norm so far is 0
+      const bool live = zn != -INFINITY;
+      const float alpha = ex2(m_run[e] - mn);            // 0 on the first tile
+      const float beta = live ? ex2(M_run[e] - zn) : 0.f;
+      const float zb = zn - kWBias;
       float ps = 0.f;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const float p = __expf(s[m] - mn);  // 0 for a token past T
-        ps += p;
-        if (h < G) wbuf[h * kWRow + qr + 8 * m] = __float2half_rn(p * vn[m] * vscale);
+        ps += ex2(s[m] - mn);  // 0 for a token past T
+        const float w = live ? ex2(z[m] - zb) : 0.f;
+        if (h < G) wbuf[h * kWRow + qr + 8 * m] = __float2half_rn(w);
       }
 #pragma unroll
       for (int sh = 4; sh < 32; sh <<= 1) ps += __shfl_xor_sync(kFull, ps, sh);
       l_run[e] = l_run[e] * alpha + ps;
       m_run[e] = mn;
+      M_run[e] = zn;
 #pragma unroll
       for (int mt2 = 0; mt2 < 8; ++mt2) {
-        o[mt2][e] *= alpha;
-        o[mt2][2 + e] *= alpha;
+        o[mt2][e] *= beta;
+        o[mt2][2 + e] *= beta;
       }
     }
     __syncwarp();
@@ -302,32 +339,42 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
     __syncwarp();  // the buffer is read before the next tile writes it
   }
 
-  // ---- merge the warps' states: CTA maximum per head, then rescaled sums by
+  // ---- merge the warps' states: CTA maxima per head, then rescaled sums by
   // shared-memory atomics.  Accumulator o[mt][i]: coordinate 16qr + 2mt + (i >> 1),
   // head 2qc + (i & 1).
   if (qr == 0) {
 #pragma unroll
     for (int e = 0; e < 2; ++e)
-      if (2 * qc + e < G) wmax[warp * G + 2 * qc + e] = m_run[e];
+      if (2 * qc + e < G) {
+        wmax[warp * 2 * G + 2 * qc + e] = m_run[e];
+        wmax[warp * 2 * G + G + 2 * qc + e] = M_run[e];
+      }
   }
   __syncthreads();
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int h = 2 * qc + e;
     if (h < G) {
-      float mx = -INFINITY;
-      for (int w = 0; w < kAWarps; ++w) mx = fmaxf(mx, wmax[w * G + h]);
-      const float f = m_run[e] == -INFINITY ? 0.f : __expf(m_run[e] - mx);
-      float* oh = part + 2 * G + h * kAD + 16 * qr;
-      if (f > 0.f) {
+      float mx = -INFINITY, zx = -INFINITY;
+      for (int w = 0; w < kAWarps; ++w) {
+        mx = fmaxf(mx, wmax[w * 2 * G + h]);
+        zx = fmaxf(zx, wmax[w * 2 * G + G + h]);
+      }
+      const float fl = m_run[e] == -INFINITY ? 0.f : ex2(m_run[e] - mx);
+      const float fo = M_run[e] == -INFINITY ? 0.f : ex2(M_run[e] - zx);
+      float* oh = part + 3 * G + h * kAD + 16 * qr;
+      if (fo > 0.f) {
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          atomicAdd(oh + 2 * mt, f * o[mt][e]);
-          atomicAdd(oh + 2 * mt + 1, f * o[mt][2 + e]);
+          atomicAdd(oh + 2 * mt, fo * o[mt][e]);
+          atomicAdd(oh + 2 * mt + 1, fo * o[mt][2 + e]);
         }
-        if (qr == 0) atomicAdd(part + G + h, f * l_run[e]);
       }
-      if (warp == 0 && qr == 0) part[h] = mx;
+      if (fl > 0.f && qr == 0) atomicAdd(part + G + h, fl * l_run[e]);
+      if (warp == 0 && qr == 0) {
+        part[h] = mx;
+        part[2 * G + h] = zx;
+      }
     }
   }
   __syncthreads();
@@ -344,27 +391,36 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
   __threadfence();
   for (int idx = tid; idx < G * (kAD + 1); idx += kAThreads) {
     const int j = idx / (kAD + 1), c = idx % (kAD + 1);
-    // unrolled so that each batch of loads is in flight at once (the order of
-    // the additions is unchanged)
+    // the sums of the value product (c < kAD) carry the maximum M, the softmax
+    // denominator (c = kAD) the maximum m.  Unrolled so that each batch of loads
+    // is in flight at once (the order of the additions is unchanged).
+    const int mo = c < kAD ? 2 * G + j : j;
     float mx = -INFINITY;
 #pragma unroll 8
-    for (int r = 0; r < S; ++r) mx = fmaxf(mx, __ldcg(states + r * L::PART_FLOATS + j));
+    for (int r = 0; r < S; ++r) mx = fmaxf(mx, __ldcg(states + r * L::PART_FLOATS + mo));
     float acc = 0.f;
 #pragma unroll 8
     for (int r = 0; r < S; ++r) {
       const float* pr = states + r * L::PART_FLOATS;
-      const float m = __ldcg(pr + j);
-      const float f = m == -INFINITY ? 0.f : __expf(m - mx);
-      acc += f * __ldcg(c < kAD ? pr + 2 * G + j * kAD + c : pr + G + j);
+      const float m = __ldcg(pr + mo);
+      const float f = m == -INFINITY ? 0.f : ex2(m - mx);
+      acc += f * __ldcg(c < kAD ? pr + 3 * G + j * kAD + c : pr + G + j);
     }
-    if (c < kAD) fin[j * kAD + c] = acc;  // Σ over every token of the rotated-domain sum
-    else fin[G * kAD + j] = acc;        // the softmax denominator
+    if (c < kAD) {
+      fin[j * kAD + c] = acc;  // Σ over every token of the rotated-domain sum
+    } else {
+      float zx = -INFINITY;
+#pragma unroll 8
+      for (int r = 0; r < S; ++r) zx = fmaxf(zx, __ldcg(states + r * L::PART_FLOATS + 2 * G + j));
+      fin[G * kAD + j] = acc;                // the softmax denominator
+      fin[G * kAD + G + j] = zx == -INFINITY ? 0.f : ex2(zx - mx - kWBias);  // 2^(M − m − kWBias)
+    }
   }
   if (tid == 0) *counter = 0u;  // every CTA of this kv head has counted: ready for the next call
   __syncthreads();
   for (int j = warp; j < G; j += kAWarps) {
     const float lsum = fin[G * kAD + j];
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const float inv = lsum > 0.f ? fin[G * kAD + G + j] / lsum : 0.f;
     float v[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) v[k] = fin[j * kAD + lane * 4 + k] * inv;
@@ -372,7 +428,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attention_decode_kernel(const At
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = lane * 4 + k;
-      const float y = v[k] * a.pv.inv_sqrt_d;
+      const float y = v[k] * a.pv.inv_d;  // 1/√d of the reconstruction, 1/√d of Πᵀ
       a.out[int64_t(g * G + j) * kAD + i] = sign_bit(a.pv.seed, i) ? -y : y;
     }
   }
@@ -411,7 +467,7 @@ int attention_splits(int hkv, int group, int64_t T) {
 size_t attention_workspace_bytes(int hq, int hkv, int64_t T) {
   const int s = attention_splits(hkv, hq / hkv, T);
   const size_t counters = (size_t(hkv) * 4 + 255) / 256 * 256;
-  return counters + size_t(hq) * s * (kAD + 2) * 4;
+  return counters + size_t(hq) * s * (kAD + 3) * 4;
 }
 
 // ------------------------------------------------ allocation-free variant

@@ -18,7 +18,7 @@ struct AttnArgs {
   const float* v_norms;     // [T·hkv]
   float* out;               // [hq × 128]
   unsigned* counters;       // [hkv] in the workspace, zero between calls
-  float* states;            // [hkv × splits × G·130] in the workspace
+  float* states;            // [hkv × splits × G·131] in the workspace
   int64_t T;
   int hq, hkv, group, splits;
   float scale;
@@ -28,7 +28,7 @@ struct AttnArgs {
 // Token ranges per kv head for a cache of T tokens on the current device (as
 // many CTAs as the device has SMs, one each), and the
 // workspace bytes a call needs: hkv counters (padded to 256 bytes), then
-// hq × splits × 130 floats of partial states.
+// hq × splits × 131 floats of partial states (per head: m, l, M and 128 sums).
 int attention_splits(int hkv, int group, int64_t T);
 size_t attention_workspace_bytes(int hq, int hkv, int64_t T);
 

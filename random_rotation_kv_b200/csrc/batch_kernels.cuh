@@ -30,8 +30,11 @@
 //    and leave in one bulk store per batch; norms are plain coalesced stores.
 #pragma once
 
+#include <cstdlib>
+
 #include "quant_kernels.cuh"
 #include "tensor_map.h"
+#include "mma_encode.cuh"
 
 namespace rrq {
 
@@ -59,11 +62,6 @@ template <> __device__ __forceinline__ float2 first_butterfly<__nv_bfloat16>(uin
   return *reinterpret_cast<float2*>(&r);
 }
 
-__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
-  float2 v;
-  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
 
 // OR code c (B bits) of coordinate i into a little-endian word array.
 template <int B>
@@ -297,6 +295,12 @@ encode_batch_kernel(const __grid_constant__ CUtensorMap xmap, int64_t n, uint8_t
 template <typename T, int D, int B>
 cudaError_t launch_encode_batch(const T* x, int64_t n, const QuantParams& p, uint8_t* codes,
                                 float* norms, cudaStream_t stream) {
+  if constexpr (D == 128 && B == 4) {
+    if (p.norm_mode == 0 && getenv("RRQ_ENC_LANE") == nullptr) {
+      const cudaError_t e = launch_encode_mma<T>(x, n, p, codes, norms, stream);
+      if (e != cudaErrorNotSupported) return e;
+    }
+  }
   using SM = EncBatch<T, D, B>;
   CUtensorMap xmap;
   if (!row_tensor_map(&xmap, x, n, D, 2, 32)) return cudaErrorNotSupported;

@@ -11,7 +11,10 @@ Tolerances (stated for this hot path, and derived where they were not):
   must be fewer than 1e-4 of all codes;
 * scores: |s_gpu − s_oracle| ≤ 1e-3·‖q‖·‖k̂‖·|scale| (per-element relative error
   is undefined near 0, so the Cauchy–Schwarz scale of the score is used);
-* norms: relative error ≤ d·2⁻²⁴ (worst case of an fp32 sum of d squares).
+* norms: relative error ≤ d·2⁻²⁴ (worst case of an fp32 sum of d squares);
+* decode attention: per query head, ‖out_gpu − out_oracle‖ ≤ 2e-3·Σ_t p_t·‖v̂_t‖
+  with p the oracle's softmax weights (the reconstruction tolerance carried
+  through the convex combination by the triangle inequality).
 """
 
 from __future__ import annotations
@@ -82,3 +85,14 @@ def assert_scores_close(s_gpu, s_orc, cs_scale, scale=1.0, what=""):
     bound = 1e-3 * cs_scale * abs(scale)
     ok = err <= bound + 1e-30
     assert ok.all(), f"{what}: {np.sum(~ok)} scores off; worst ratio {np.max(err / np.maximum(bound, 1e-300))}"
+
+
+def attention_bound(p, v_packed, v_norms, t_len, hkv, d, v_bits, v_seed, v_levels=None,
+                    rel=2e-3):
+    """rel·Σ_t p[h,t]·‖v̂_{t,g(h)}‖ per query head, v̂ the oracle's value reconstructions."""
+    from oracle import rrq as orc
+    v_hat = orc.decode_exact(v_packed, v_norms, v_bits, d, v_seed, v_levels).reshape(t_len, hkv, d)
+    vnorm = np.linalg.norm(v_hat, axis=2)  # [T, hkv]
+    hq = p.shape[0]
+    g = np.array([orc.kv_group(h, hq, hkv) for h in range(hq)])
+    return rel * np.einsum("ht,ht->h", p, vnorm[:, g].T)

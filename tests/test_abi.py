@@ -150,15 +150,16 @@ def test_other_entry_points_validate():
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 1), (16, 2), (32, 32), (64, 8)])
 def test_attention_splits_fill_the_sms_in_one_wave(hq, hkv):
     """The token ranges per kv head that rrq_attention_workspace_bytes implies: one CTA
-    per SM, rounded down so that hkv × ranges never exceeds the SM count (148 on this
-    part, and the library's default when no device is visible); a range per 16 tiles
-    of 32 tokens at most; at least one."""
+    per SM, rounded down so that hkv × ranges never exceeds the SM count (that of
+    the visible device; 148, the library's default, when none is visible); a range
+    per 16 tiles of 32 tokens at most; at least one."""
+    import torch
     lib = B.lib()
-    sms = 148
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
     counters = (hkv * 4 + 255) // 256 * 256
     for t_len in (1, 100, 4096, 1 << 17, 1 << 20):
         ws = lib.rrq_attention_workspace_bytes(hq, hkv, 128, t_len)
-        per_range = hq * 130 * 4
+        per_range = hq * 131 * 4
         assert (ws - counters) % per_range == 0
         s = (ws - counters) // per_range
         ntile = (t_len + 31) // 32

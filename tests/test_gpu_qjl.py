@@ -101,24 +101,37 @@ def test_qjl_codes_equal_plain_encode():
 
 
 def test_qjl_full_size_sampled():
-    """Workload 4: 1,048,576 bf16 vectors; sampled rows against the oracle."""
+    """Workload 4: 1,048,576 bf16 vectors in one launch; 2000 sampled rows (plus the
+    first and the last) held to the same rules as the small cases: codes with the
+    boundary exemption, norms to fp32 summation order, residual norms to 1e-4 and
+    sign bits outside the 1e-5·ρ band, with the exempt bits under 1e-4."""
     w = W.turbo()
     x = w.flat()
     xd = to_dev(x, "bf16")
     s_dev = B.rrq_qjl_matrix(4242, 128, device=DEV)
     codes, norms, qb, rn = B.rrq_encode(xd, 2, 42, qjl_S=s_dev)
     torch.cuda.synchronize()
+    assert torch.all(torch.isfinite(rn)), "a tensor-core stage timed out (NaN residual norm)"
     rows = np.sort(np.random.default_rng(4).choice(x.shape[0], 2000, replace=False))
-    rows = np.concatenate([rows, [0, x.shape[0] - 1]])
+    rows = np.concatenate([[0], rows, [x.shape[0] - 1]])
     r_t = torch.from_numpy(rows).to(DEV)
     enc = oqjl.encode(x[rows].astype(np.float64), 2, 42, s_matrix())
+    tau = ocb.thresholds(ocb.lloyd_max(2))
     gc = P.unpack_codes(codes[r_t].cpu().numpy(), 2, 128)
+    P.assert_codes_match(gc, enc.enc.codes, enc.enc.u, tau, "qjl full size")
+    P.assert_norms_close(norms[r_t].cpu().numpy(), enc.enc.norm64, 128, "qjl full size")
     same = np.all(gc == enc.enc.codes, axis=1)
+    assert same.mean() > 0.99
+    rho = enc.rnorm.astype(np.float64)
+    rn_s = rn[r_t].cpu().numpy().astype(np.float64)
+    rel = np.abs(rn_s[same] - rho[same]) / np.maximum(rho[same], 1e-30)
+    assert np.all(rel <= 1e-4), f"residual norm error {rel.max()}"
     gb = np.unpackbits(qb[r_t].cpu().numpy()[same], axis=1, bitorder="little")
     ob = np.unpackbits(enc.bits[same], axis=1, bitorder="little")
-    near = np.abs(enc.v[same]) < 1e-5 * enc.rnorm[same, None].astype(np.float64)
-    assert not np.any((gb != ob) & ~near)
-    assert torch.all(torch.isfinite(rn))
+    diff = gb != ob
+    near = np.abs(enc.v[same]) < 1e-5 * rho[same, None]
+    assert not np.any(diff & ~near), f"{int(np.sum(diff & ~near))} sign bits differ outside the band"
+    assert diff.sum() < 1e-4 * diff.size + 1, f"{int(diff.sum())} exempt sign bits"
 
 
 def test_qjl_estimator_reduces_inner_product_bias():
