@@ -30,11 +30,10 @@
 //    and leave in one bulk store per batch; norms are plain coalesced stores.
 #pragma once
 
-#include <cstdlib>
-
 #include "quant_kernels.cuh"
 #include "tensor_map.h"
 #include "mma_encode.cuh"
+#include "mma_decode.cuh"
 
 namespace rrq {
 
@@ -296,7 +295,7 @@ template <typename T, int D, int B>
 cudaError_t launch_encode_batch(const T* x, int64_t n, const QuantParams& p, uint8_t* codes,
                                 float* norms, cudaStream_t stream) {
   if constexpr (D == 128 && B == 4) {
-    if (p.norm_mode == 0 && getenv("RRQ_ENC_LANE") == nullptr) {
+    if (p.norm_mode == 0) {
       const cudaError_t e = launch_encode_mma<T>(x, n, p, codes, norms, stream);
       if (e != cudaErrorNotSupported) return e;
     }
@@ -492,6 +491,10 @@ decode_batch_kernel(const uint8_t* __restrict__ codes, const float* __restrict__
 template <typename T, int D>
 cudaError_t launch_decode_batch(const uint8_t* codes, const float* norms, int64_t n,
                                 const QuantParams& p, T* out, cudaStream_t stream) {
+  if constexpr (D == 128 && std::is_same<T, __half>::value) {
+    const cudaError_t e = launch_decode_mma<T>(codes, norms, n, p, out, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   constexpr int W = dec_batch_warps<T>();
   using SM = DecBatch<T, D, W>;
   CUtensorMap omap;

@@ -23,20 +23,29 @@
 // block, i.e. the 4-byte code words 4a + c of its rows.
 //
 // Per batch that is 64 MMAs, 16 ldmatrix loads of the inputs and 16 of the
-// tables, 128 packed butterfly operations and the code search, against 64 sign
-// XORs, 192 conversion-and-first-stage operations and 384 packed butterfly
-// operations of the one-lane-per-vector kernel (batch_kernels.cuh), whose
-// staging, code search and output this kernel keeps:
+// tables and 128 packed butterfly operations, where the one-lane-per-vector
+// kernel (batch_kernels.cuh) spends 64 sign XORs, 192 conversion-and-first-
+// stage operations and 384 packed butterfly operations on the transform:
 //  * inputs arrive as TMA tensor boxes (32 rows × 128 bytes, 128-byte swizzle,
-//    two stages per warp, zero fill past the end);
+//    zero fill past the end), one stage per warp: the stage is refilled as soon
+//    as the warp's fragments are in registers, and 12 warps per SM cover the
+//    copy latency;
 //  * ν² = ‖y'‖²/d from the thread's 32 values per row and two quad shuffles;
-//    each thread of a quad computes ν and A/ν of one of its 4 rows and shares
-//    A/ν by shuffles;
-//  * the cell table decides each code (code = lo + (s > thr), s = sat(u·A + 1/2));
+//    each thread of a quad computes ν and 2^18/ν of one of its 4 rows and shares
+//    the scale by shuffles;
+//  * the code search is the fixed-point table search below (FixedSearch);
 //  * codes go to a per-warp 32 × 64-byte tile in the 64-byte swizzle (the
 //    quad-strided word stores are conflict-free in it) and leave in one TMA
 //    tensor store per batch, which clips rows past the end.
+// The shared layout is fixed (the dynamic base must be shared address 0x400;
+// the launch checks the device's reserved shared memory and the kernel checks
+// the address): the search table sits at 0x10000, the warps' buffers below
+// and above it.
 #pragma once
+
+#include <cmath>
+#include <cstdlib>
+#include <type_traits>
 
 #include "tensor_map.h"
 
@@ -78,54 +87,122 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
-template <typename T, int WARPS_ = 8, int NS_ = 2> struct EncMma {
-  static constexpr int D = 128, NB = D / 32;   // four 32-coordinate blocks
-  static constexpr int ROW = D * 2;            // input row bytes
-  static constexpr int BOXES = ROW / 128;      // 128-byte boxes per row
-  static constexpr int NS = NS_;               // input stages per warp
-  static constexpr int CB = D / 2;             // code bytes per vector (4-bit codes)
-  static constexpr int STAGE = 32 * ROW;       // 1024-aligned
-  static constexpr int CTILE = 32 * CB;        // one batch of codes, 64-byte swizzle
-  static constexpr int WARP_BYTES = (NS * STAGE + 2 * CTILE + 1023) / 1024 * 1024;
-  static constexpr int TABLE = (kMaxCells + 1) * 32 * 8;  // lane-replicated (thr, lo) pairs
-  static constexpr int HROW = 80;              // bytes per row of a block table (64 + 16 padding)
-  static constexpr int HTAB = NB * 32 * HROW;  // B_a^T, rows n, 32 columns k each
-  static constexpr int SIGNS = D;              // one byte per coordinate (set-up only)
-  static constexpr int WARPS = WARPS_;
-  static constexpr int THREADS = WARPS * 32;
-  static constexpr int BARS = WARPS * NS * 8;
-  static constexpr int HEAD = (TABLE + HTAB + SIGNS + BARS + 1023) / 1024 * 1024;
-  // + 1024: the dynamic shared memory base is rounded up to a 1024-byte boundary
-  static constexpr size_t total() { return 1024 + size_t(HEAD) + size_t(WARPS) * WARP_BYTES; }
-  static_assert(total() <= 227 * 1024, "shared memory");
+// Fixed-point code search.  The kernel forms I = round(u·2^18) for the
+// normalised coordinate u = y'/ν as the integer bits of one fp32 FMA,
+//     f = y'·(2^18/ν) + 1.5·2^23,   bits(f) = 0x4B400000 + I   (|I| < 2^22),
+// so the cell j = ⌊I / 2^16⌋ (a quarter of a unit of u wide) is byte 2 of
+// bits(f) minus 0x40, and the decision u > τ_k is the integer comparison
+// I > T_k with T_k = ⌊τ_k·2^18⌋ (exact, from the levels in double on the host).
+// I resolves u to 2^-18 ≈ 3.8·10^-6, inside the 10^-5 band of the decision
+// rule.  |u| ≤ √d = 11.3 keeps j within ±46, so a 128-row table holds every
+// reachable cell.  Byte 2 of bits(f) and the lane's column are merged by one
+// byte permute into the address of the lane-replicated entry (thr_j, lo_j) at
+// shared address 0x10000 + byte·256 + lane·8:
+//     code = lo_j + (I > thr_j),   thr_j = the one T_k in cell j (or none),
+// the comparison being the carry of I − (thr_j + 1) added to lo_j,
+// with no saturation and no separate s.  A codebook with two thresholds within
+// one cell of the reachable range (closer than 1/4) takes another encoder.
+struct FixedSearch {
+  int ok;          // 0: the table cannot serve this codebook (another encoder runs)
+  float num;       // 2^18 (scaled by 1/ν per vector)
+  float bias;      // 1.5·2^23
+  uint2 rows[128]; // row r = cell r − 64: (biased threshold inside it + 1, or 2^32 − 1; lo)
 };
 
-template <typename T, int WARPS_ = 8, int NS_ = 2>
-__global__ void __launch_bounds__(EncMma<T, WARPS_, NS_>::THREADS, 1)
+// Host: the fixed-point parameters for a codebook (levels ascending, L = 2^bits)
+// at d = 128, or ok = 0 when two thresholds share a reachable cell.
+inline FixedSearch make_fixed_search(const QuantParams& p) {
+  FixedSearch fs{};
+  const int L = 1 << p.bits, nthr = L - 1;
+  const double G = 262144.0;
+  int32_t T[kMaxLevels];
+  for (int k = 0; k < nthr; ++k) {
+    const double tau = (double(p.levels[k]) + double(p.levels[k + 1])) * 0.5;
+    // |I| < 2^22 always, so clamping far thresholds at ±2^23 keeps every decision
+    const double t = std::floor(tau * G);
+    T[k] = int32_t(t < -8388608.0 ? -8388608.0 : (t > 8388608.0 ? 8388608.0 : t));
+  }
+  for (int k = 1; k < nthr; ++k) {
+    const bool reachable = T[k] >= -(64 << 16) && T[k - 1] < (64 << 16);
+    if (reachable && (T[k] >> 16) == (T[k - 1] >> 16)) return fs;
+  }
+  fs.ok = 1;
+  fs.num = float(G);
+  fs.bias = float(1.5 * 8388608.0);
+  for (int r = 0; r < 128; ++r) {
+    const int64_t edge = int64_t(r - 64) * 65536;  // I at the cell's lower end
+    uint32_t lo = 0, thr = 0xFFFFFFFFu;
+    for (int k = 0; k < nthr; ++k) {
+      if (T[k] < edge) ++lo;
+      else if (T[k] < edge + 65536) thr = uint32_t(int32_t(0x4B400000) + T[k]) + 1u;
+    }
+    fs.rows[r] = make_uint2(thr, lo);
+  }
+  return fs;
+}
+
+// Code of one coordinate from its biased fixed-point value f and the address of
+// its cell's entry (thr + 1, lo): lo plus the carry of f − (thr + 1), i.e.
+// lo + (f > thr), in one subtract-with-carry and one add-carry.
+__device__ __forceinline__ uint32_t code_at(uint32_t f, uint32_t addr) {
+  uint32_t thr1, lo, c;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(thr1), "=r"(lo) : "r"(addr));
+  asm("{\n\t.reg .u32 t;\n\tsub.cc.u32 t, %1, %2;\n\taddc.u32 %0, %3, 0;\n\t}"
+      : "=r"(c)
+      : "r"(f), "r"(thr1), "r"(lo));
+  return c;
+}
+
+template <int WARPS_, int NS_, int CT_> struct EncMma {
+  static constexpr int D = 128, NB = 4, ROW = 256, BOXES = 2, CB = 64;
+  static constexpr int NS = NS_, CT = CT_, WARPS = WARPS_, THREADS = WARPS * 32;
+  static constexpr int STAGE = 32 * ROW, CTILE = 32 * CB;
+  static constexpr int WB = (NS * STAGE + CT * CTILE + 1023) / 1024 * 1024;
+  static constexpr uint32_t kBase = 0x400;      // dynamic shared memory base (checked)
+  static constexpr uint32_t kTable = 0x10000;   // lane-replicated entries, rows 0..127
+  static constexpr uint32_t kTableEnd = kTable + 128 * 256;
+  static constexpr int HROW = 80, HTAB = NB * 32 * HROW;
+  static constexpr uint32_t HT = 0, SIGNS = HTAB, BARS = SIGNS + D;  // offsets from kBase
+  static constexpr uint32_t FRONT = kBase + (BARS + WARPS * NS * 8 + 1023) / 1024 * 1024;
+  static constexpr int NFRONT = (kTable - FRONT) / WB < WARPS ? int((kTable - FRONT) / WB) : WARPS;
+  static constexpr uint32_t warp_base(int w) {  // shared address of warp w's buffers
+    return w < NFRONT ? FRONT + uint32_t(w) * WB : kTableEnd + uint32_t(w - NFRONT) * WB;
+  }
+  static constexpr size_t total() { return size_t(warp_base(WARPS)) - kBase; }
+  static_assert(total() <= 227 * 1024, "shared memory");
+  static_assert(FRONT % 1024 == 0 && kTableEnd % 1024 == 0, "1024-aligned stages");
+};
+
+template <typename T, int WARPS_, int NS_, int CT_, bool SPLIT>
+__global__ void __launch_bounds__(WARPS_ * 32, 1)
 encode_mma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
-                  int64_t n, float* __restrict__ norms, const QuantParams p) {
-  using SM = EncMma<T, WARPS_, NS_>;
+                   int64_t n, float* __restrict__ norms, const QuantParams p,
+                   const __grid_constant__ FixedSearch fs) {
+  using SM = EncMma<WARPS_, NS_, CT_>;
   constexpr int NB = SM::NB, NS = SM::NS;
   pdl_release();
-  extern __shared__ __align__(1024) uint8_t dsm_raw[];
-  uint8_t* dsm = dsm_raw + ((1024u - (smem_addr(dsm_raw) & 1023u)) & 1023u);
-  float2* tab = reinterpret_cast<float2*>(dsm);
-  uint8_t* htab = dsm + SM::TABLE;
-  uint8_t* signs = htab + SM::HTAB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(signs + SM::SIGNS);
+  extern __shared__ __align__(1024) uint8_t dsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* wmem = dsm + SM::HEAD + warp * SM::WARP_BYTES;
+  if (smem_addr(dsm) != SM::kBase) {
+    // not the layout the launch assumed: mark every norm of this CTA's batches NaN
+    pdl_wait();
+    for (int64_t b = int64_t(warp) * gridDim.x + blockIdx.x; b < (n + 31) >> 5;
+         b += int64_t(gridDim.x) * SM::WARPS)
+      if ((b << 5) + lane < n) norms[(b << 5) + lane] = __uint_as_float(0x7fc00000u);
+    return;
+  }
+  uint8_t* htab = dsm + SM::HT;
+  uint8_t* signs = dsm + SM::SIGNS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dsm + SM::BARS);
+  uint2* tab = reinterpret_cast<uint2*>(dsm + (SM::kTable - SM::kBase));
 
-  const int N = p.cell.cells;
-  for (int i = threadIdx.x; i < (N + 1) * 32; i += blockDim.x)
-    tab[i] = make_float2(p.cell.thr[i >> 5], __uint_as_float(p.cell.lo[i >> 5]));
   for (int i = threadIdx.x; i < SM::D; i += blockDim.x) signs[i] = uint8_t(sign_bit(p.seed, i));
+  for (int i = threadIdx.x; i < 128 * 32; i += blockDim.x) tab[i] = fs.rows[i >> 5];
   if (lane == 0) {
-    for (int s = 0; s < NS; ++s) mbarrier_init(smem_addr(&bars[warp * NS + s]), 1);
+    for (int st = 0; st < NS; ++st) mbarrier_init(smem_addr(&bars[warp * NS + st]), 1);
     fence_mbarrier_init();
   }
   __syncthreads();
-  // B_a^T[n][k] = s_{32a+k}·H_32[π(n), k], π swapping bit fields 1–2 and 3–4 of n
   for (int i = threadIdx.x; i < NB * 32 * 32; i += blockDim.x) {
     const int k = i & 31, nn = (i >> 5) & 31, a = i >> 10;
     const int pn = (nn & 1) | (((nn >> 3) & 3) << 1) | (((nn >> 1) & 3) << 3);
@@ -134,158 +211,164 @@ encode_mma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constan
         neg ? MmaType<T>::kMinusOne : MmaType<T>::kOne;
   }
   __syncthreads();
-  pdl_wait();  // the shared tables are built: from here on, global memory
+  pdl_wait();
 
   const int64_t nb = (n + 31) >> 5;
   const int64_t tw = int64_t(gridDim.x) * SM::WARPS;
-  // warp-major numbering: every SM gets the same number of batches (±1)
   const int64_t gw = int64_t(warp) * gridDim.x + blockIdx.x;
+  const uint32_t wbase = SM::warp_base(warp);
   const uint32_t bar0 = smem_addr(&bars[warp * NS]);
-  const uint32_t stage0 = smem_addr(wmem);
-  const uint32_t tab_lane = smem_addr(tab) + lane * 8;
-  const uint32_t ctile0 = smem_addr(wmem + NS * SM::STAGE);
+  const uint32_t stage0 = wbase;
+  const uint32_t ctile0 = wbase + NS * SM::STAGE;
   const int qr = lane >> 2, qc = lane & 3;
-  // ldmatrix row addresses: A rows 16mt + (l mod 8) + 8·bit3(l), 16-byte column
-  // chunk bit4(l); table rows 8nt + (l mod 8), 16-byte column chunk l / 8
   const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8, a_chunk = lane >> 4;
   const uint32_t h_lane = smem_addr(htab) + uint32_t((lane & 7) * SM::HROW + (lane >> 3) * 16);
-  uint32_t pending = 0;  // bit s: a load into stage s is in flight
+  const uint32_t lane_word = SM::kTable | uint32_t(lane) * 8u;  // bytes 0 and 2 of the address
+  uint32_t pending = 0;
 
-  auto issue = [&](int s, int64_t b) {
+  auto issue = [&](int st, int64_t b) {
     if (b >= nb) return;
     if (lane == 0) {
-      const uint32_t bar = bar0 + 8 * s;
+      const uint32_t bar = bar0 + 8 * st;
       mbarrier_expect_tx(bar, SM::STAGE);
 #pragma unroll
       for (int h = 0; h < SM::BOXES; ++h)
-        tma_load_2d(stage0 + s * SM::STAGE + h * 4096, &xmap, h * 64, int(b << 5), bar);
+        tma_load_2d(stage0 + st * SM::STAGE + h * 4096, &xmap, h * 64, int(b << 5), bar);
     }
-    pending |= 1u << s;
+    pending |= 1u << st;
   };
 #pragma unroll
-  for (int s = 0; s < NS; ++s) issue(s, gw + s * tw);
+  for (int st = 0; st < NS; ++st) issue(st, gw + st * tw);
 
-  const float Nf = float(N);
-  const float A = p.cell.a;
+  const float num = fs.num, bias = fs.bias;
+  // codes of a coordinate pair: byte = code(v.x) | code(v.y) << 4
+  auto pair_code = [&](float2 v, float sc) -> uint32_t {
+    const float2 f = fma2(v, make_float2(sc, sc), make_float2(bias, bias));
+    const uint32_t fx = __float_as_uint(f.x), fy = __float_as_uint(f.y);
+    return code_at(fx, __byte_perm(fx, lane_word, 0x7624u)) +
+           (code_at(fy, __byte_perm(fy, lane_word, 0x7624u)) << 4);
+  };
+
   uint32_t parity = 0;
-  int s = 0, ct = 0;
+  int st = 0, ct = 0;
   bool failed = false;
   int64_t b = gw;
   for (; b < nb; b += tw) {
-    if (!mbarrier_wait(bar0 + 8 * s, (parity >> s) & 1u)) {
+    if (!mbarrier_wait(bar0 + 8 * st, (parity >> st) & 1u)) {
       failed = true;
       break;
     }
-    parity ^= 1u << s;
-    pending &= ~(1u << s);
+    parity ^= 1u << st;
+    pending &= ~(1u << st);
     const int64_t v0 = b << 5;
+    const uint32_t sbase = stage0 + st * SM::STAGE;
+    if (lane == 0 && CT_ == 2) bulk_wait_read_1();
+    if (lane == 0 && CT_ == 1) bulk_wait_read_all();
+    const uint32_t tile = ctile0 + (CT_ == 2 ? ct : 0) * SM::CTILE;
+    const uint32_t swz = uint32_t((qr >> 1) & 3);
+    float my_nu = 0.f;
 
-    // z[a] = X_a · B_a on m16n8k16 tiles: acc[a][mt][nt] covers rows
-    // 16mt + {qr, qr + 8}, columns 8nt + 2qc + {0, 1} of block a
-    float acc[NB][2][4][4];
-    const uint32_t st = stage0 + s * SM::STAGE;
+    // one m-tile of 16 rows (mt), or both at once
+    auto run = [&](auto mts) {
+      constexpr int M0 = decltype(mts)::value >= 2 ? 0 : decltype(mts)::value;
+      constexpr int MN = decltype(mts)::value >= 2 ? 2 : 1;
+      float acc[NB][MN][4][4];
 #pragma unroll
-    for (int a = 0; a < NB; ++a) {
-      uint32_t bf[4][4];
+      for (int a = 0; a < NB; ++a) {
+        uint32_t bf[4][4];
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) ldsm_x4(bf[nt], h_lane + uint32_t((a * 32 + 8 * nt) * SM::HROW));
+        for (int nt = 0; nt < 4; ++nt) ldsm_x4(bf[nt], h_lane + uint32_t((a * 32 + 8 * nt) * SM::HROW));
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
+        for (int m = 0; m < MN; ++m) {
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) acc[a][mt][nt][0] = acc[a][mt][nt][1] = acc[a][mt][nt][2] = acc[a][mt][nt][3] = 0.f;
+          for (int nt = 0; nt < 4; ++nt) acc[a][m][nt][0] = acc[a][m][nt][1] = acc[a][m][nt][2] = acc[a][m][nt][3] = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const int colb = 64 * a + 32 * ks + 16 * a_chunk;  // byte within the 256-byte row
-          uint32_t af[4];
-          ldsm_x4(af, st + (colb >> 7) * 4096 + swz128(16 * mt + a_row, (colb & 127) >> 4));
+          for (int ks = 0; ks < 2; ++ks) {
+            const int colb = 64 * a + 32 * ks + 16 * a_chunk;
+            uint32_t af[4];
+            ldsm_x4(af, sbase + (colb >> 7) * 4096 + swz128(16 * (M0 + m) + a_row, (colb & 127) >> 4));
 #pragma unroll
-          for (int nt = 0; nt < 4; ++nt) mma_t<T>(acc[a][mt][nt], af, bf[nt][2 * ks], bf[nt][2 * ks + 1]);
+            for (int nt = 0; nt < 4; ++nt) mma_t<T>(acc[a][m][nt], af, bf[nt][2 * ks], bf[nt][2 * ks + 1]);
+          }
         }
       }
-    }
-    __syncwarp();  // every lane's fragments are in registers: the stage may be refilled
-    fence_proxy_async_smem();
-    issue(s, b + NS * tw);
-
-    // y'[32a + b] = Σ_a' H_4[a, a']·z[a', b] on packed pairs, and ν² per row:
-    // row index r = h + 2mt is row qr + 8r of the batch
-    float2 y[NB][2][4][2];
-    float2 q2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                    make_float2(0.f, 0.f)};
+      if (M0 + MN == 2) {  // every fragment of the stage is in registers: refill it
+        __syncwarp();
+        fence_proxy_async_smem();
+        issue(st, b + NS * tw);
+      }
+      // H_4 over the blocks, ν² per row (r = h + 2m)
+      float2 q2[2 * MN];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+      for (int r = 0; r < 2 * MN; ++r) q2[r] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+      for (int m = 0; m < MN; ++m)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float2 z[NB];
+#pragma unroll
+            for (int a = 0; a < NB; ++a) z[a] = make_float2(acc[a][m][nt][2 * h], acc[a][m][nt][2 * h + 1]);
+#pragma unroll
+            for (int mm = 1; mm < NB; mm <<= 1)
+#pragma unroll
+              for (int a = 0; a < NB; ++a)
+                if ((a & mm) == 0) {
+                  const float2 u = z[a], w = z[a | mm];
+                  z[a] = add2(u, w);
+                  z[a | mm] = sub2(u, w);
+                }
+#pragma unroll
+            for (int a = 0; a < NB; ++a) {
+              acc[a][m][nt][2 * h] = z[a].x;
+              acc[a][m][nt][2 * h + 1] = z[a].y;
+              q2[h + 2 * m] = fma2(z[a], z[a], q2[h + 2 * m]);
+            }
+          }
+      float ss[2 * MN];
+#pragma unroll
+      for (int r = 0; r < 2 * MN; ++r) {
+        ss[r] = q2[r].x + q2[r].y;
+        ss[r] += __shfl_xor_sync(kFull, ss[r], 1);
+        ss[r] += __shfl_xor_sync(kFull, ss[r], 2);
+      }
+      // thread qc: ν of local row qc mod 2·MN; rows are qr + 8(h + 2(M0 + m))
+      float mine = ss[0];
+#pragma unroll
+      for (int r = 1; r < 2 * MN; ++r) mine = (qc % (2 * MN)) == r ? ss[r] : mine;
+      const float nu = sqrtf(mine * p.inv_d);
+      const float msc = nu > 0.f ? __fdiv_rn(num, nu) : 0.f;
+      if (MN == 2 || (qc >> 1) == M0) my_nu = nu;
+      float sc[2 * MN];
+#pragma unroll
+      for (int r = 0; r < 2 * MN; ++r) sc[r] = __shfl_sync(kFull, msc, (lane & ~3) | r);
+#pragma unroll
+      for (int m = 0; m < MN; ++m)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          float2 z[NB];
-#pragma unroll
-          for (int a = 0; a < NB; ++a) z[a] = make_float2(acc[a][mt][nt][2 * h], acc[a][mt][nt][2 * h + 1]);
-#pragma unroll
-          for (int m = 1; m < NB; m <<= 1)
-#pragma unroll
-            for (int a = 0; a < NB; ++a)
-              if ((a & m) == 0) {
-                const float2 u = z[a], v = z[a | m];
-                z[a] = add2(u, v);
-                z[a | m] = sub2(u, v);
-              }
+          const int row = qr + 8 * (h + 2 * (M0 + m));
 #pragma unroll
           for (int a = 0; a < NB; ++a) {
-            y[a][mt][nt][h] = z[a];
-            q2[h + 2 * mt] = fma2(z[a], z[a], q2[h + 2 * mt]);
+            uint32_t word = 0;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+              word += pair_code(make_float2(acc[a][m][nt][2 * h], acc[a][m][nt][2 * h + 1]), sc[h + 2 * m])
+                      << (8 * nt);
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(tile + uint32_t(row * 64) + ((uint32_t(a) ^ swz) << 4) +
+                                                             uint32_t(qc * 4)),
+                         "r"(word)
+                         : "memory");
           }
         }
-    float ss[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      ss[r] = q2[r].x + q2[r].y;
-      ss[r] += __shfl_xor_sync(kFull, ss[r], 1);
-      ss[r] += __shfl_xor_sync(kFull, ss[r], 2);
+    };
+    if constexpr (SPLIT) {
+      run(std::integral_constant<int, 0>());
+      run(std::integral_constant<int, 1>());
+    } else {
+      run(std::integral_constant<int, 2>());
     }
-    // thread qc of the quad: ν and A/ν of row qr + 8qc (‖y'‖² = d·‖x‖²)
-    const float my_ss = qc == 0 ? ss[0] : qc == 1 ? ss[1] : qc == 2 ? ss[2] : ss[3];
-    const float nu = sqrtf(my_ss * p.inv_d);
-    const float my_sc = nu > 0.f ? __fdiv_rn(A, nu) : 0.f;  // s = sat(y'·A/ν + 1/2)
-    float sc[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) sc[r] = __shfl_sync(kFull, my_sc, (lane & ~3) | r);
-
-    // codes: row qr + 8r, word 4a + qc holds coordinates 32a + 8qc + [0, 8)
-    if (lane == 0) bulk_wait_read_1();  // the store from this tile two batches ago has read it
-    __syncwarp();
-    const uint32_t tile = ctile0 + ct * SM::CTILE;
-    const uint32_t swz = uint32_t((qr >> 1) & 3);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = h + 2 * mt;
-        const float scr = sc[r];
-#pragma unroll
-        for (int a = 0; a < NB; ++a) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt) {
-            const float2 v = y[a][mt][nt][h];
-            const float sx = __saturatef(fmaf(v.x, scr, 0.5f));
-            const float sy = __saturatef(fmaf(v.y, scr, 0.5f));
-            const float2 f = fma2(make_float2(sx, sy), make_float2(Nf, Nf), make_float2(8388608.f, 8388608.f));
-            // the float bits are 0x4B000000 + round(s·N); ·256 drops the exponent
-            const float2 ex = lds_f2(tab_lane + (__float_as_uint(f.x) << 8));
-            const float2 ey = lds_f2(tab_lane + (__float_as_uint(f.y) << 8));
-            const uint32_t cx = __float_as_uint(ex.y) + (sx > ex.x ? 1u : 0u);
-            const uint32_t cy = __float_as_uint(ey.y) + (sy > ey.x ? 1u : 0u);
-            word |= (cx + (cy << 4)) << (8 * nt);
-          }
-          const int row = qr + 8 * r;
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(tile + uint32_t(row * 64) + ((uint32_t(a) ^ swz) << 4) +
-                                                           uint32_t(qc * 4)),
-                       "r"(word)
-                       : "memory");
-        }
-      }
-    if (v0 + qr + 8 * qc < n) norms[v0 + qr + 8 * qc] = nu;
+    if (v0 + qr + 8 * qc < n) norms[v0 + qr + 8 * qc] = my_nu;
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -293,41 +376,50 @@ encode_mma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constan
       bulk_commit();
     }
     ct ^= 1;
-    s = (s + 1 == NS) ? 0 : s + 1;
+    st = (st + 1 == NS) ? 0 : st + 1;
   }
 
   if (failed) {
-    // A stage never completed: mark every vector this warp still owns with a
-    // NaN norm, and wait (bounded) for the copies still in flight.
     for (; b < nb; b += tw) {
       const int64_t v0 = b << 5;
       if (lane < n - v0) norms[v0 + lane] = __uint_as_float(0x7fc00000u);
     }
 #pragma unroll
-    for (int st = 0; st < NS; ++st)
-      if (pending & (1u << st)) mbarrier_wait(bar0 + 8 * st, (parity >> st) & 1u);
+    for (int s2 = 0; s2 < NS; ++s2)
+      if (pending & (1u << s2)) mbarrier_wait(bar0 + 8 * s2, (parity >> s2) & 1u);
   }
   if (lane == 0) bulk_wait_all();
 }
 
-// cudaErrorNotSupported when no tensor map can be made (the caller then uses
-// another encoder).
-template <typename T>
-cudaError_t launch_encode_mma(const T* x, int64_t n, const QuantParams& p, uint8_t* codes,
-                              float* norms, cudaStream_t stream) {
-  using SM = EncMma<T>;
-  CUtensorMap xmap, cmap;
-  if (!row_tensor_map(&xmap, x, n, SM::D, 2, 32)) return cudaErrorNotSupported;
-  if (!code_tensor_map(&cmap, codes, n, SM::CB, 32)) return cudaErrorNotSupported;
-  auto k = encode_mma_kernel<T>;
+template <typename T, int W, int NS, int CT, bool SPLIT>
+cudaError_t launch_encode_mma_v(const CUtensorMap& xmap, const CUtensorMap& cmap, int64_t n,
+                                 const QuantParams& p, const FixedSearch& fs, float* norms,
+                                 cudaStream_t stream) {
+  using SM = EncMma<W, NS, CT>;
+  auto k = encode_mma_kernel<T, W, NS, CT, SPLIT>;
   constexpr size_t smem = SM::total();
   const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int64_t batches = (n + 31) / 32;
-  const int grid = grid_for(reinterpret_cast<const void*>(k), SM::THREADS, smem,
-                            (batches + SM::WARPS - 1) / SM::WARPS);
-  return launch_pdl(k, grid, SM::THREADS, smem, stream, xmap, cmap, n, norms, p);
+  const int grid = grid_for(reinterpret_cast<const void*>(k), SM::THREADS, smem, (batches + W - 1) / W);
+  return launch_pdl(k, grid, SM::THREADS, smem, stream, xmap, cmap, n, norms, p, fs);
+}
+
+template <typename T>
+cudaError_t launch_encode_mma(const T* x, int64_t n, const QuantParams& p, uint8_t* codes,
+                               float* norms, cudaStream_t stream) {
+  const FixedSearch fs = make_fixed_search(p);
+  if (!fs.ok) return cudaErrorNotSupported;
+  int dev = 0, reserved = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      uint32_t(reserved) != EncMma<12, 1, 2>::kBase)
+    return cudaErrorNotSupported;
+  CUtensorMap xmap, cmap;
+  if (!row_tensor_map(&xmap, x, n, 128, 2, 32)) return cudaErrorNotSupported;
+  if (!code_tensor_map(&cmap, codes, n, 64, 32)) return cudaErrorNotSupported;
+  return launch_encode_mma_v<T, 12, 1, 2, false>(xmap, cmap, n, p, fs, norms, stream);
 }
 
 }  // namespace rrq
