@@ -437,7 +437,13 @@ struct MmaScoreSmem {
   static constexpr int KK = CB / 8;         // k-steps of 16 coordinates
   static constexpr int CW = CB / 16;        // words of a thread's row slice
   static constexpr int NS = 3;              // ring stages
-  static constexpr int STAGE = 32 * CB + 32 * 4;
+  // ring rows padded so the quads' slice loads (tokens 4r + j, r = 0..7) are
+  // conflict-free: 80 bytes at d = 128 (16-byte copies), 40 at d = 64 (8-byte)
+  // ring rows padded so the quads' slice loads (tokens 4r + j, r = 0..7) are
+  // conflict-free: 80 bytes at d = 128 (16-byte copies), 40 at d = 64 (8-byte)
+  static constexpr int RS = D == 128 ? CB + 16 : CB + 8;
+  static constexpr int CP = D == 128 ? 16 : 8;  // cp.async chunk bytes
+  static constexpr int STAGE = 32 * RS + 32 * 4;
   static constexpr int RING = NS * STAGE;   // per warp
   __host__ __device__ static constexpr size_t table() { return 256 * 64 * 4; }  // entry e at byte e·256 + lane·4
   __host__ __device__ static size_t bq(int hkv) { return size_t(hkv) * 32 * CB; }  // B fragments
@@ -550,49 +556,63 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
   }
   __syncthreads();  // qf is dead: its space becomes the rings
 
+  // units u = tile·hkv + g (token-major); warp w takes u = w, w + nw, w + 2nw, …
+  // so the warps working at one moment read whole token rows of the cache
+  // together.  The launch makes nw a multiple of hkv, so all units of a warp
+  // have the same kv head g (its B fragments stay in registers) and consecutive
+  // units are TS = nw/hkv tiles apart: every address advances by a constant.
   const int lg_hkv = __ffs(a.hkv) - 1;  // hkv is a power of two
   const int64_t nbt = (a.T + 31) >> 5;
-  const int64_t units = nbt << lg_hkv;
   const int64_t nw = int64_t(gridDim.x) * W, gw = int64_t(blockIdx.x) * W + warp;
-  const int64_t u_begin = units * gw / nw, u_end = units * (gw + 1) / nw;
-  const char* tab_bytes = reinterpret_cast<const char*>(ptab);
+  const int g = int(gw & (a.hkv - 1));
+  const int64_t tile0 = gw >> lg_hkv, TS = nw >> lg_hkv;
+  const int64_t my_units = tile0 < nbt ? (nbt - tile0 + TS - 1) / TS : 0;
   // FOLD: byte 2 of the permute's second operand is the table's address bit 16
+  const char* tab_bytes = reinterpret_cast<const char*>(ptab);
   const uint32_t lane4 = uint32_t(lane) * 4u | (FOLD ? Sm::kFoldTable : 0u);
-  const float post = a.scale * p.inv_d;
-  const int qc = lane & 3, qr = lane >> 2;  // quad position, row in an 8-row group
+  const int qc = lane & 3, qr = lane >> 2;  // quad position, token group 4qr .. 4qr + 3
 
-  // Copy k of a unit moves chunk c = lane % CPR of row t = lane / CPR + k·(32 / CPR):
-  // per-lane offsets are fixed, the unit adds one base.
-  constexpr int CPR = CB / 16;  // 16-byte chunks per row
+  // Copy k of a unit moves chunk c = lane % CPR of row t = lane / CPR + k·(32 / CPR)
+  constexpr int CPR = CB / Sm::CP;  // copies per row
   const int lt = lane / CPR, lc = lane % CPR;
   const int64_t row_bytes = int64_t(a.hkv) * CB;  // global stride between tokens
-  const int64_t lane_src = lt * row_bytes + lc * 16;
-  const uint32_t lane_dst = uint32_t(lt * CB + lc * 16);
-  auto issue = [&](int stage, int64_t u) {
-    if (u < u_end) {
-      const int g = int(u & (a.hkv - 1));
-      const int64_t t0 = (u >> lg_hkv) << 5;
-      const uint8_t* src = a.codes + (t0 * a.hkv + g) * CB + lane_src;
-      const uint32_t dst = smem_addr(ring + stage * Sm::STAGE) + lane_dst;
-      if (t0 + 32 <= a.T) {
+  const int64_t unit_step = TS * 32;              // tokens between consecutive units
+  const int64_t src_step = unit_step * row_bytes;
+  const uint8_t* src_next = a.codes + (tile0 * 32 * a.hkv + g) * CB + lt * row_bytes + lc * Sm::CP;
+  const float* nrm_next = a.norms + (tile0 * 32 + lane) * a.hkv + g;
+  int64_t t_next = tile0 * 32;  // first token of the next unit to load
+  const uint32_t ring0 = smem_addr(ring);
+  const uint32_t lane_dst = uint32_t(lt * Sm::RS + lc * Sm::CP);
+  auto copy = [&](uint32_t dst, const uint8_t* src, bool ok) {
+    if constexpr (Sm::CP == 16) cp_async16(dst, ok ? src : a.codes, ok ? 16 : 0);
+    else cp_async8(dst, ok ? src : a.codes, ok ? 8 : 0);
+  };
+  int64_t issued = 0;
+  auto issue = [&](int stage) {
+    if (issued < my_units) {
+      const uint32_t sbase = ring0 + uint32_t(stage * Sm::STAGE);
+      if (t_next + 32 <= a.T) {
 #pragma unroll
         for (int k = 0; k < CPR; ++k)
-          cp_async16(dst + k * (32 / CPR) * CB, src + k * (32 / CPR) * row_bytes, 16);
-        cp_async4(dst - lane_dst + 32 * CB + lane * 4, a.norms + (t0 + lane) * a.hkv + g, 4);
+          copy(sbase + lane_dst + k * (32 / CPR) * Sm::RS, src_next + k * (32 / CPR) * row_bytes, true);
+        cp_async4(sbase + 32 * Sm::RS + lane * 4, nrm_next, 4);
       } else {
 #pragma unroll
-        for (int k = 0; k < CPR; ++k) {
-          const bool ok = t0 + lt + k * (32 / CPR) < a.T;
-          cp_async16(dst + k * (32 / CPR) * CB, ok ? src + k * (32 / CPR) * row_bytes : a.codes, ok ? 16 : 0);
-        }
-        const bool ok = t0 + lane < a.T;
-        cp_async4(dst - lane_dst + 32 * CB + lane * 4, a.norms + (ok ? (t0 + lane) * a.hkv + g : 0), ok ? 4 : 0);
+        for (int k = 0; k < CPR; ++k)
+          copy(sbase + lane_dst + k * (32 / CPR) * Sm::RS, src_next + k * (32 / CPR) * row_bytes,
+               t_next + lt + k * (32 / CPR) < a.T);
+        const bool ok = t_next + lane < a.T;
+        cp_async4(sbase + 32 * Sm::RS + lane * 4, ok ? nrm_next : a.norms, ok ? 4 : 0);
       }
+      ++issued;
+      src_next += src_step;
+      nrm_next += unit_step * a.hkv;
+      t_next += unit_step;
     }
     cp_async_commit();
   };
 #pragma unroll
-  for (int k = 0; k < NS - 1; ++k) issue(k, u_begin + k);
+  for (int k = 0; k < NS - 1; ++k) issue(k);
 
   auto level_pair = [&](uint32_t word, int pos) -> uint32_t {
     uint32_t cv;
@@ -606,55 +626,74 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
     return cv;
   };
 
+  // the lane's B fragments (k-step kk: words 2kk, 2kk + 1) and head scales
+  uint32_t bfr[KK][2];
+#pragma unroll
+  for (int j = 0; j < KK / 2; ++j) {
+    const uint4 v = bq[(g * (KK / 2) + j) * 32 + lane];
+    bfr[2 * j][0] = v.x;
+    bfr[2 * j][1] = v.y;
+    bfr[2 * j + 1][0] = v.z;
+    bfr[2 * j + 1][1] = v.w;
+  }
+  float hsc[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+    hsc[e] = 2 * qc + e < G ? a.scale * p.inv_d * inv_s[g * G + 2 * qc + e] : 0.f;
+  const bool vec_out = (a.T & 3) == 0;  // 16-byte score stores stay aligned
+  const int h0 = g * G + 2 * qc;        // the lane's first head
+  float* out_next = a.scores + int64_t(h0) * a.T + tile0 * 32 + 4 * qr;
+  int64_t t0 = tile0 * 32;
+
   int stage = 0;
-  for (int64_t u = u_begin; u < u_end; ++u) {
+  for (int64_t k = 0; k < my_units; ++k) {
     cp_async_wait<NS - 2>();
     __syncwarp();
     const uint8_t* st = ring + stage * Sm::STAGE;
-    // rows qr + 8m, m = 0..3: tile 0 holds m = 0, 1 and tile 1 m = 2, 3
+    // token 4qr + j (j = 2mt + h) is row qr + 8h of m-tile mt
     Chunk cw[4];
-    float nu[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      cw[m] = *reinterpret_cast<const Chunk*>(st + (qr + 8 * m) * CB + qc * (CB / 4));
-      nu[m] = reinterpret_cast<const float*>(st + 32 * CB)[qr + 8 * m];
-    }
+    for (int j = 0; j < 4; ++j) cw[j] = *reinterpret_cast<const Chunk*>(st + (4 * qr + j) * Sm::RS + qc * (CB / 4));
+    const float4 nu = *reinterpret_cast<const float4*>(st + 32 * Sm::RS + 16 * qr);
     __syncwarp();  // every lane has read this stage before it is refilled
-    issue(stage == 0 ? NS - 1 : stage - 1, u + NS - 1);
+    issue(stage == 0 ? NS - 1 : stage - 1);
     stage = (stage + 1 == NS) ? 0 : stage + 1;
-
-    const int g = int(u & (a.hkv - 1));
-    const int64_t t0 = (u >> lg_hkv) << 5;
-    uint4 bv[KK / 2];
-#pragma unroll
-    for (int j = 0; j < KK / 2; ++j) bv[j] = bq[(g * (KK / 2) + j) * 32 + lane];
 
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < KK; ++kk) {
       const int wi = kk >> 1, pos = 2 * (kk & 1);
-      const uint32_t b0 = word_of(bv[kk >> 1], pos), b1 = word_of(bv[kk >> 1], pos + 1);
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         const uint32_t lo = word_of(cw[2 * mt], wi), hi = word_of(cw[2 * mt + 1], wi);
         mma_16816(acc[mt], level_pair(lo, pos), level_pair(hi, pos), level_pair(lo, pos + 1),
-                  level_pair(hi, pos + 1), b0, b1);
+                  level_pair(hi, pos + 1), bfr[kk][0], bfr[kk][1]);
       }
     }
 
-    // accumulator i of tile mt: token row qr + 8·(i >> 1) + 16·mt, head 2·qc + (i & 1)
+    // accumulator i of tile mt: token 4qr + 2mt + (i >> 1), head 2qc + (i & 1)
+    const bool full = vec_out && t0 + 32 <= a.T;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int h = 2 * qc + e;
-      if (h < G) {
-        const float hs = post * inv_s[g * G + h];
-        float* out = a.scores + int64_t(g * G + h) * a.T + t0 + qr;
+      if (2 * qc + e < G) {
+        float* out = out_next + int64_t(e) * a.T;
+        const float2 hs2 = make_float2(hsc[e], hsc[e]);
+        const float2 s01 = mul2(make_float2(nu.x, nu.y), hs2), s23 = mul2(make_float2(nu.z, nu.w), hs2);
+        const float2 v01 = mul2(make_float2(acc[0][e], acc[0][2 + e]), s01);
+        const float2 v23 = mul2(make_float2(acc[1][e], acc[1][2 + e]), s23);
+        const float4 v = make_float4(v01.x, v01.y, v23.x, v23.y);
+        if (full) {
+          *reinterpret_cast<float4*>(out) = v;
+        } else {
+          const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          if (t0 + qr + 8 * m < a.T) out[8 * m] = acc[m >> 1][2 * (m & 1) + e] * (nu[m] * hs);
+          for (int j = 0; j < 4; ++j)
+            if (t0 + 4 * qr + j < a.T) out[j] = vv[j];
         }
       }
     }
+    out_next += TS * 32;
+    t0 += TS * 32;
   }
   cp_async_wait<0>();
 }
@@ -672,7 +711,13 @@ cudaError_t launch_scores_mma_w(const ScoreArgs& a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int64_t units = ((a.T + 31) / 32) * a.hkv;
-  const int grid = grid_for(reinterpret_cast<const void*>(k), W * 32, smem, (units + W - 1) / W);
+  int grid = grid_for(reinterpret_cast<const void*>(k), W * 32, smem, (units + W - 1) / W);
+  // the kernel needs the warp count grid·W to be a multiple of hkv (a power of
+  // two): round the grid to a multiple of hkv/W when hkv exceeds W
+  if (a.hkv > W) {
+    const int m = a.hkv / W;
+    grid = grid < m ? m : grid / m * m;
+  }
   return launch_pdl(k, grid, W * 32, smem, stream, a);
 }
 
