@@ -152,7 +152,7 @@ def test_attention_splits_fill_the_sms_in_one_wave(hq, hkv):
     """The token ranges per kv head that rrq_attention_workspace_bytes implies: one CTA
     per SM, rounded down so that hkv × ranges never exceeds the SM count (that of
     the visible device; 148, the library's default, when none is visible); a range
-    per 16 tiles of 32 tokens at most; at least one."""
+    per 12 tiles of 32 tokens (one per warp) at most; at least one."""
     import torch
     lib = B.lib()
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
@@ -163,5 +163,5 @@ def test_attention_splits_fill_the_sms_in_one_wave(hq, hkv):
         assert (ws - counters) % per_range == 0
         s = (ws - counters) // per_range
         ntile = (t_len + 31) // 32
-        assert s == max(1, min(sms // hkv, (ntile + 15) // 16))
+        assert s == max(1, min(sms // hkv, (ntile + 11) // 12))
         assert s * hkv <= max(sms, hkv)
