@@ -17,10 +17,14 @@
 // units of 32 consecutive tokens of that kv head, and each unit's two dot
 // products are mma.sync m16n8k16 tiles (fp16 operands, fp32 accumulation):
 // tokens are M, the group's heads N (zero columns pad G to 8), coordinates K.
-// Thread quad position c owns coordinate pairs [16c, 16c + 16) of its rows, so
-// it loads B code words and one sign word per row (the next unit's while it
-// works on this one); table lookups turn them into the A fragments: fp16
-// level pairs for the codes, (±1, ±1) pairs for a nibble of sign bits.
+// Thread quad position c owns coordinates [32c, 32c + 32) of its rows, so it
+// loads B code words and one sign word per row (the next unit's while it works
+// on this one).  Each A register of the code product is one load from a
+// lane-replicated table of fp16 level pairs (coordinates 2j, 2j + 1).  The
+// sign product pairs coordinates j and j + 16 of a sign word instead: their
+// bits are 16 apart, so one shift and one logic operation place both (negated)
+// into the sign bits of an fp16 pair of ±1, with no table.  The query operand
+// of each product uses its product's coordinate order.
 #include <cmath>
 
 #include "rrq_device.cuh"
@@ -34,13 +38,14 @@ constexpr int kSWarps = 16;
 constexpr int kSThreads = kSWarps * 32;
 
 // Level table of the b-bit codes, lane-replicated, at a shared address aligned
-// to its size so that entry | lane column | base is one OR:
-//   b = 1: a code nibble (two coordinate pairs) → two half2, 16 entries × 256 B;
-//   b = 2: a code byte (two pairs) → two half2, 256 entries × 256 B;
-//   b = 3: six bits (one pair) → one half2, 64 entries × 128 B;
-//   b = 4: a code byte (one pair) → one half2, 256 entries × 256 B
-//     (the upper half of each entry is unused: the byte permute places the
-//     byte at bits 8..15).
+// to its size so that entry | lane column | base is one OR.  An entry is 256
+// bytes: the 32 lanes' copies of its first level pair, then (b ≤ 2) of its
+// second, so each half2 is one 32-bit load:
+//   b = 1: a code nibble (two coordinate pairs), 16 entries;
+//   b = 2: a code byte (two pairs), 256 entries;
+//   b = 3: six bits (one pair), 64 entries of 128 B;
+//   b = 4: a code byte (one pair), 256 entries (the second half unused: the
+//     byte permute places the byte at bits 8..15).
 template <int B> struct LevelTable {
   static constexpr uint32_t kEntries = B == 1 ? 16 : B == 3 ? 64 : 256;
   static constexpr uint32_t kStride = B == 3 ? 128 : 256;
@@ -51,24 +56,22 @@ template <int B> struct LevelTable {
 // Shared memory, as offsets from the dynamic base at shared address `base`
 // (the host computes it for the device's reserved shared memory; the kernel
 // checks it):
-//   sgn  sign-nibble table, 16 entries × 256 B, 4 KB-aligned;
 //   bf   B fragments of q'' and v'', [2][4][32] × 16 B;
 //   qf   q' and v in fp32 (prologue), [2][G][128];
 //   sc   1/s_q, 1/s_v and max|v| bits per head;
 //   tab  the level table, aligned to its size.
 struct QjlLayout {
-  uint32_t sgn, bf, qf, sc, tab, total;
+  uint32_t bf, qf, sc, tab, total;
 };
 template <int B, int G>
 __host__ __device__ constexpr QjlLayout qjl_layout(uint32_t base) {
   const uint32_t tb = LevelTable<B>::kBytes;
-  const uint32_t sgn = (base + 4095u) / 4096u * 4096u;
-  const uint32_t bf = sgn + 4096u;
+  const uint32_t bf = (base + 15u) / 16u * 16u;
   const uint32_t qf = bf + 2u * 4u * 32u * 16u;
   const uint32_t sc = qf + 2u * G * kSD * 4u;
   const uint32_t end = (sc + 3u * G * 4u + 15u) / 16u * 16u;
   const uint32_t tab = (end + tb - 1u) / tb * tb;
-  return QjlLayout{sgn - base, bf - base, qf - base, sc - base, tab - base, tab + tb - base};
+  return QjlLayout{bf - base, qf - base, sc - base, tab - base, tab + tb - base};
 }
 
 // The slice of one key row that quad position c owns: coordinate pairs
@@ -80,10 +83,9 @@ template <int B> struct RowSlice {
 };
 
 template <int B>
-__device__ __forceinline__ void load_slice(RowSlice<B>& r, const QjlScoreArgs& a, int64_t t, int g,
+__device__ __forceinline__ void load_slice(RowSlice<B>& r, const QjlScoreArgs& a, int64_t n, bool ok,
                                            int qc) {
-  if (t < a.T) {
-    const int64_t n = t * a.hkv + g;
+  if (ok) {
     const uint32_t* cw = reinterpret_cast<const uint32_t*>(a.codes + n * (16 * B)) + B * qc;
     if constexpr (B == 4) {
       const uint4 v = __ldcs(reinterpret_cast<const uint4*>(cw));
@@ -107,17 +109,19 @@ __device__ __forceinline__ void load_slice(RowSlice<B>& r, const QjlScoreArgs& a
   }
 }
 
-// Table address of nibble kk of w: (nibble << 8) | col (kk compile-time after unrolling).
-__device__ __forceinline__ uint32_t nibble_addr(uint32_t w, int kk, uint32_t col) {
+// Nibble kk of w at bits 8..11 (kk compile-time after unrolling).
+__device__ __forceinline__ uint32_t nibble_bits(uint32_t w, int kk) {
   const uint32_t t = kk <= 2 ? (w << (8 - 4 * kk)) : (w >> (4 * kk - 8));
-  return (t & 0xF00u) | col;
+  return t & 0xF00u;
 }
 
-__device__ __forceinline__ uint2 lds2(uint32_t addr) {
-  uint2 v;
-  asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
+// fp16 pair (±1, ±1) from bits j and j + 16 of the negated sign word nw (a set
+// bit of the sign word is +1): the two bits moved to bits 15 and 31, the rest
+// of both halves the pattern of 1.0.
+__device__ __forceinline__ uint32_t sign_pair(uint32_t nw, int j) {
+  return ((nw << (15 - j)) & 0x80008000u) | 0x3C003C00u;
 }
+
 __device__ __forceinline__ uint32_t lds1(uint32_t addr) {
   uint32_t v;
   asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
@@ -134,13 +138,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Level pairs of coordinate pairs 2kk (x) and 2kk + 1 (y) of a row slice.
+// Level pairs of coordinate pairs 2kk (x) and 2kk + 1 (y) of a row slice;
+// col addresses the entry's first half, col2 = col | 128 its second.
 template <int B>
-__device__ __forceinline__ uint2 level_pairs(const uint32_t (&c)[B], int kk, uint32_t col) {
+__device__ __forceinline__ uint2 level_pairs(const uint32_t (&c)[B], int kk, uint32_t col, uint32_t col2) {
   if constexpr (B == 1) {
-    return lds2(nibble_addr(c[0], kk, col));
+    const uint32_t t = nibble_bits(c[0], kk);
+    return make_uint2(lds1(t | col), lds1(t | col2));
   } else if constexpr (B == 2) {
-    return lds2(__byte_perm(c[kk >> 2], col, 0x7604u | ((kk & 3) << 4)));
+    const uint32_t sel = 0x7604u | ((kk & 3) << 4);
+    return make_uint2(lds1(__byte_perm(c[kk >> 2], col, sel)), lds1(__byte_perm(c[kk >> 2], col2, sel)));
   } else if constexpr (B == 4) {
     const uint32_t w = c[kk >> 1], pos = 2 * (kk & 1);
     return make_uint2(lds1(__byte_perm(w, col, 0x7604u | (pos << 4))),
@@ -172,7 +179,6 @@ __global__ void __launch_bounds__(kSThreads, 1) qk_scores_qjl_kernel(const QjlSc
       for (int j = 0; j < G; ++j) a.scores[int64_t(g * G + j) * a.T + t] = __int_as_float(0x7fc00000);
     return;
   }
-  uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + lay.sgn);
   uint32_t* bf = reinterpret_cast<uint32_t*>(smem + lay.bf);
   float* qf = reinterpret_cast<float*>(smem + lay.qf);
   float* vf = qf + G * kSD;
@@ -188,8 +194,8 @@ __global__ void __launch_bounds__(kSThreads, 1) qk_scores_qjl_kernel(const QjlSc
   for (uint32_t i = tid; i < LT::kBytes / 4; i += kSThreads) {
     const uint32_t e = i / (LT::kStride / 4), wv = i % (LT::kStride / 4);
     float lo, hi;
-    if constexpr (LT::kTwoPairs) {  // word wv = 2·lane + hh: pair hh of the entry
-      const uint32_t pr = (e >> (4 * B / 2 * (wv & 1))) & ((1u << (2 * B)) - 1u);
+    if constexpr (LT::kTwoPairs) {  // word wv = 32·hh + lane: pair hh of the entry
+      const uint32_t pr = (e >> (2 * B * (wv >> 5))) & ((1u << (2 * B)) - 1u);
       lo = p.levels[pr & M];
       hi = p.levels[pr >> B];
     } else {
@@ -198,11 +204,6 @@ __global__ void __launch_bounds__(kSThreads, 1) qk_scores_qjl_kernel(const QjlSc
     }
     const __half2 v = __floats2half2_rn(lo, hi);
     tab[i] = *reinterpret_cast<const uint32_t*>(&v);
-  }
-  for (uint32_t i = tid; i < 1024; i += kSThreads) {  // sign nibble → (±1, ±1), (±1, ±1)
-    const uint32_t e = i >> 6, pr = (e >> (2 * (i & 1))) & 3u;
-    const __half2 v = __floats2half2_rn((pr & 1u) ? 1.f : -1.f, (pr & 2u) ? 1.f : -1.f);
-    sgn[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
   if (tid < G) vmax[tid] = 0u;
   pdl_wait();  // from here on, global memory
@@ -277,17 +278,20 @@ __global__ void __launch_bounds__(kSThreads, 1) qk_scores_qjl_kernel(const QjlSc
     inv_sv[tid] = mx > 0.f ? ldexpf(1.f, ex) : 1.f;
   }
   __syncthreads();
-  // B fragment word w = 2kk + hh of lane l (quad position c, column n): the
-  // pair β = 16c + 2kk + hh of head n's q'' (part 0) or v'' (part 1), zero for n ≥ G.
+  // B fragment word w = 2kk + hh of lane l (quad position c, column n), zero
+  // for n ≥ G: part 0, head n's q'' at coordinates 2β, 2β + 1 with the pair
+  // β = 16c + 2kk + hh; part 1, head n's v'' at coordinates 32c + 2kk + hh and
+  // that + 16 (the sign product's order).
   for (int i = tid; i < 2 * 4 * 32 * 4; i += kSThreads) {
     const int comp = i & 3, l = (i >> 2) & 31, j = (i >> 7) & 3, part = i >> 9;
     const int w = 4 * j + comp, kk = w >> 1, hh = w & 1, c = l & 3, n = l >> 2;
-    const int beta = 16 * c + 2 * kk + hh;
     __half2 v = __floats2half2_rn(0.f, 0.f);
     if (n < G) {
       const float* src = (part ? vf : qf) + n * kSD;
       const float s = 1.f / (part ? inv_sv[n] : inv_sq[n]);  // a power of two
-      v = __floats2half2_rn(src[2 * beta] * s, src[2 * beta + 1] * s);
+      const int i0 = part ? 32 * c + 2 * kk + hh : 2 * (16 * c + 2 * kk + hh);
+      const int i1 = part ? i0 + 16 : i0 + 1;
+      v = __floats2half2_rn(src[i0] * s, src[i1] * s);
     }
     bf[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
@@ -311,33 +315,45 @@ __global__ void __launch_bounds__(kSThreads, 1) qk_scores_qjl_kernel(const QjlSc
     km[e] = h < G ? a.scale * p.inv_d * inv_sq[h] : 0.f;
     ks[e] = h < G ? a.scale * cq * inv_sv[h] : 0.f;
   }
-  const uint32_t col_t = (base + lay.tab) | uint32_t(lane) * (LT::kTwoPairs ? 8u : 4u);
-  const uint32_t col_s = (base + lay.sgn) | uint32_t(lane) * 8u;
+  const uint32_t col_t = (base + lay.tab) | uint32_t(lane) * 4u;
+  const uint32_t col_t2 = col_t | 128u;
 
-  // ---- units of 32 tokens of kv head g; rows qr + 8m (m = 0..3) per thread
+  // ---- units of 32 tokens of kv head g, warp-major over the CTAs of g; rows
+  // qr + 8m (m = 0..3) per thread
   const int cpg = gridDim.x / a.hkv;
   const int64_t ntile = (a.T + 31) / 32;
   const int64_t stride = int64_t(cpg) * kSWarps;
   int64_t tile = int64_t(warp) * cpg + blockIdx.x / a.hkv;  // warp-major: equal tiles per CTA
   RowSlice<B> cur[4], nxt[4];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) load_slice<B>(cur[m], a, tile * 32 + qr + 8 * m, g, qc);
+  for (int m = 0; m < 4; ++m) {
+    const int64_t t = tile * 32 + qr + 8 * m;
+    load_slice<B>(cur[m], a, t * a.hkv + g, t < a.T, qc);
+  }
   for (; tile < ntile; tile += stride) {
     const int64_t t0 = tile * 32;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) load_slice<B>(nxt[m], a, t0 + stride * 32 + qr + 8 * m, g, qc);
+    for (int m = 0; m < 4; ++m) {
+      const int64_t t = t0 + stride * 32 + qr + 8 * m;
+      load_slice<B>(nxt[m], a, t * a.hkv + g, t < a.T, qc);
+    }
     float am[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     float as[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    uint32_t nsw[4];  // negated sign words of the four rows
+#pragma unroll
+    for (int m = 0; m < 4; ++m) nsw[m] = ~cur[m].s;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        const uint2 lo = level_pairs<B>(cur[2 * mt].c, kk, col_t);
-        const uint2 hi = level_pairs<B>(cur[2 * mt + 1].c, kk, col_t);
+        const uint2 lo = level_pairs<B>(cur[2 * mt].c, kk, col_t, col_t2);
+        const uint2 hi = level_pairs<B>(cur[2 * mt + 1].c, kk, col_t, col_t2);
         mma16816(am[mt], lo.x, hi.x, lo.y, hi.y, bq[2 * kk], bq[2 * kk + 1]);
-        const uint2 slo = lds2(nibble_addr(cur[2 * mt].s, kk, col_s));
-        const uint2 shi = lds2(nibble_addr(cur[2 * mt + 1].s, kk, col_s));
-        mma16816(as[mt], slo.x, shi.x, slo.y, shi.y, bv[2 * kk], bv[2 * kk + 1]);
+        // A columns 2qc, 2qc + 1: coordinates 2kk, 2kk + 16; columns 2qc + 8,
+        // 2qc + 9: coordinates 2kk + 1, 2kk + 17 of the thread's sign word
+        mma16816(as[mt], sign_pair(nsw[2 * mt], 2 * kk), sign_pair(nsw[2 * mt + 1], 2 * kk),
+                 sign_pair(nsw[2 * mt], 2 * kk + 1), sign_pair(nsw[2 * mt + 1], 2 * kk + 1),
+                 bv[2 * kk], bv[2 * kk + 1]);
       }
     }
     // accumulator i of tile mt: row qr + 8·(i >> 1) + 16·mt, head 2·qc + (i & 1)
