@@ -37,7 +37,6 @@
 namespace rrq {
 namespace {
 
-constexpr int kScoreWarpsMax = 16;  // warps per CTA: 16, or 8 / 4 when the tiles do not fit
 constexpr int kScoreTile = 32;   // tokens per warp tile
 constexpr int kScoreStages = 3;  // ring depth (steps)
 template <int W> constexpr int score_u() { return W >= 16 ? 2 : 4; }  // iterations per step
@@ -408,351 +407,18 @@ cudaError_t launch_scores_dbg(const ScoreArgs& a, cudaStream_t stream) {
   return cudaErrorInvalidValue;
 }
 
-// ------------------------------------------------ tensor-core tiles, 4-bit codes
-// 4-bit codes, d = 64 or 128, GQA group G ∈ {1, 2, 4, 8}.  For one kv head g
-// the scores of a 32-token unit are a [32 × d]·[d × G] product of the code
-// levels and the group's rotated queries, run as mma.sync m16n8k16 tiles
-// (fp16 operands, fp32 accumulation): tokens are M (two 16-row tiles), the
-// group's query heads are N (zero columns pad G to 8), d is K.
-//  * Because the dot product sums over coordinates, any assignment of code
-//    pairs to K positions serves, as long as the query operand uses the same
-//    one.  Thread quad position c owns code bytes [c·d/8, (c+1)·d/8) of a row
-//    (one 16- or 8-byte load per row), and in k-step kk its A-fragment columns
-//    2c, 2c+1 hold code byte 2kk of that slice and columns 2c+8, 2c+9 byte
-//    2kk+1.  Each byte becomes its fp16 level pair with one byte permute and
-//    one load from a lane-replicated table, which is the A register itself.
-//  * The B fragments (query pairs in the same order) are built once per CTA in
-//    shared memory, [g][j][lane] 16-byte words, so a unit loads them with
-//    d/32 conflict-free 16-byte loads.
-//  * A unit's codes (32 rows of d/2 bytes, hkv rows apart) and norms stream
-//    through a per-warp cp.async ring of unpadded rows; each 16-byte
-//    (8-byte) fragment load of a quarter (half) warp covers 128 contiguous
-//    bytes, so it is conflict-free.  The warps split the units evenly.
-//  * Epilogue: each accumulator is scaled by ν_t·scale/d and the head's
-//    power-of-two factor and stored; for a head, eight lanes write 32
-//    consecutive bytes.
-template <int D, int W>
-struct MmaScoreSmem {
-  static constexpr int CB = D / 2;          // code bytes per key-head
-  static constexpr int KK = CB / 8;         // k-steps of 16 coordinates
-  static constexpr int CW = CB / 16;        // words of a thread's row slice
-  static constexpr int NS = 3;              // ring stages
-  // ring rows padded so the quads' slice loads (tokens 4r + j, r = 0..7) are
-  // conflict-free: 80 bytes at d = 128 (16-byte copies), 40 at d = 64 (8-byte)
-  // ring rows padded so the quads' slice loads (tokens 4r + j, r = 0..7) are
-  // conflict-free: 80 bytes at d = 128 (16-byte copies), 40 at d = 64 (8-byte)
-  static constexpr int RS = D == 128 ? CB + 16 : CB + 8;
-  static constexpr int CP = D == 128 ? 16 : 8;  // cp.async chunk bytes
-  static constexpr int STAGE = 32 * RS + 32 * 4;
-  static constexpr int RING = NS * STAGE;   // per warp
-  __host__ __device__ static constexpr size_t table() { return 256 * 64 * 4; }  // entry e at byte e·256 + lane·4
-  __host__ __device__ static size_t bq(int hkv) { return size_t(hkv) * 32 * CB; }  // B fragments
-  __host__ __device__ static size_t inv(int hq) { return (size_t(hq) * 4 + 15) / 16 * 16; }
-  __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }  // prologue only (aliases rings)
-  __host__ __device__ static constexpr size_t rings() { return size_t(W) * RING; }
-  __host__ __device__ static size_t head(int hq, int hkv) { return bq(hkv) + inv(hq); }
-  // Plain layout: [table | B fragments | inv | rings (qf aliased)].
-  __host__ __device__ static size_t total(int hq, int hkv) {
-    return table() + head(hq, hkv) + (qf(hq) > rings() ? qf(hq) : rings());
-  }
-  // Folded layout, for a dynamic base at shared address kFoldBase: the table
-  // sits at shared address 0x10000 so that the byte-permuted offset
-  // 0x10000 | byte·256 | lane·4 is the load address itself.  Below it: the B
-  // fragments, inv and the first `front` rings; above it: the other rings
-  // (qf aliased).
-  static constexpr uint32_t kFoldBase = 0x400, kFoldTable = 0x10000;
-  __host__ __device__ static size_t fold_front_rings(int hq, int hkv) {
-    const size_t start = head(hq, hkv);
-    const size_t room = kFoldTable - kFoldBase;
-    const size_t n = start < room ? (room - start) / RING : 0;
-    return n < size_t(W) ? n : size_t(W);
-  }
-  __host__ __device__ static size_t fold_back() { return kFoldTable - kFoldBase + table(); }
-  __host__ __device__ static size_t fold_ring(int hq, int hkv, int w) {
-    const size_t nf = fold_front_rings(hq, hkv);
-    return size_t(w) < nf ? head(hq, hkv) + size_t(w) * RING : fold_back() + (size_t(w) - nf) * RING;
-  }
-  __host__ __device__ static size_t fold_total(int hq, int hkv) {
-    const size_t back = (size_t(W) - fold_front_rings(hq, hkv)) * RING;
-    return head(hq, hkv) <= kFoldTable - kFoldBase ? fold_back() + (qf(hq) > back ? qf(hq) : back)
-                                                   : ~size_t(0);
-  }
-};
+}  // namespace
+}  // namespace rrq
 
-// d += A·B for one m16n8k16 tile: fp16 A (row-major) and B (column-major)
-// fragments, fp32 accumulators.
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+#include "scores_mma.cuh"
 
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-__device__ __forceinline__ uint32_t word_of(const uint2& v, int i) { return i == 0 ? v.x : v.y; }
-
-template <int D, int G, int W, bool FOLD>
-__global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArgs a) {
-  pdl_release();
-  using Sm = MmaScoreSmem<D, W>;
-  constexpr int CB = Sm::CB, KK = Sm::KK, NS = Sm::NS;
-  using Chunk = std::conditional_t<D == 128, uint4, uint2>;  // a thread's slice of a row
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const QuantParams& p = a.p;
-  uint32_t* ptab;
-  uint4* bq;
-  float* inv_s;
-  float* qf;
-  uint8_t* ring;
-  if constexpr (FOLD) {
-    if (smem_addr(smem) != Sm::kFoldBase) {
-      // not the layout the launch assumed: mark every score as invalid
-      pdl_wait();
-      for (int64_t i = int64_t(blockIdx.x) * W * 32 + tid; i < int64_t(a.hq) * a.T; i += int64_t(gridDim.x) * W * 32)
-        a.scores[i] = __int_as_float(0x7fc00000);
-      return;
-    }
-    bq = reinterpret_cast<uint4*>(smem);
-    inv_s = reinterpret_cast<float*>(smem + Sm::bq(a.hkv));
-    ptab = reinterpret_cast<uint32_t*>(smem + (Sm::kFoldTable - Sm::kFoldBase));
-    qf = reinterpret_cast<float*>(smem + Sm::fold_back());
-    ring = smem + Sm::fold_ring(a.hq, a.hkv, warp);
-  } else {
-    ptab = reinterpret_cast<uint32_t*>(smem);
-    bq = reinterpret_cast<uint4*>(smem + Sm::table());
-    inv_s = reinterpret_cast<float*>(smem + Sm::table() + Sm::bq(a.hkv));
-    uint8_t* work = smem + Sm::table() + Sm::head(a.hq, a.hkv);
-    qf = reinterpret_cast<float*>(work);  // prologue only
-    ring = work + warp * Sm::RING;
-  }
-
-  for (int i = tid; i < 256 * 64; i += W * 32) {
-    const int e = i >> 6;
-    const __half2 v = __floats2half2_rn(p.levels[e & 15], p.levels[e >> 4]);
-    ptab[i] = *reinterpret_cast<const uint32_t*>(&v);
-  }
-  pdl_wait();  // from here on, global memory
-  rotate_queries<D>(a, qf, inv_s, warp, lane, W);
-  __syncthreads();
-  // B fragment word w = 2kk + hh of lane l (quad position c, column n): the
-  // rotated pair β = c·d/8 + 2kk + hh of head g·G + n, zero for n ≥ G.
-  {
-    uint32_t* bw = reinterpret_cast<uint32_t*>(bq);
-    for (int i = tid; i < a.hkv * 32 * 2 * KK; i += W * 32) {
-      const int comp = i & 3, l = (i >> 2) & 31, j = (i >> 7) % (KK / 2), g = (i >> 7) / (KK / 2);
-      const int w = 4 * j + comp, kk = w >> 1, hh = w & 1, c = l & 3, n = l >> 2;
-      const int beta = c * (CB / 4) + 2 * kk + hh;
-      __half2 v = __floats2half2_rn(0.f, 0.f);
-      if (n < G) {
-        const float* qh = qf + (g * G + n) * D;
-        v = __floats2half2_rn(qh[2 * beta], qh[2 * beta + 1]);
-      }
-      bw[i] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-  }
-  __syncthreads();  // qf is dead: its space becomes the rings
-
-  // units u = tile·hkv + g (token-major); warp w takes u = w, w + nw, w + 2nw, …
-  // so the warps working at one moment read whole token rows of the cache
-  // together.  The launch makes nw a multiple of hkv, so all units of a warp
-  // have the same kv head g (its B fragments stay in registers) and consecutive
-  // units are TS = nw/hkv tiles apart: every address advances by a constant.
-  const int lg_hkv = __ffs(a.hkv) - 1;  // hkv is a power of two
-  const int64_t nbt = (a.T + 31) >> 5;
-  const int64_t nw = int64_t(gridDim.x) * W, gw = int64_t(blockIdx.x) * W + warp;
-  const int g = int(gw & (a.hkv - 1));
-  const int64_t tile0 = gw >> lg_hkv, TS = nw >> lg_hkv;
-  const int64_t my_units = tile0 < nbt ? (nbt - tile0 + TS - 1) / TS : 0;
-  // FOLD: byte 2 of the permute's second operand is the table's address bit 16
-  const char* tab_bytes = reinterpret_cast<const char*>(ptab);
-  const uint32_t lane4 = uint32_t(lane) * 4u | (FOLD ? Sm::kFoldTable : 0u);
-  const int qc = lane & 3, qr = lane >> 2;  // quad position, token group 4qr .. 4qr + 3
-
-  // Copy k of a unit moves chunk c = lane % CPR of row t = lane / CPR + k·(32 / CPR)
-  constexpr int CPR = CB / Sm::CP;  // copies per row
-  const int lt = lane / CPR, lc = lane % CPR;
-  const int64_t row_bytes = int64_t(a.hkv) * CB;  // global stride between tokens
-  const int64_t unit_step = TS * 32;              // tokens between consecutive units
-  const int64_t src_step = unit_step * row_bytes;
-  const uint8_t* src_next = a.codes + (tile0 * 32 * a.hkv + g) * CB + lt * row_bytes + lc * Sm::CP;
-  const float* nrm_next = a.norms + (tile0 * 32 + lane) * a.hkv + g;
-  int64_t t_next = tile0 * 32;  // first token of the next unit to load
-  const uint32_t ring0 = smem_addr(ring);
-  const uint32_t lane_dst = uint32_t(lt * Sm::RS + lc * Sm::CP);
-  auto copy = [&](uint32_t dst, const uint8_t* src, bool ok) {
-    if constexpr (Sm::CP == 16) cp_async16(dst, ok ? src : a.codes, ok ? 16 : 0);
-    else cp_async8(dst, ok ? src : a.codes, ok ? 8 : 0);
-  };
-  int64_t issued = 0;
-  auto issue = [&](int stage) {
-    if (issued < my_units) {
-      const uint32_t sbase = ring0 + uint32_t(stage * Sm::STAGE);
-      if (t_next + 32 <= a.T) {
-#pragma unroll
-        for (int k = 0; k < CPR; ++k)
-          copy(sbase + lane_dst + k * (32 / CPR) * Sm::RS, src_next + k * (32 / CPR) * row_bytes, true);
-        cp_async4(sbase + 32 * Sm::RS + lane * 4, nrm_next, 4);
-      } else {
-#pragma unroll
-        for (int k = 0; k < CPR; ++k)
-          copy(sbase + lane_dst + k * (32 / CPR) * Sm::RS, src_next + k * (32 / CPR) * row_bytes,
-               t_next + lt + k * (32 / CPR) < a.T);
-        const bool ok = t_next + lane < a.T;
-        cp_async4(sbase + 32 * Sm::RS + lane * 4, ok ? nrm_next : a.norms, ok ? 4 : 0);
-      }
-      ++issued;
-      src_next += src_step;
-      nrm_next += unit_step * a.hkv;
-      t_next += unit_step;
-    }
-    cp_async_commit();
-  };
-#pragma unroll
-  for (int k = 0; k < NS - 1; ++k) issue(k);
-
-  auto level_pair = [&](uint32_t word, int pos) -> uint32_t {
-    uint32_t cv;
-    if constexpr (FOLD) {  // address 0x10000 | byte·256 | lane·4
-      const uint32_t addr = __byte_perm(word, lane4, 0x7604u | (pos << 4));
-      asm("ld.shared.b32 %0, [%1];" : "=r"(cv) : "r"(addr));
-    } else {
-      const uint32_t off = __byte_perm(word, lane4, 0x5504u | (pos << 4));
-      cv = *reinterpret_cast<const uint32_t*>(tab_bytes + off);
-    }
-    return cv;
-  };
-
-  // the lane's B fragments (k-step kk: words 2kk, 2kk + 1) and head scales
-  uint32_t bfr[KK][2];
-#pragma unroll
-  for (int j = 0; j < KK / 2; ++j) {
-    const uint4 v = bq[(g * (KK / 2) + j) * 32 + lane];
-    bfr[2 * j][0] = v.x;
-    bfr[2 * j][1] = v.y;
-    bfr[2 * j + 1][0] = v.z;
-    bfr[2 * j + 1][1] = v.w;
-  }
-  float hsc[2];
-#pragma unroll
-  for (int e = 0; e < 2; ++e)
-    hsc[e] = 2 * qc + e < G ? a.scale * p.inv_d * inv_s[g * G + 2 * qc + e] : 0.f;
-  const bool vec_out = (a.T & 3) == 0;  // 16-byte score stores stay aligned
-  const int h0 = g * G + 2 * qc;        // the lane's first head
-  float* out_next = a.scores + int64_t(h0) * a.T + tile0 * 32 + 4 * qr;
-  int64_t t0 = tile0 * 32;
-
-  int stage = 0;
-  for (int64_t k = 0; k < my_units; ++k) {
-    cp_async_wait<NS - 2>();
-    __syncwarp();
-    const uint8_t* st = ring + stage * Sm::STAGE;
-    // token 4qr + j (j = 2mt + h) is row qr + 8h of m-tile mt
-    Chunk cw[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) cw[j] = *reinterpret_cast<const Chunk*>(st + (4 * qr + j) * Sm::RS + qc * (CB / 4));
-    const float4 nu = *reinterpret_cast<const float4*>(st + 32 * Sm::RS + 16 * qr);
-    __syncwarp();  // every lane has read this stage before it is refilled
-    issue(stage == 0 ? NS - 1 : stage - 1);
-    stage = (stage + 1 == NS) ? 0 : stage + 1;
-
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int kk = 0; kk < KK; ++kk) {
-      const int wi = kk >> 1, pos = 2 * (kk & 1);
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const uint32_t lo = word_of(cw[2 * mt], wi), hi = word_of(cw[2 * mt + 1], wi);
-        mma_16816(acc[mt], level_pair(lo, pos), level_pair(hi, pos), level_pair(lo, pos + 1),
-                  level_pair(hi, pos + 1), bfr[kk][0], bfr[kk][1]);
-      }
-    }
-
-    // accumulator i of tile mt: token 4qr + 2mt + (i >> 1), head 2qc + (i & 1)
-    const bool full = vec_out && t0 + 32 <= a.T;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      if (2 * qc + e < G) {
-        float* out = out_next + int64_t(e) * a.T;
-        const float2 hs2 = make_float2(hsc[e], hsc[e]);
-        const float2 s01 = mul2(make_float2(nu.x, nu.y), hs2), s23 = mul2(make_float2(nu.z, nu.w), hs2);
-        const float2 v01 = mul2(make_float2(acc[0][e], acc[0][2 + e]), s01);
-        const float2 v23 = mul2(make_float2(acc[1][e], acc[1][2 + e]), s23);
-        const float4 v = make_float4(v01.x, v01.y, v23.x, v23.y);
-        if (full) {
-          *reinterpret_cast<float4*>(out) = v;
-        } else {
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (t0 + 4 * qr + j < a.T) out[j] = vv[j];
-        }
-      }
-    }
-    out_next += TS * 32;
-    t0 += TS * 32;
-  }
-  cp_async_wait<0>();
-}
-
-template <int D, int G, int W>
-cudaError_t launch_scores_mma_w(const ScoreArgs& a, cudaStream_t stream) {
-  using Sm = MmaScoreSmem<D, W>;
-  int dev = 0, reserved = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-  const bool fold = reserved == int(Sm::kFoldBase) && Sm::fold_total(a.hq, a.hkv) <= 227 * 1024;
-  auto k = fold ? qk_scores_mma_kernel<D, G, W, true> : qk_scores_mma_kernel<D, G, W, false>;
-  const size_t smem = fold ? Sm::fold_total(a.hq, a.hkv) : Sm::total(a.hq, a.hkv);
-  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  const int64_t units = ((a.T + 31) / 32) * a.hkv;
-  int grid = grid_for(reinterpret_cast<const void*>(k), W * 32, smem, (units + W - 1) / W);
-  // the kernel needs the warp count grid·W to be a multiple of hkv (a power of
-  // two): round the grid to a multiple of hkv/W when hkv exceeds W
-  if (a.hkv > W) {
-    const int m = a.hkv / W;
-    grid = grid < m ? m : grid / m * m;
-  }
-  return launch_pdl(k, grid, W * 32, smem, stream, a);
-}
-
-// The tensor-core kernel applies (4-bit codes, d ≤ 128, a power-of-two group
-// ≤ 8, and its shared memory fits with 16 or 8 warps); returns its warps or 0.
-template <int D>
-int mma_score_warps(int bits, int hq, int hkv) {
-  const int group = hq / hkv;
-  if (bits != 4 || (D != 64 && D != 128) || group > 8 || (group & (group - 1))) return 0;
-  if (MmaScoreSmem<D, 16>::total(hq, hkv) <= 227 * 1024) return 16;
-  if (MmaScoreSmem<D, 8>::total(hq, hkv) <= 227 * 1024) return 8;
-  return 0;
-}
-
-template <int D, int G>
-cudaError_t launch_scores_mma_g(const ScoreArgs& a, cudaStream_t stream) {
-  if (mma_score_warps<D>(4, a.hq, a.hkv) == 16) return launch_scores_mma_w<D, G, 16>(a, stream);
-  return launch_scores_mma_w<D, G, 8>(a, stream);
-}
-
-template <int D>
-cudaError_t launch_scores_mma(const ScoreArgs& a, cudaStream_t stream) {
-  switch (a.group) {
-    case 1: return launch_scores_mma_g<D, 1>(a, stream);
-    case 2: return launch_scores_mma_g<D, 2>(a, stream);
-    case 4: return launch_scores_mma_g<D, 4>(a, stream);
-    case 8: return launch_scores_mma_g<D, 8>(a, stream);
-  }
-  return cudaErrorInvalidValue;
-}
+namespace rrq {
+namespace {
 
 template <int D, int B>
 cudaError_t launch_scores_db(const ScoreArgs& a, cudaStream_t stream) {
-  if constexpr (B == 4 && D <= 128) {
-    if (mma_score_warps<D>(B, a.hq, a.hkv) > 0) return launch_scores_mma<D>(a, stream);
+  if constexpr (D <= 256) {
+    if (mma_score_warps<D, B>(a.hq, a.hkv) > 0) return launch_scores_mma<D, B>(a, stream);
   }
   switch (a.group) {
     case 1: return launch_scores_dbg<D, B, 1>(a, stream);
@@ -790,8 +456,13 @@ bool qk_scores_supported(int d, int bits, int hq, int hkv) {
   }
   (void)hb;
   if (w > 0) return true;  // a warp's head block is fixed: head blocks divide the warps
-  if (d == 64) return mma_score_warps<64>(bits, hq, hkv) > 0;
-  if (d == 128) return mma_score_warps<128>(bits, hq, hkv) > 0;
+  switch (d * 10 + bits) {
+#define RRQ_MW(DD, BB) case DD * 10 + BB: return mma_score_warps<DD, BB>(hq, hkv) > 0;
+    RRQ_MW(64, 1) RRQ_MW(64, 2) RRQ_MW(64, 3) RRQ_MW(64, 4)
+    RRQ_MW(128, 1) RRQ_MW(128, 2) RRQ_MW(128, 3) RRQ_MW(128, 4)
+    RRQ_MW(256, 1) RRQ_MW(256, 2) RRQ_MW(256, 3) RRQ_MW(256, 4)
+#undef RRQ_MW
+  }
   return false;
 }
 
