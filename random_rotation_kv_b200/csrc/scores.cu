@@ -417,9 +417,7 @@ namespace {
 
 template <int D, int B>
 cudaError_t launch_scores_db(const ScoreArgs& a, cudaStream_t stream) {
-  if constexpr (D <= 256) {
-    if (mma_score_warps<D, B>(a.hq, a.hkv) > 0) return launch_scores_mma<D, B>(a, stream);
-  }
+  if (mma_score_warps<D, B>(a.hq, a.hkv) > 0) return launch_scores_mma<D, B>(a, stream);
   switch (a.group) {
     case 1: return launch_scores_dbg<D, B, 1>(a, stream);
     case 2: return launch_scores_dbg<D, B, 2>(a, stream);
@@ -461,6 +459,7 @@ bool qk_scores_supported(int d, int bits, int hq, int hkv) {
     RRQ_MW(64, 1) RRQ_MW(64, 2) RRQ_MW(64, 3) RRQ_MW(64, 4)
     RRQ_MW(128, 1) RRQ_MW(128, 2) RRQ_MW(128, 3) RRQ_MW(128, 4)
     RRQ_MW(256, 1) RRQ_MW(256, 2) RRQ_MW(256, 3) RRQ_MW(256, 4)
+    RRQ_MW(512, 1) RRQ_MW(512, 2) RRQ_MW(512, 3) RRQ_MW(512, 4)
 #undef RRQ_MW
   }
   return false;

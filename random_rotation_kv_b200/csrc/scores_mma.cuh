@@ -1,5 +1,5 @@
 // scores_mma.cuh — the tensor-core score kernel for b ∈ {1, 2, 3, 4} and
-// d ∈ {64, 128, 256}, included by scores.cu (ScoreArgs, rotate_queries).
+// d ∈ {64, 128, 256, 512}, included by scores.cu (ScoreArgs, rotate_queries).
 //
 // "Random-rotation quantization" page, "Three decoders, one rotation",
 // inner-product decoder: s[h,t] = scale·(ν/d)·Σ_i q'_{h,i}·c[code_i], q' = H·D·q.
@@ -50,18 +50,17 @@ template <int D, int B, int W> struct ScoreMmaCfg {
   static constexpr int PADT = SB >= 16 ? 16 : SB >= 8 ? 8 : 4;
   static constexpr int RS = CB + ((PADT - CB % 32) % 32 + 32) % 32;
   static constexpr int CP = RS % 16 == 0 ? 16 : RS % 8 == 0 ? 8 : 4;  // cp.async bytes
-  static constexpr int NS = 3;                       // ring stages
+  static constexpr int NS = D >= 512 ? 2 : 3;        // ring stages
   static constexpr int STAGE = (32 * RS + 32 * 4 + 15) / 16 * 16;
   static constexpr int RING = NS * STAGE;
   static constexpr bool TABLE = B != 1;
   static constexpr uint32_t kBase = 0x400, kTable = 0x10000;
   static constexpr uint32_t TABLE_BYTES = B == 3 ? 64 * 256 : B == 1 ? 0 : 256 * 256;
   static constexpr int SW = (SB + 3) / 4;            // slice words per chunk
-  // [bq | inv | qsum | front rings] below 0x10000, the table, [back rings] (qf
+  // [inv | qsum | front rings] below 0x10000, the table, [back rings] (qf
   // aliases the back region in the prologue)
-  __host__ __device__ static size_t bq(int hkv) { return size_t(hkv) * 32 * KK * 8; }
   __host__ __device__ static size_t inv(int hq) { return (size_t(hq) * 8 + 15) / 16 * 16; }
-  __host__ __device__ static size_t head(int hq, int hkv) { return bq(hkv) + inv(hq); }
+  __host__ __device__ static size_t head(int hq, int hkv) { return (void)hkv, inv(hq); }
   __host__ __device__ static size_t qf(int hq) { return size_t(hq) * D * 4; }
   __host__ __device__ static size_t front(int hq, int hkv) {
     const size_t start = (head(hq, hkv) + 15) / 16 * 16, room = kTable - kBase;
@@ -140,8 +139,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
       a.scores[i] = __int_as_float(0x7fc00000);
     return;
   }
-  uint2* bq = reinterpret_cast<uint2*>(smem);
-  float* inv_s = reinterpret_cast<float*>(smem + Cf::bq(a.hkv));
+  float* inv_s = reinterpret_cast<float*>(smem);
   float* qsum = inv_s + a.hq;  // Σ_i q'_{h,i} (1-bit codes)
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + (Cf::kTable - Cf::kBase));
   float* qf = reinterpret_cast<float*>(smem + Cf::back0());
@@ -179,26 +177,6 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
       if (lane == 0) qsum[h] = acc * inv_s[h];
     }
   }
-  // B fragments: [g][kk][lane] words (b0, b1): head n = lane/4 of group g
-  // (zero for n ≥ G), quad position c = lane % 4; in chunk ch, k-step kc,
-  // b0 holds pair 2kc and b1 pair 2kc + 1 of thread c's slice.
-  for (int i = tid; i < a.hkv * KK * 32; i += W * 32) {
-    const int l = i & 31, kk = (i >> 5) % KK, g = (i >> 5) / KK;
-    const int c = l & 3, n = l >> 2, ch = kk / KC, kc = kk % KC;
-    uint32_t w[2] = {0u, 0u};
-    if (n < G) {
-      const float* qh = qf + (g * G + n) * D + ch * Cf::CS + c * CC;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int pr = 2 * kc + j;
-        const __half2 v = __floats2half2_rn(qh[pair_coord<B, CC>(pr, 0)], qh[pair_coord<B, CC>(pr, 1)]);
-        w[j] = *reinterpret_cast<const uint32_t*>(&v);
-      }
-    }
-    bq[i] = make_uint2(w[0], w[1]);
-  }
-  __syncthreads();  // qf is dead: its space becomes the back rings
-
   // ---- units u = tile·hkv + g, warp-strided (the launch makes nw a multiple of hkv)
   const int lg_hkv = __ffs(a.hkv) - 1;  // hkv is a power of two
   const int64_t nbt = (a.T + 31) >> 5;
@@ -208,6 +186,26 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
   const int64_t my_units = tile0 < nbt ? (nbt - tile0 + TS - 1) / TS : 0;
   const uint32_t col = Cf::kTable | uint32_t(lane) * 4u, col2 = col | 128u;
   const int qc = lane & 3, qr = lane >> 2;
+
+  // this lane's B fragments (the kv head is fixed): head qr of group g (zero for
+  // qr ≥ G); in chunk ch, k-step kc, b0 holds pair 2kc and b1 pair 2kc + 1 of
+  // quad thread qc's slice
+  uint32_t bfr[KK][2];
+#pragma unroll
+  for (int kk = 0; kk < KK; ++kk) {
+    const int ch = kk / KC, kc = kk % KC;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      __half2 v = __floats2half2_rn(0.f, 0.f);
+      if (qr < G) {
+        const float* qh = qf + (g * G + qr) * D + ch * Cf::CS + qc * CC;
+        const int pr = 2 * kc + j;
+        v = __floats2half2_rn(qh[pair_coord<B, CC>(pr, 0)], qh[pair_coord<B, CC>(pr, 1)]);
+      }
+      bfr[kk][j] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  }
+  __syncthreads();  // qf is dead: its space becomes the back rings
 
   // copy k of a unit (k < CPR) moves chunk i % CPR of row i / CPR, i = lane + 32k
   constexpr int CPR = CB / Cf::CP;  // copies per row = copies per lane
@@ -252,14 +250,7 @@ __global__ void __launch_bounds__(W * 32, 1) qk_scores_mma_kernel(const ScoreArg
 #pragma unroll
   for (int k = 0; k < NS - 1; ++k) issue(k);
 
-  // this lane's B fragments and head scales (the kv head is fixed)
-  uint32_t bfr[KK][2];
-#pragma unroll
-  for (int kk = 0; kk < KK; ++kk) {
-    const uint2 v = bq[(g * KK + kk) * 32 + lane];
-    bfr[kk][0] = v.x;
-    bfr[kk][1] = v.y;
-  }
+  // head scales of the lane's two accumulator columns
   float hsc[2], hoff[2];  // scale·inv_d/s_h (× h for b = 1) and scale·inv_d·m·Σq'
   {
     const float cm = 0.5f * (p.levels[0] + p.levels[1]), ch = 0.5f * (p.levels[1] - p.levels[0]);
@@ -382,13 +373,13 @@ cudaError_t launch_scores_mma_w(const ScoreArgs& a, cudaStream_t stream) {
 }
 
 // Warps of the tensor-core kernel for (d, b, hq, hkv): 16 for d ≤ 128, 8 for
-// d = 256, as long as the shared layout fits; 0 when it does not apply (a
-// group above 8 or not a power of two, d = 512, a device whose reserved
-// shared memory is not the 1 KB the fixed layout assumes).
+// d ≥ 256, as long as the shared layout fits; 0 when it does not apply (a
+// group above 8 or not a power of two, a device whose reserved shared memory
+// is not the 1 KB the fixed layout assumes).
 template <int D, int B>
 int mma_score_warps(int hq, int hkv) {
   const int group = hq / hkv;
-  if (D > 256 || group > 8 || (group & (group - 1))) return 0;
+  if (group > 8 || (group & (group - 1))) return 0;
   int dev = 0, reserved = 0;
   if (cudaGetDevice(&dev) == cudaSuccess &&
       cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
