@@ -34,6 +34,7 @@
 #include "tensor_map.h"
 #include "mma_encode.cuh"
 #include "mma_decode.cuh"
+#include "tc_encode.cuh"
 
 namespace rrq {
 
@@ -296,7 +297,9 @@ cudaError_t launch_encode_batch(const T* x, int64_t n, const QuantParams& p, uin
                                 float* norms, cudaStream_t stream) {
   if constexpr (D == 128 && B == 4) {
     if (p.norm_mode == 0) {
-      const cudaError_t e = launch_encode_mma<T>(x, n, p, codes, norms, stream);
+      cudaError_t e = launch_encode_tc<T>(x, n, p, codes, norms, stream);
+      if (e != cudaErrorNotSupported) return e;
+      e = launch_encode_mma<T>(x, n, p, codes, norms, stream);
       if (e != cudaErrorNotSupported) return e;
     }
   }

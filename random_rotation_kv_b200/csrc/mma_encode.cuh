@@ -102,11 +102,18 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
 // the comparison being the carry of I − (thr_j + 1) added to lo_j,
 // with no saturation and no separate s.  A codebook with two thresholds within
 // one cell of the reachable range (closer than 1/4) takes another encoder.
+// The same decision in one integer add: with off_j chosen so that
+//     bits(f) + off_j ≡ (lo_j + 1)·2^16 + (I − thr_j − 1)   (cell with a threshold)
+//     bits(f) + off_j ≡  lo_j·2^16      + (I − 2^16·j)      (cell without one)
+// modulo 2^24, byte 2 of bits(f) + off_j is the code itself: in the first case
+// I − thr_j − 1 lies in [−2^16, 2^16) and borrows from byte 2 exactly when
+// I ≤ thr_j; in the second it lies in [0, 2^16).
 struct FixedSearch {
-  int ok;          // 0: the table cannot serve this codebook (another encoder runs)
-  float num;       // 2^18 (scaled by 1/ν per vector)
-  float bias;      // 1.5·2^23
-  uint2 rows[128]; // row r = cell r − 64: (biased threshold inside it + 1, or 2^32 − 1; lo)
+  int ok;            // 0: the table cannot serve this codebook (another encoder runs)
+  float num;         // 2^18 (scaled by 1/ν per vector)
+  float bias;        // 1.5·2^23
+  uint2 rows[128];   // row r = cell r − 64: (biased threshold inside it + 1, or 2^32 − 1; lo)
+  uint32_t off[128]; // row r: off_j above (mod 2^32)
 };
 
 // Host: the fixed-point parameters for a codebook (levels ascending, L = 2^bits)
@@ -132,11 +139,18 @@ inline FixedSearch make_fixed_search(const QuantParams& p) {
   for (int r = 0; r < 128; ++r) {
     const int64_t edge = int64_t(r - 64) * 65536;  // I at the cell's lower end
     uint32_t lo = 0, thr = 0xFFFFFFFFu;
+    int64_t anchor = edge;  // the I that lands on a whole multiple of 2^16: edge, or thr_j + 1
     for (int k = 0; k < nthr; ++k) {
-      if (T[k] < edge) ++lo;
-      else if (T[k] < edge + 65536) thr = uint32_t(int32_t(0x4B400000) + T[k]) + 1u;
+      if (T[k] < edge) {
+        ++lo;
+      } else if (T[k] < edge + 65536) {
+        thr = uint32_t(int32_t(0x4B400000) + T[k]) + 1u;
+        anchor = int64_t(T[k]) + 1;
+      }
     }
     fs.rows[r] = make_uint2(thr, lo);
+    const int64_t target = int64_t(lo + (thr == 0xFFFFFFFFu ? 0u : 1u)) << 16;
+    fs.off[r] = uint32_t(uint64_t(target - (int64_t(0x4B400000) + anchor)));
   }
   return fs;
 }

@@ -245,6 +245,13 @@ __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
   return v;
 }
 
+// One 32-bit word from shared memory.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 // Waits until at most one committed bulk store still reads shared memory.
 __device__ __forceinline__ void bulk_wait_read_1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");

@@ -69,6 +69,24 @@ inline bool code_tensor_map(CUtensorMap* map, const void* base, int64_t rows, in
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map over `rows` rows of `row_bytes` bytes (a multiple of 32) at `base`,
+// moved in boxes of 32 bytes × `box_rows` rows with the 32-byte swizzle: inside
+// each 256-byte block of shared memory, the 16-byte chunk c of 32-byte line r
+// sits at chunk position c ^ ((r >> 2) mod 2).  Stores clip rows past the end
+// of the array.  False if the driver rejects the map.
+inline bool code_box32_tensor_map(CUtensorMap* map, const void* base, int64_t rows, int row_bytes,
+                                  int box_rows) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr || rows <= 0 || rows > (int64_t(1) << 32) || row_bytes % 32 != 0) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(row_bytes), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(row_bytes)};
+  const cuuint32_t box[2] = {32, cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Map over `rows` rows of `row_elems` 16-bit elements at `base` (16-byte
 // aligned, row pitch a multiple of 16 bytes), moved in boxes of 32 elements
 // (64 bytes) × `box_rows` rows with the 64-byte swizzle (as code_tensor_map).
