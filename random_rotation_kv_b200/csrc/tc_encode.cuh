@@ -1,32 +1,35 @@
 // tc_encode.cuh — encoder for d = 128, 4-bit codes and 16-bit inputs (the
-// KV-cache case) with the 32×32 Hadamard blocks on tcgen05 and the
-// accumulators in tensor memory.
+// KV-cache case) with the rotation on tcgen05 and the accumulators in tensor
+// memory.
 //
 // "Random-rotation quantization" page: scheme steps 1–2, "Why rotation works"
 // (the randomized Hadamard transform), "History", EDEN and TurboQuant bullets.
-// As in mma_encode.cuh, H_128 = H_4 ⊗ H_32 over c = 32a + b:
-//     z[a, b] = Σ_b' H_32[b, b']·s_{32a+b'}·x_{32a+b'},   y'[32a + b] = Σ_a' H_4[a, a']·z[a', b].
-// A CTA has two groups of eight warps; each group owns 128-row tiles:
+// The rotated vector y' = H_128·D·x is formed as one dense product per tile:
+// the ±1 matrix B^T[n][k] = s_k·H_128[n, k] (Sylvester order, the seeded signs
+// folded in) is exact in fp16 and bf16, so tcgen05.mma (M = 128 rows, N = 128,
+// K = 16, operands as stored, fp32 accumulation) gives every y'_n of a row
+// with no butterfly left on the CUDA cores, which bound this kernel; the tensor
+// pipe runs a few per cent busy.  A CTA has two groups of eight warps; each
+// group owns 128-row tiles:
 //  * one elected thread of the group loads a tile with two TMA boxes (128 rows
-//    × 128 bytes, 128-byte swizzle) and issues, per block a, two
-//    tcgen05.mma (M = 128, N = 32, K = 16, fp16/bf16 operands as stored, fp32
-//    accumulation) of the tile's K slice against B_a = the ±1 table with the
-//    rotation signs folded in; the accumulators are 4 × 32 columns of tensor
-//    memory, two buffers per group, so the next tile's products run while the
-//    warps finish this one;
+//    × 128 bytes, 128-byte swizzle) and issues its eight products into one of
+//    the group's two 128-column tensor-memory buffers, so the next tile's
+//    products run while the warps finish this one;
 //  * tensor-memory lane r (row r of the tile) is read by two threads, warp
-//    w and w + 4 of the group: both sum all 128 z² (ν² = ‖y'‖²/d = 4·Σ z²/d),
-//    then read the row again in column quarters and form y' and the codes
-//    of blocks 2h and 2h + 1 only (thread half h), i.e. bytes [32h, 32h + 32)
-//    of the code row; registers hold at most 64 z values at a time;
+//    w and w + 4 of the group: thread half h takes coordinates [64h, 64h + 64),
+//    i.e. bytes [32h, 32h + 32) of the code row; the two halves of ‖y'‖²
+//    meet through shared memory and a 64-thread named barrier (ν² = ‖y'‖²/d),
+//    summed in one order by both;
 //  * the code of a coordinate is byte 2 of bits(f) + off_j, one lane-replicated
 //    table load and one add (FixedSearch, mma_encode.cuh), and eight codes go
 //    into a word by byte permutes;
 //  * codes leave through a per-warp 32 × 32-byte tile in the 32-byte swizzle
 //    (conflict-free for row-per-thread stores) and a TMA tensor store.
-// Every wait is bounded; after a timeout the tile's norms are NaN, the copies
-// and products still in flight are waited for (bounded) and the tensor memory
-// is freed.
+// Every wait is bounded, and each pair of warps takes its go/stop decision
+// for a tile together (a barrier reduction), so a pair never splits at its
+// named barrier; after a timeout the tile's norms are NaN, the copies and
+// products still in flight are waited for (bounded) and the tensor memory is
+// freed.
 #pragma once
 
 #include "mma_encode.cuh"
@@ -35,25 +38,27 @@
 namespace rrq {
 
 struct EncTc {
-  static constexpr int D = 128, NB = 4, TILE = 128, GROUPS = 2, WARPS = 16, THREADS = WARPS * 32;
-  static constexpr uint32_t kBase = 0x400;       // dynamic shared memory base (checked)
-  static constexpr uint32_t HT = 0;              // 4 blocks × [32 n × 32 k] core matrices, 2 KB each
-  static constexpr uint32_t SIGNS = HT + NB * 2048;
-  static constexpr uint32_t BARS = SIGNS + D;    // [group][stage]: in_full, mma_done, tmem_free
-  static constexpr uint32_t TSLOT = BARS + GROUPS * 2 * 3 * 8;
-  static constexpr uint32_t FLAGS = TSLOT + 16;  // [group] failure flags
-  static constexpr uint32_t CTILE = 0x3000;      // shared address: 16 warps × 2 × 1 KB code tiles
-  static constexpr uint32_t kTable = 0x10000;    // off_j at kTable + j·256 + lane·4
+  static constexpr int D = 128, TILE = 128, GROUPS = 2, WARPS = 16, THREADS = WARPS * 32;
+  // shared addresses (the dynamic base is checked to be kBase)
+  static constexpr uint32_t kBase = 0x400;
+  static constexpr uint32_t HT = 0x400;       // B^T: 16 n-groups × 16 k-groups of 8×8 core matrices, 32 KB
+  static constexpr uint32_t SIGNS = 0x8400;   // 128 sign bits, bit k of word k / 32
+  static constexpr uint32_t BARS = 0x8480;    // [group][stage]: in_full, mma_done, tmem_free
+  static constexpr uint32_t TSLOT = 0x84E0;
+  static constexpr uint32_t FLAGS = 0x84F0;   // [group] failure flags
+  static constexpr uint32_t PSUM = 0x8800;    // [group][tile parity][half][row] partial ‖y'‖², 4 KB
+  static constexpr uint32_t CTILE = 0x9800;   // 16 warps × 1 KB code tiles
+  static constexpr uint32_t kTable = 0x10000; // off_j at kTable + j·256 + lane·4
   static constexpr uint32_t kStages = 0x18000;
   static constexpr uint32_t STAGE = TILE * D * 2;   // 32 KB: two boxes of 16 KB
   static constexpr size_t kTotal = size_t(kStages + GROUPS * 2 * STAGE) - kBase;
-  static_assert(kBase + FLAGS + 16 <= CTILE, "head");
-  static_assert(CTILE + WARPS * 2 * 1024 <= kTable, "code tiles");
+  static_assert(HT + D * D * 2 <= SIGNS && BARS + GROUPS * 2 * 3 * 8 <= TSLOT && FLAGS + 16 <= PSUM, "head");
+  static_assert(PSUM + GROUPS * 2 * 2 * TILE * 4 <= CTILE && CTILE + WARPS * 1024 <= kTable, "code tiles");
   static_assert(kTotal <= 227 * 1024, "shared memory");
   // instruction descriptor, kind::f16: D fp32, A and B fp16 (or both bf16),
-  // K-major, N = 32, M = 128
+  // K-major, N = 128, M = 128
   static constexpr uint32_t idesc(bool bf16) {
-    return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | ((32u / 8) << 17) | ((128u / 16) << 24);
+    return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | ((128u / 8) << 17) | ((128u / 16) << 24);
   }
 };
 
@@ -65,17 +70,33 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// AND of `v` over the `nthreads` threads (whole warps) meeting at named barrier `id`.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_named(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <typename T>
 __global__ void __launch_bounds__(EncTc::THREADS, 1)
 encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
                  int64_t n, float* __restrict__ norms, const QuantParams p,
                  const __grid_constant__ FixedSearch fs) {
   using L = EncTc;
-  constexpr int NB = L::NB;
   pdl_release();
   extern __shared__ __align__(1024) uint8_t dsm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = warp >> 3, h = (warp >> 2) & 1, q = warp & 3;  // group, block half, lane quarter
+  const int g = warp >> 3, h = (warp >> 2) & 1, q = warp & 3;  // group, row half, lane quarter
   const int64_t ntiles = (n + L::TILE - 1) / L::TILE;
   const int64_t tstride = int64_t(L::GROUPS) * gridDim.x;
   const int64_t t0 = int64_t(g) * gridDim.x + blockIdx.x;
@@ -89,18 +110,22 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     }
     return;
   }
-  uint8_t* htab = dsm + L::HT;
-  uint8_t* signs = dsm + L::SIGNS;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(dsm + L::BARS);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(dsm + L::TSLOT);
-  volatile int* gfail = reinterpret_cast<volatile int*>(dsm + L::FLAGS);
-  uint32_t* tab = reinterpret_cast<uint32_t*>(dsm + (L::kTable - L::kBase));
+  auto at = [&](uint32_t addr) { return dsm + (addr - L::kBase); };
+  uint32_t* smask = reinterpret_cast<uint32_t*>(at(L::SIGNS));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(at(L::BARS));
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(at(L::TSLOT));
+  volatile int* gfail = reinterpret_cast<volatile int*>(at(L::FLAGS));
+  float* psum = reinterpret_cast<float*>(at(L::PSUM));
+  uint32_t* tab = reinterpret_cast<uint32_t*>(at(L::kTable));
   auto in_full = [&](int s) { return &bars[(g * 2 + s) * 3 + 0]; };
   auto mma_done = [&](int s) { return &bars[(g * 2 + s) * 3 + 1]; };
   auto tmem_free = [&](int s) { return &bars[(g * 2 + s) * 3 + 2]; };
 
   // ---- tables, barriers, tensor memory
-  for (int i = tid; i < L::D; i += blockDim.x) signs[i] = uint8_t(sign_bit(p.seed, i));
+  if (warp < L::D / 32) {
+    const uint32_t m = __ballot_sync(kFull, sign_bit(p.seed, 32 * warp + lane) != 0);
+    if (lane == 0) smask[warp] = m;
+  }
   for (int i = tid; i < 128 * 32; i += blockDim.x) tab[(i >> 5) * 64 + (i & 31)] = fs.off[i >> 5];
   if (tid == 0) {
     for (int i = 0; i < L::GROUPS * 2; ++i) {
@@ -118,15 +143,25 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   __syncthreads();
-  // B_a^T[n][k] = s_{32a+k}·H_32[n, k] in the no-swizzle core-matrix layout
-  // (8 n × 8 k per 128 bytes; 128 bytes between k groups, 512 between n groups)
-  for (int i = tid; i < NB * 32 * 32; i += blockDim.x) {
-    const int k = i & 31, nn = (i >> 5) & 31, a = i >> 10;
-    const int neg = (signs[32 * a + k] ^ __popc(nn & k)) & 1;
-    const uint32_t off = uint32_t(a * 2048 + (nn >> 3) * 512 + (k >> 3) * 128 + (nn & 7) * 16 + (k & 7) * 2);
-    *reinterpret_cast<uint16_t*>(htab + off) = neg ? MmaType<T>::kMinusOne : MmaType<T>::kOne;
+  // B^T[n][k] = s_k·(−1)^popc(n & k), K-major, no swizzle: core matrix (n/8, k/8)
+  // of 8 n × 8 k at 2048·(n/8) + 128·(k/8), row n % 8 at 16·(n % 8), one
+  // 16-byte row per item.  For k = 8kb + j the sign bit is s_k ⊕ parity(n & 8kb)
+  // ⊕ parity((n mod 8) & j); the last term over j = 0..7 is the byte
+  // 0xAA·n₀ ⊕ 0xCC·n₁ ⊕ 0xF0·n₂ (n_i the bits of n mod 8).
+  for (int i = tid; i < L::D * L::D / 8; i += blockDim.x) {
+    const int m = i & 7, kb = (i >> 3) & 15, nn = ((i >> 7) << 3) | m;
+    uint32_t e = (m & 1 ? 0xAAu : 0u) ^ (m & 2 ? 0xCCu : 0u) ^ (m & 4 ? 0xF0u : 0u);
+    e ^= (smask[kb >> 2] >> (8 * (kb & 3))) & 0xFFu;
+    e ^= (__popc(nn & (kb << 3)) & 1) ? 0xFFu : 0u;
+    constexpr uint32_t one2 = uint32_t(MmaType<T>::kOne) * 0x10001u;  // −1 = 1 with bit 15 set
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) w[t] = one2 | (((e >> (2 * t)) & 1u) << 15) | (((e >> (2 * t + 1)) & 1u) << 31);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(L::HT + uint32_t((nn >> 3) * 2048 + kb * 128 + m * 16)),
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                 : "memory");
   }
-  fence_proxy_async_smem();  // the tables are visible to the tensor cores
+  fence_proxy_async_smem();  // the table is visible to the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -135,7 +170,6 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
 
   const bool leader = tid == 256 * g;  // lane 0 of the group's first warp
   const uint32_t stage0 = L::kStages + uint32_t(g * 2) * L::STAGE;
-  const uint32_t ht0 = smem_addr(htab);
   constexpr uint32_t IDESC = L::idesc(MmaType<T>::kOne == 0x3F80u);
   auto issue_tma = [&](int64_t k) {
     const int s = int(k & 1);
@@ -148,12 +182,9 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     const int s = int(k & 1);
     const uint32_t st = stage0 + s * L::STAGE;
 #pragma unroll
-    for (int a = 0; a < NB; ++a)
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks)
-        tc_mma_f16(tmem + uint32_t(s * 128 + a * 32),
-                   smem_desc_sw128(st + (a >> 1) * (L::STAGE / 2) + (a & 1) * 64 + ks * 32),
-                   smem_desc(ht0 + a * 2048 + ks * 256, 128, 512), IDESC, uint32_t(ks));
+    for (int ks = 0; ks < L::D / 16; ++ks)
+      tc_mma_f16(tmem + uint32_t(s * 128), smem_desc_sw128(st + (ks >> 2) * (L::STAGE / 2) + (ks & 3) * 32),
+                 smem_desc(L::HT + uint32_t(ks) * 256, 128, 2048), IDESC, uint32_t(ks));
     mma_commit(mma_done(s));
   };
 
@@ -178,18 +209,18 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     }
   }
 
-  const uint32_t ctile0 = L::CTILE + uint32_t(warp) * 2 * 1024;
+  const uint32_t pair_bar = uint32_t(1 + 4 * g + q);  // warps (g, 0, q) and (g, 1, q)
+  const uint32_t tile = L::CTILE + uint32_t(warp) * 1024;
   const uint32_t swz = uint32_t((lane >> 2) & 1);
   const float2 bias2 = make_float2(fs.bias, fs.bias);
   const float num = fs.num;
-  const float hsign = h ? -1.f : 1.f;  // y'[32(2h)+b] = p0 + (±p1), y'[32(2h+1)+b] = m0 + (±m1)
   const uint32_t lane_word = L::kTable | uint32_t(lane) * 4u;
-  int ct = 0;
+  const int row = 32 * q + lane;
   int64_t k = 0;
   for (; k < my_tiles; ++k) {
     const int s = int(k & 1);
     const uint32_t ph = uint32_t(k >> 1) & 1u;
-    if (!__all_sync(kFull, gfail[g] == 0 && tc_wait(mma_done(s), ph))) break;
+    if (!bar_and(pair_bar, 64, gfail[g] == 0 && tc_wait(mma_done(s), ph))) break;
     tc_fence_after();
     if (leader) {
       // the next tile's products into the other buffer, once its copy has
@@ -212,71 +243,59 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     }
     __syncwarp();
 
-    // ---- row 32q + lane of the tile (tensor-memory lane), buffer s.  First
-    // Σ z² over all 128 columns, then, per column quarter b ∈ [8c, 8c + 8),
-    // the H_4 rows 2h + ab on packed pairs (coordinates 2j, 2j + 1) and their
-    // codes: word 4ab + c holds coordinates 32(2h + ab) + 8c + [0, 8)
-    const uint32_t tb = tmem + (uint32_t(32 * q) << 16) + uint32_t(s * 128);
+    // ---- y'[64h + c], c < 64, of tile row `row` (tensor-memory lane), buffer s
+    uint32_t v[4][16];
+    const uint32_t tb = tmem + (uint32_t(32 * q) << 16) + uint32_t(s * 128 + 64 * h);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_ld16(tb + uint32_t(16 * i), v[i]);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tmem_free(s));
     float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[2][16];
-      tmem_ld16(tb + uint32_t(32 * c), v[0]);
-      tmem_ld16(tb + uint32_t(32 * c + 16), v[1]);
-      tmem_ld_wait();
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float2 z0 = make_float2(__uint_as_float(v[0][2 * j]), __uint_as_float(v[0][2 * j + 1]));
-        const float2 z1 = make_float2(__uint_as_float(v[1][2 * j]), __uint_as_float(v[1][2 * j + 1]));
-        acc = fma2(z0, z0, acc);
-        acc2 = fma2(z1, z1, acc2);
+      for (int j = 0; j < 8; j += 2) {
+        const float2 a = make_float2(__uint_as_float(v[i][2 * j]), __uint_as_float(v[i][2 * j + 1]));
+        const float2 b = make_float2(__uint_as_float(v[i][2 * j + 2]), __uint_as_float(v[i][2 * j + 3]));
+        acc = fma2(a, a, acc);
+        acc2 = fma2(b, b, acc2);
       }
-    }
     const float2 qa = add2(acc, acc2);
-    const float nu = sqrtf(((qa.x + qa.y) * 4.f) * p.inv_d);  // ‖y'‖² = 4·Σ z² = d·‖x‖²
-    const float sc = nu > 0.f ? __fdiv_rn(num, nu) : 0.f;
+    float* ps = psum + (g * 2 + s) * 2 * L::TILE;
+    ps[h * L::TILE + row] = qa.x + qa.y;
+    bar_named(pair_bar, 64);
+    const float nu2 = (ps[row] + ps[L::TILE + row]) * p.inv_d;  // the same order in both halves
+    const float nu = sqrtf(nu2);
+    // 2^18/ν to a few ulp: moves I by a fraction of a unit, inside the decision band
+    const float sc = nu2 > 0.f ? num * rsqrtf(nu2) : 0.f;
     const float2 sc2 = make_float2(sc, sc);
-    const float2 hs2 = make_float2(hsign, hsign);
 
+    // codes: word w holds coordinates 64h + 8w + [0, 8)
     uint32_t words[8];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[NB][8];
+    for (int w = 0; w < 8; ++w) {
+      uint32_t cv[8];
 #pragma unroll
-      for (int a = 0; a < NB; ++a) tmem_ld8(tb + uint32_t(a * 32 + 8 * c), v[a]);
-      tmem_ld_wait();
-      if (c == 3) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tmem_free(s));
+      for (int t = 0; t < 4; ++t) {
+        const int c = 8 * w + 2 * t;
+        const float2 f = fma2(make_float2(__uint_as_float(v[c >> 4][c & 15]), __uint_as_float(v[c >> 4][(c & 15) + 1])),
+                              sc2, bias2);
+        const uint32_t fx = __float_as_uint(f.x), fy = __float_as_uint(f.y);
+        cv[2 * t] = fx + lds_u32(__byte_perm(fx, lane_word, 0x7624u));
+        cv[2 * t + 1] = fy + lds_u32(__byte_perm(fy, lane_word, 0x7624u));
       }
-#pragma unroll
-      for (int ab = 0; ab < 2; ++ab) {
-        uint32_t cv[8];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          float2 z[NB];
-#pragma unroll
-          for (int a = 0; a < NB; ++a) z[a] = make_float2(__uint_as_float(v[a][2 * t]), __uint_as_float(v[a][2 * t + 1]));
-          const float2 u = ab ? sub2(z[0], z[1]) : add2(z[0], z[1]);
-          const float2 w = ab ? sub2(z[2], z[3]) : add2(z[2], z[3]);
-          const float2 f = fma2(fma2(w, hs2, u), sc2, bias2);
-          const uint32_t fx = __float_as_uint(f.x), fy = __float_as_uint(f.y);
-          cv[2 * t] = fx + lds_u32(__byte_perm(fx, lane_word, 0x7624u));
-          cv[2 * t + 1] = fy + lds_u32(__byte_perm(fy, lane_word, 0x7624u));
-        }
-        // byte 2 of each cv is a code: gather the even and the odd coordinates'
-        const uint32_t ev =
-            __byte_perm(__byte_perm(cv[0], cv[2], 0x0062u), __byte_perm(cv[4], cv[6], 0x6200u), 0x7610u);
-        const uint32_t od =
-            __byte_perm(__byte_perm(cv[1], cv[3], 0x0062u), __byte_perm(cv[5], cv[7], 0x6200u), 0x7610u);
-        words[4 * ab + c] = ev + (od << 4);
-      }
+      // byte 2 of each cv is a code: gather the even and the odd coordinates'
+      const uint32_t ev =
+          __byte_perm(__byte_perm(cv[0], cv[2], 0x0062u), __byte_perm(cv[4], cv[6], 0x6200u), 0x7610u);
+      const uint32_t od =
+          __byte_perm(__byte_perm(cv[1], cv[3], 0x0062u), __byte_perm(cv[5], cv[7], 0x6200u), 0x7610u);
+      words[w] = ev + (od << 4);
     }
 
     const int64_t row0 = (t0 + k * tstride) * L::TILE + 32 * q;
-    const uint32_t tile = ctile0 + uint32_t(ct) * 1024;
-    if (lane == 0) bulk_wait_read_1();  // the store from this tile two tiles ago has read it
+    if (lane == 0) bulk_wait_read_all();  // the previous tile's store has read the code tile
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < 2; ++c)
@@ -290,7 +309,6 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
       tma_store_2d(&cmap, 32 * h, int(row0), tile);
       bulk_commit();
     }
-    ct ^= 1;
   }
   if (k < my_tiles) {
     // a wait gave up: the rest of this thread's rows get NaN norms
