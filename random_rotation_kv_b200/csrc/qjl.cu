@@ -34,6 +34,7 @@
 #include <cstring>
 
 #include "batch_kernels.cuh"
+#include "qjl_tc.cuh"
 #include "tcgen05.cuh"
 
 namespace rrq {
@@ -600,6 +601,10 @@ __global__ void __launch_bounds__(kQ2Threads, 1) qjl_batch_kernel(const __grid_c
 
 template <typename T, int B>
 cudaError_t launch_qjl_tb(const QjlArgs& a, cudaStream_t stream) {
+  if constexpr (Elem<T>::kBytes == 2) {
+    const cudaError_t e = launch_qjl_tc<T, B>(a.x, a.n, a.p, a.S, a.codes, a.norms, a.qbits, a.rnorm, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if constexpr (Elem<T>::kBytes == 2) {
     // the swizzled input boxes need a 1024-byte-aligned start of dynamic shared
     // memory, which follows from the per-block reservation before it

@@ -62,7 +62,8 @@ struct EncTc {
   }
 };
 
-constexpr uint32_t kTcWaitLimit = 1u << 24;  // try_wait polls before a wait gives up
+// Bounded wait: up to 2^24 polls of the phase (a few seconds in all).
+constexpr uint32_t kTcWaitLimit = 1u << 24;
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t i = 0; i < kTcWaitLimit; ++i)
