@@ -51,8 +51,14 @@ FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["random_rotation_kv_b200/csrc/rrq_device.cuh",
                   "random_rotation_kv_b200/csrc/quant_kernels.cuh",
                   "random_rotation_kv_b200/csrc/batch_kernels.cuh",
+                  "random_rotation_kv_b200/csrc/tc_encode.cuh",
+                  "random_rotation_kv_b200/csrc/tcgen05.cuh",
+                  "random_rotation_kv_b200/csrc/mma_encode.cuh",
+                  "random_rotation_kv_b200/csrc/mma_decode.cuh",
                   "random_rotation_kv_b200/csrc/tensor_map.h",
                   "random_rotation_kv_b200/csrc/rrq_params.h"]
+# the kernels the headline's two calls run on this workload (d = 128, 4-bit, fp16)
+ENCODE_KERNEL, DECODE_KERNEL = "encode_tc_kernel", "decode_mma_kernel"
 
 
 def workload_config(extra=None):
@@ -422,8 +428,8 @@ def run_gpu(args):
 
     if rank == 0:
         peak, peak_kind = peaks()
-        dom, dom_ms, dom_bytes = (("encode_batch_kernel", enc_avg, BYTES_PER_VEC_ENC) if enc_avg >= dec_avg
-                                  else ("decode_batch_kernel", dec_avg, BYTES_PER_VEC_DEC))
+        dom, dom_ms, dom_bytes = ((ENCODE_KERNEL, enc_avg, BYTES_PER_VEC_ENC) if enc_avg >= dec_avg
+                                  else (DECODE_KERNEL, dec_avg, BYTES_PER_VEC_DEC))
         achieved = dom_bytes * N_VEC / (dom_ms / 1e3) / 1e9
         traffic = recorded_traffic(dom)
         step_gbs = (BYTES_PER_VEC_ENC + BYTES_PER_VEC_DEC) * N_VEC / (ms_per_step / 1e3) / 1e9
@@ -645,6 +651,34 @@ def extra_kernels(torch, dev, flush, reps, peak, sel=None):
                                    "us": 1e3 * ms, "bytes": by, "gbs": by / ms / 1e6,
                                    "frac_of_hbm": by / ms / 1e6 / peak}
         del caches, kc, kn_, vc, vn_
+
+    # decode attention at the other shapes (the score kernel, then the fp32 value sums):
+    # random codes and log-normal norms of 131072 tokens x 8 kv heads; the bytes count
+    # the cache read once and the output, not the scores' round trip through the workspace
+    if want("attention_shapes"):
+        rows = w.x.shape[0] * 8
+        g = torch.Generator(device=dev).manual_seed(77)
+        lines = []
+        for d, kb, vb in ((128, 2, 2), (128, 3, 3), (64, 4, 4), (256, 4, 4)):
+            qd = torch.randn(32, d, device=dev, generator=g).half()
+            caches = []
+            for _ in range(2):
+                caches.append((torch.randint(0, 256, (rows, d * kb // 8), device=dev, generator=g, dtype=torch.uint8),
+                               torch.exp(torch.randn(rows, device=dev, generator=g) * 0.5) * 10,
+                               torch.randint(0, 256, (rows, d * vb // 8), device=dev, generator=g, dtype=torch.uint8),
+                               torch.exp(torch.randn(rows, device=dev, generator=g) * 0.5) * 10))
+            ao = torch.empty(32, d, dtype=torch.float32, device=dev)
+            ws = torch.zeros(B.rrq_attention_workspace_bytes(32, 8, d, w.x.shape[0], kb, vb), dtype=torch.uint8,
+                             device=dev)
+            ms = time_loop(torch, stream, lambda i: B.rrq_attention_decode(
+                qd, *caches[i % 2], 8, d, 42, 43, k_bits=kb, v_bits=vb, scale=d ** -0.5, out=ao, workspace=ws),
+                max(reps // 5, 5))
+            by = rows * (d * kb // 8 + 4 + d * vb // 8 + 4) + 32 * d * 4
+            lines.append({"d": d, "k_bits": kb, "v_bits": vb, "us": 1e3 * ms, "bytes": by,
+                          "gbs": by / ms / 1e6, "frac_of_hbm": by / ms / 1e6 / peak})
+            del caches, ws
+        out["attention_shapes"] = {"workload": "32 q heads over [131072 tokens x 8 kv heads], random codes",
+                                   "lines": lines}
 
         # unbiased scores on the same keys stored TurboQuant-style: 2-bit codes + QJL bits
     if want("qk_scores_qjl"):

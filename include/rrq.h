@@ -245,24 +245,28 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
  *     out[h]  = Σ_t p[h][t] · v̂_{t,g}          (v̂ as rrq_decode, V codebook and seed).
  * The values are summed in their rotated domain and rotated back once per head.
  *   q          [hq × d] fp16
- *   k_codes    [T·hkv × d/2] bytes (4-bit), row t·hkv + g;  k_norms [T·hkv] float
- *   v_codes    [T·hkv × d/2] bytes (4-bit);                 v_norms [T·hkv] float
- *   k_codebook, v_codebook: HOST float[16] or NULL (the default codebook)
+ *   k_codes    [T·hkv × d·k_bits/8] bytes, row t·hkv + g;  k_norms [T·hkv] float
+ *   v_codes    [T·hkv × d·v_bits/8] bytes;                 v_norms [T·hkv] float
+ *   k_codebook, v_codebook: HOST float[2^bits] or NULL (the default codebook)
  *   workspace  device scratch of workspace_bytes ≥ rrq_attention_workspace_bytes(
- *              hq, hkv, d, T), 256-byte aligned, owned by the caller, and ZERO before
- *              its first use: each call leaves its counters at zero again.  Calls
- *              that share a workspace must not overlap on the GPU.
+ *              hq, hkv, d, k_bits, v_bits, T), 256-byte aligned, owned by the caller,
+ *              and ZERO before its first use: each call leaves its counters at zero
+ *              again.  Calls that share a workspace must not overlap on the GPU.
  *   out        [hq × d] float (output)
- * d must be 128 and both codes 4-bit; hq a multiple of hkv with hq/hkv in
- * {1, 2, 4, 8}; T ≥ 1.  Scores as rrq_qk_scores (fp16 operands, fp32 sums);
- * softmax in fp32.  The value sums take fp16 levels and fp16 weights with fp32
- * accumulation; the weights are p·ν relative to the largest p·ν of the head
- * (exponent and log2 ν added before the one exponential), so any finite value
- * norm keeps its precision: per head the output is within 2e-3·Σ_t p_t·‖v̂_t‖ of
- * the exact softmax-weighted sum of the reconstructions.
+ * d ∈ {64, 128, 256, 512}, K and V codes of 1 to 4 bits; hq a multiple of hkv
+ * with hq/hkv in {1, 2, 4, 8} (at most 4 for d = 512); T ≥ 1.  Scores as
+ * rrq_qk_scores (fp16 operands, fp32 sums); softmax in fp32.  d = 128 with 4-bit
+ * K and V runs as one fused kernel whose value sums take fp16 levels and fp16
+ * weights with fp32 accumulation; the weights are p·ν relative to the largest
+ * p·ν of the head (exponent and log2 ν added before the one exponential), so any
+ * finite value norm keeps its precision.  Every other shape writes the scores
+ * to the workspace (hq × T floats) and sums the values in fp32.  Either way, per
+ * head the output is within 2e-3·Σ_t p_t·‖v̂_t‖ of the exact softmax-weighted sum
+ * of the reconstructions.
  * Errors: RRQ_ERR_INVALID (incl. a workspace that is too small), RRQ_ERR_UNSUPPORTED
- * (d, bits, group size, or a device whose per-block reserved shared memory is not
- * the 1 KB the kernel's shared layout assumes), RRQ_ERR_CUDA.
+ * (d, bits, group size; for d = 128 with 4-bit codes also a device whose
+ * per-block reserved shared memory is not the 1 KB the fused kernel's shared
+ * layout assumes), RRQ_ERR_CUDA.
  */
 int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
                          const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,
@@ -299,10 +303,13 @@ int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
 
 /*
  * rrq_attention_workspace_bytes — the workspace rrq_attention_decode needs for
- * (hq, hkv, d, T) on the current device (it depends on the SM count), or 0 for an
- * invalid shape.  No CUDA work beyond reading the device's attributes.
+ * (hq, hkv, d, k_bits, v_bits, T) on the current device (it depends on the SM
+ * count), or 0 for an invalid shape.  d = 128 with 4-bit K and V needs the
+ * counters and partial states only (well under 1 MB for 32 query heads); every
+ * other shape adds hq × T floats of scores.  No CUDA work beyond reading the
+ * device's attributes.
  */
-size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int64_t T);
+size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int k_bits, int v_bits, int64_t T);
 
 /*
  * rrq_q4_0_rot — "Attn-rot" (TurboQuant lite): rotate, then q4_0.

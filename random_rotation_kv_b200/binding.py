@@ -45,7 +45,7 @@ SIGNATURES = {
     "rrq_attention_decode": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _c_i64, _int, _int, _int,
                                     _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float, _vp,
                                     ctypes.c_size_t, _vp, _vp]),
-    "rrq_attention_workspace_bytes": (ctypes.c_size_t, [_int, _int, _int, _c_i64]),
+    "rrq_attention_workspace_bytes": (ctypes.c_size_t, [_int, _int, _int, _int, _int, _c_i64]),
     "rrq_attention_decode_noalloc": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _c_i64, _int, _int,
                                             _int, _c_u64, _vp, _int, _c_u64, _vp, ctypes.c_float,
                                             _vp, _vp]),
@@ -292,7 +292,7 @@ def rrq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.
                          k_codebook=None, v_codebook=None, scale: float = 1.0, out=None,
                          workspace=None):
     """One decode step of attention, out [hq, d] float32, of unrotated fp16 queries q [hq, d]
-    over a K/V cache of 4-bit codes + norms (rows t*hkv + g).
+    over a K/V cache of k_bits / v_bits codes + norms (rows t*hkv + g).
 
     ``workspace``: a uint8 device tensor of at least rrq_attention_workspace_bytes(...)
     bytes, zero before its first use (each call leaves it ready for the next); a zeroed
@@ -314,7 +314,7 @@ def rrq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.
     if out is None:
         out = torch.empty(hq, d, dtype=torch.float32, device=q.device)
     _dev_tensor(out, "out", (torch.float32,))
-    need = rrq_attention_workspace_bytes(hq, hkv, d, t_len)
+    need = rrq_attention_workspace_bytes(hq, hkv, d, t_len, k_bits, v_bits)
     if workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     _dev_tensor(workspace, "workspace", (torch.uint8,))
@@ -327,9 +327,10 @@ def rrq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.
     return out
 
 
-def rrq_attention_workspace_bytes(hq: int, hkv: int, d: int, t_len: int) -> int:
+def rrq_attention_workspace_bytes(hq: int, hkv: int, d: int, t_len: int, k_bits: int = 4,
+                                  v_bits: int = 4) -> int:
     """Workspace bytes rrq_attention_decode needs on the current device."""
-    return int(lib().rrq_attention_workspace_bytes(hq, hkv, d, t_len))
+    return int(lib().rrq_attention_workspace_bytes(hq, hkv, d, k_bits, v_bits, t_len))
 
 
 def rrq_q4_0_rot(x: torch.Tensor, seed: int, rotate: bool = True, out=None):

@@ -265,12 +265,17 @@ int rrq_qk_scores_qjl(const void* q, int hq, const uint8_t* codes, const float* 
   return status_of(rrq::launch_qk_scores_qjl(a, as_stream(stream)));
 }
 
-int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
-                                 const float* k_norms, const uint8_t* v_codes,
-                                 const float* v_norms, int64_t T, int hkv, int d, int k_bits,
-                                 uint64_t k_seed, const float* k_codebook, int v_bits,
-                                 uint64_t v_seed, const float* v_codebook, float scale,
-                                 float* out, void* stream) {
+namespace {
+// Whether the fused kernel (d = 128, 4-bit K and V) serves the shape.
+bool attention_fused(int d, int k_bits, int v_bits) { return d == 128 && k_bits == 4 && v_bits == 4; }
+size_t attention_ws(int hq, int hkv, int d, int k_bits, int v_bits, int64_t T) {
+  return attention_fused(d, k_bits, v_bits) ? rrq::attention_workspace_bytes(hq, hkv, T)
+                                            : rrq::attention_general_workspace_bytes(hq, hkv, d, T);
+}
+// Validation shared by the two attention entries: RRQ_OK, or the status to return.
+int attention_check(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
+                    const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d, int k_bits,
+                    int v_bits, float scale, const float* out) {
   if (T < 1 || !d_ok(d) || !bits_ok(k_bits) || !bits_ok(v_bits) || hq < 1 || hkv < 1 ||
       hq % hkv != 0 || !std::isfinite(scale))
     return RRQ_ERR_INVALID;
@@ -279,15 +284,69 @@ int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
       !arr_ok(v_norms, T, 4))
     return RRQ_ERR_INVALID;
   const int group = hq / hkv;
-  if (d != 128 || k_bits != 4 || v_bits != 4 ||
-      (group != 1 && group != 2 && group != 4 && group != 8))
+  if (group != 1 && group != 2 && group != 4 && group != 8) return RRQ_ERR_UNSUPPORTED;
+  if (!attention_fused(d, k_bits, v_bits) && !rrq::attention_general_supported(d, k_bits, hq, hkv))
     return RRQ_ERR_UNSUPPORTED;
-  if (rrq::attention_workspace_bytes(hq, hkv, T) > rrq::kAttentionScratchBytes)
-    return RRQ_ERR_SCRATCH;
-  rrq::AttnArgs a;
-  if (make_params(k_bits, k_codebook, k_seed, d, &a.pk) != RRQ_OK ||
-      make_params(v_bits, v_codebook, v_seed, d, &a.pv) != RRQ_OK)
+  return RRQ_OK;
+}
+// The general path's launch with its workspace (counters zero on entry).
+int attention_general(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
+                      const uint8_t* v_codes, const float* v_norms, int64_t T, int hkv, int d,
+                      const rrq::QuantParams& pk, const rrq::QuantParams& pv, float scale, void* workspace,
+                      float* out, cudaStream_t stream) {
+  rrq::AttnGenArgs g;
+  g.q = q;
+  g.k_codes = k_codes;
+  g.k_norms = k_norms;
+  g.v_codes = v_codes;
+  g.v_norms = v_norms;
+  g.out = out;
+  g.T = T;
+  g.hq = hq;
+  g.hkv = hkv;
+  g.group = hq / hkv;
+  g.d = d;
+  g.scale = scale;
+  g.pk = pk;
+  g.pv = pv;
+  const cudaError_t e = rrq::launch_attention_general(g, workspace, stream);
+  return e == cudaErrorNotSupported ? RRQ_ERR_UNSUPPORTED : status_of(e);
+}
+}  // namespace
+
+size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int k_bits, int v_bits, int64_t T) {
+  if (T < 1 || !d_ok(d) || !bits_ok(k_bits) || !bits_ok(v_bits) || hq < 1 || hkv < 1 || hq % hkv != 0)
+    return 0;
+  return attention_ws(hq, hkv, d, k_bits, v_bits, T);
+}
+
+int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
+                                 const float* k_norms, const uint8_t* v_codes,
+                                 const float* v_norms, int64_t T, int hkv, int d, int k_bits,
+                                 uint64_t k_seed, const float* k_codebook, int v_bits,
+                                 uint64_t v_seed, const float* v_codebook, float scale,
+                                 float* out, void* stream) {
+  const int chk = attention_check(q, hq, k_codes, k_norms, v_codes, v_norms, T, hkv, d, k_bits, v_bits,
+                                  scale, out);
+  if (chk != RRQ_OK) return chk;
+  if (attention_ws(hq, hkv, d, k_bits, v_bits, T) > rrq::kAttentionScratchBytes) return RRQ_ERR_SCRATCH;
+  rrq::QuantParams pk, pv;
+  if (make_params(k_bits, k_codebook, k_seed, d, &pk) != RRQ_OK ||
+      make_params(v_bits, v_codebook, v_seed, d, &pv) != RRQ_OK)
     return RRQ_ERR_INVALID;
+  if (!attention_fused(d, k_bits, v_bits)) {
+    void* base = nullptr;
+    cudaError_t e = rrq::attention_scratch(&base);
+    if (e != cudaSuccess) return status_of(e);
+    // the counters must start at zero; the rest is overwritten before it is read
+    e = cudaMemsetAsync(base, 0, (size_t(hkv) * 4 + 255) / 256 * 256, as_stream(stream));
+    if (e != cudaSuccess) return status_of(e);
+    return attention_general(q, hq, k_codes, k_norms, v_codes, v_norms, T, hkv, d, pk, pv, scale, base, out,
+                             as_stream(stream));
+  }
+  rrq::AttnArgs a;
+  a.pk = pk;
+  a.pv = pv;
   a.q = static_cast<const __half*>(q);
   a.k_codes = k_codes;
   a.k_norms = k_norms;
@@ -297,16 +356,11 @@ int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
   a.T = T;
   a.hq = hq;
   a.hkv = hkv;
-  a.group = group;
-  a.splits = rrq::attention_splits(hkv, group, T);
+  a.group = hq / hkv;
+  a.splits = rrq::attention_splits(hkv, a.group, T);
   a.scale = scale;
   const cudaError_t e = rrq::launch_attention_decode_in_scratch(a, as_stream(stream));
   return e == cudaErrorNotSupported ? RRQ_ERR_UNSUPPORTED : status_of(e);
-}
-
-size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int64_t T) {
-  if (T < 1 || !d_ok(d) || hq < 1 || hkv < 1 || hq % hkv != 0) return 0;
-  return rrq::attention_workspace_bytes(hq, hkv, T);
 }
 
 int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,
@@ -314,24 +368,22 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
                          int k_bits, uint64_t k_seed, const float* k_codebook, int v_bits,
                          uint64_t v_seed, const float* v_codebook, float scale, void* workspace,
                          size_t workspace_bytes, float* out, void* stream) {
-  if (T < 1 || !d_ok(d) || !bits_ok(k_bits) || !bits_ok(v_bits) || hq < 1 || hkv < 1 ||
-      hq % hkv != 0 || !std::isfinite(scale))
-    return RRQ_ERR_INVALID;
-  if (q == nullptr || !aligned(q, 16) || out == nullptr || !aligned(out, 16)) return RRQ_ERR_INVALID;
-  if (!arr_ok(k_codes, T, 16) || !arr_ok(k_norms, T, 4) || !arr_ok(v_codes, T, 16) ||
-      !arr_ok(v_norms, T, 4))
-    return RRQ_ERR_INVALID;
-  const int group = hq / hkv;
-  if (d != 128 || k_bits != 4 || v_bits != 4 ||
-      (group != 1 && group != 2 && group != 4 && group != 8))
-    return RRQ_ERR_UNSUPPORTED;
+  const int chk = attention_check(q, hq, k_codes, k_norms, v_codes, v_norms, T, hkv, d, k_bits, v_bits,
+                                  scale, out);
+  if (chk != RRQ_OK) return chk;
   if (workspace == nullptr || !aligned(workspace, 256) ||
-      workspace_bytes < rrq::attention_workspace_bytes(hq, hkv, T))
+      workspace_bytes < attention_ws(hq, hkv, d, k_bits, v_bits, T))
     return RRQ_ERR_INVALID;
+  rrq::QuantParams pk, pv;
+  if (make_params(k_bits, k_codebook, k_seed, d, &pk) != RRQ_OK ||
+      make_params(v_bits, v_codebook, v_seed, d, &pv) != RRQ_OK)
+    return RRQ_ERR_INVALID;
+  if (!attention_fused(d, k_bits, v_bits))
+    return attention_general(q, hq, k_codes, k_norms, v_codes, v_norms, T, hkv, d, pk, pv, scale, workspace,
+                             out, as_stream(stream));
   rrq::AttnArgs a;
-  if (make_params(k_bits, k_codebook, k_seed, d, &a.pk) != RRQ_OK ||
-      make_params(v_bits, v_codebook, v_seed, d, &a.pv) != RRQ_OK)
-    return RRQ_ERR_INVALID;
+  a.pk = pk;
+  a.pv = pv;
   a.q = static_cast<const __half*>(q);
   a.k_codes = k_codes;
   a.k_norms = k_norms;
@@ -341,8 +393,8 @@ int rrq_attention_decode(const void* q, int hq, const uint8_t* k_codes, const fl
   a.T = T;
   a.hq = hq;
   a.hkv = hkv;
-  a.group = group;
-  a.splits = rrq::attention_splits(hkv, group, T);
+  a.group = hq / hkv;
+  a.splits = rrq::attention_splits(hkv, a.group, T);
   a.scale = scale;
   a.counters = static_cast<unsigned*>(workspace);
   a.states = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +

@@ -40,5 +40,33 @@ cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);
 // checked attention_workspace_bytes(...) ≤ kAttentionScratchBytes.
 constexpr size_t kAttentionScratchBytes = size_t(4) << 20;
 cudaError_t launch_attention_decode_in_scratch(AttnArgs a, cudaStream_t stream);
+// That array's address on the current device (looked up once per device).
+cudaError_t attention_scratch(void** addr);
+
+// ---- every other shape (attention_gen.cu): d ∈ {64, 128, 256, 512}, 1- to 4-bit
+// K and V codes, group ∈ {1, 2, 4, 8} (d = 512 with group ≤ 4), K widths the
+// score kernel takes.  The scores go to the workspace first.
+struct AttnGenArgs {
+  const void* q;            // [hq × d] fp16 query heads (unrotated)
+  const uint8_t* k_codes;   // [T·hkv × d·kb/8], row t·hkv + g
+  const float* k_norms;     // [T·hkv]
+  const uint8_t* v_codes;   // [T·hkv × d·vb/8]
+  const float* v_norms;     // [T·hkv]
+  float* out;               // [hq × d]
+  unsigned* counters;       // set by launch_attention_general
+  float* states;            // set by launch_attention_general
+  float* scores;            // set by launch_attention_general
+  int64_t T;
+  int hq, hkv, group, splits, d;
+  float scale;
+  QuantParams pk, pv;
+};
+bool attention_general_supported(int d, int k_bits, int hq, int hkv);
+int attention_general_splits(int hkv, int group, int d, int64_t T);
+// counters (256-byte padded), partial states, then hq × T fp32 scores
+size_t attention_general_workspace_bytes(int hq, int hkv, int d, int64_t T);
+// Asynchronous on `stream`: the score launch, then the value launch.  The
+// workspace's counters are zero before the call and after it.
+cudaError_t launch_attention_general(AttnGenArgs a, void* workspace, cudaStream_t stream);
 
 }  // namespace rrq

@@ -118,14 +118,22 @@ def test_other_entry_points_validate():
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 96, 0, 1, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot(P, B.RRQ_F16, 4, 128, 0, 3, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_q4_0_rot_decode(P, 4, 128, 0, 1, P, 5, None) == B.RRQ_ERR_INVALID
-    # attention: 4-bit codes and d = 128 only; T must be at least 1; a big enough workspace
-    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 128, 2, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_UNSUPPORTED
-    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 64, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_UNSUPPORTED
+    # attention: group sizes 1, 2, 4, 8 (at most 4 at d = 512); T must be at least 1;
+    # a big enough workspace (every call here is refused before any launch)
+    assert lib.rrq_attention_decode(P, 24, P, P, P, P, 16, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_UNSUPPORTED
+    assert lib.rrq_attention_decode(P, 64, P, P, P, P, 16, 8, 512, 2, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_UNSUPPORTED
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 96, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 128, 5, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_INVALID
+    assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 64, 2, 0, None, 3, 1, None, 1.0, P, 64, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_attention_decode(P, 32, P, P, P, P, 0, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_attention_decode(P, 32, P, P, P_MIS, P, 16, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 1 << 30, P, None) == B.RRQ_ERR_INVALID
     assert lib.rrq_attention_decode(P, 32, P, P, P, P, 16, 8, 128, 4, 0, None, 4, 1, None, 1.0, P, 16, P, None) == B.RRQ_ERR_INVALID
-    assert lib.rrq_attention_workspace_bytes(32, 8, 128, 1 << 17) > 0
-    assert lib.rrq_attention_workspace_bytes(30, 8, 128, 16) == 0
+    assert lib.rrq_attention_workspace_bytes(32, 8, 128, 4, 4, 1 << 17) > 0
+    assert lib.rrq_attention_workspace_bytes(30, 8, 128, 4, 4, 16) == 0
+    assert lib.rrq_attention_workspace_bytes(32, 8, 128, 4, 0, 16) == 0
+    # the fused shape needs no score buffer; every other shape does (hq × T floats)
+    assert lib.rrq_attention_workspace_bytes(32, 8, 128, 2, 2, 1 << 17) >= 32 * (1 << 17) * 4
+    assert lib.rrq_attention_workspace_bytes(32, 8, 128, 4, 4, 1 << 17) < 32 * (1 << 17) * 4
     # unbiased scores: d other than 128 and odd group sizes are unsupported; S must be given
     assert lib.rrq_qk_scores_qjl(P, 32, P, P, P, P, P, 16, 8, 64, 2, 0, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
     assert lib.rrq_qk_scores_qjl(P, 48, P, P, P, P, P, 16, 3, 128, 2, 0, None, 1.0, P, None) == B.RRQ_ERR_UNSUPPORTED
@@ -158,10 +166,32 @@ def test_attention_splits_fill_the_sms_in_one_wave(hq, hkv):
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
     counters = (hkv * 4 + 255) // 256 * 256
     for t_len in (1, 100, 4096, 1 << 17, 1 << 20):
-        ws = lib.rrq_attention_workspace_bytes(hq, hkv, 128, t_len)
+        ws = lib.rrq_attention_workspace_bytes(hq, hkv, 128, 4, 4, t_len)
         per_range = hq * 131 * 4
         assert (ws - counters) % per_range == 0
         s = (ws - counters) // per_range
         ntile = (t_len + 31) // 32
         assert s == max(1, min(sms // hkv, (ntile + 11) // 12))
         assert s * hkv <= max(sms, hkv)
+
+
+@pytest.mark.parametrize("hq,hkv,d", [(32, 8, 64), (32, 8, 256), (8, 1, 512), (64, 8, 128)])
+def test_general_attention_workspace(hq, hkv, d):
+    """Shapes other than d = 128 with 4-bit K and V: counters (256-byte padded), the
+    ranges' partial states (hq × ranges × (d + 2) floats, 256-byte padded), then the
+    scores (hq × T floats); as many CTAs as the SMs hold at once (one or two each, by
+    the value kernel's occupancy: one when no device is visible), at most 296 ranges
+    per kv head, at least 32 tokens per range, at least one range."""
+    import torch
+    lib = B.lib()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    counters = (hkv * 4 + 255) // 256 * 256
+    for t_len in (1, 100, 4096, 1 << 17):
+        ws = lib.rrq_attention_workspace_bytes(hq, hkv, d, 2, 3, t_len)
+        sizes = []
+        for per_sm in (1, 2):
+            s = max(1, min(per_sm * sms // hkv, 296, (t_len + 31) // 32))
+            sizes.append(counters + (hq * s * (d + 2) * 4 + 255) // 256 * 256 + hq * t_len * 4)
+        assert ws in sizes, (ws, sizes)
+        if not torch.cuda.is_available():
+            assert ws == sizes[0]

@@ -70,6 +70,33 @@ def test_attention_parity_on_oracle_encoded_cache(hq, hkv, t_len):
     _check(q, kp, kn, vp, vn, t_len, hkv, 42, 43, 1.0 / math.sqrt(D), f"hq={hq} hkv={hkv} T={t_len}")
 
 
+@pytest.mark.parametrize("d,kb,vb", [(128, 2, 2), (128, 3, 3), (64, 4, 4), (256, 4, 4), (128, 4, 2),
+                                     (64, 1, 3), (512, 2, 4), (256, 3, 1)])
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (4, 1), (16, 2)])
+@pytest.mark.parametrize("t_len", [1, 37, 2000])
+def test_attention_general_shapes(d, kb, vb, hq, hkv, t_len):
+    """Every shape other than d = 128 with 4-bit K and V (the scores through the score
+    kernel into the workspace, then the fp32 value sums): the same per-head bound."""
+    if d == 512 and hq // hkv == 8:
+        pytest.skip("d = 512 takes groups of at most 4")
+    rg = np.random.Generator(np.random.PCG64(d * 100 + kb * 10 + vb + hq + 7 * t_len))
+    kp, kn, vp, vn = _cache(rg, t_len, hkv, 42, 43, d, kb, vb)
+    q = rg.standard_normal((hq, d)).astype(np.float16)
+    _check(q, kp, kn, vp, vn, t_len, hkv, 42, 43, 1.0 / math.sqrt(d), f"d={d} b={kb}/{vb} hq={hq} hkv={hkv} T={t_len}",
+           d, kb, vb)
+
+
+def test_attention_general_value_norm_range():
+    """The general path sums in fp32: value norms from 1e-30 to 1e30 keep the bound."""
+    rg = np.random.Generator(np.random.PCG64(71))
+    hq, hkv, t_len, d = 8, 2, 500, 64
+    kp, kn, vp, vn = _cache(rg, t_len, hkv, 42, 43, d, 2, 3)
+    q = rg.standard_normal((hq, d)).astype(np.float16)
+    for v_scale in (1e-30, 1e30):
+        vs = (vn * v_scale * np.exp(rg.standard_normal(vn.shape))).astype(np.float32)
+        _check(q, kp, kn, vp, vs, t_len, hkv, 42, 43, 0.125, f"general v scale {v_scale}", d, 2, 3)
+
+
 def test_attention_special_cases():
     """One token returns its value; a zero query averages the values; a large scale
     picks the top-scoring token's value.  Each is held to the reconstruction

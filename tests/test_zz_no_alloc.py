@@ -34,12 +34,12 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _noalloc(q, kc, kn, vc, vn, hkv, out, scale):
+def _noalloc(q, kc, kn, vc, vn, hkv, out, scale, d=D, kb=4, vb=4):
     hq = q.shape[0]
     t_len = kn.numel() // hkv
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return B.lib().rrq_attention_decode_noalloc(
-        _ptr(q), hq, _ptr(kc), _ptr(kn), _ptr(vc), _ptr(vn), t_len, hkv, D, 4, 42, None, 4, 43,
+        _ptr(q), hq, _ptr(kc), _ptr(kn), _ptr(vc), _ptr(vn), t_len, hkv, d, kb, 42, None, vb, 43,
         None, ctypes.c_float(scale), _ptr(out), stream)
 
 
@@ -65,6 +65,28 @@ def test_noalloc_attention_matches_the_workspace_entry_twice():
         torch.cuda.synchronize()
         err = torch.linalg.norm((out - ref).double(), dim=1)
         assert torch.all(err <= bound), float(err.max())
+
+
+def test_noalloc_attention_other_shapes_twice():
+    """d = 64 with 2-bit K and 3-bit V (the scores go to the scratch array too)."""
+    rg = np.random.Generator(np.random.PCG64(2025))
+    t_len, hkv, hq, d = 3000, 4, 16, 64
+    rows = t_len * hkv
+    kc = torch.from_numpy(rg.integers(0, 256, size=(rows, d * 2 // 8), dtype=np.uint8)).to(DEV)
+    vc = torch.from_numpy(rg.integers(0, 256, size=(rows, d * 3 // 8), dtype=np.uint8)).to(DEV)
+    kn = torch.from_numpy((np.exp(rg.standard_normal(rows) * 0.5) * 8.0).astype(np.float32)).to(DEV)
+    vn = torch.from_numpy((np.exp(rg.standard_normal(rows) * 0.5) * 6.0).astype(np.float32)).to(DEV)
+    q = torch.from_numpy(rg.standard_normal((hq, d)).astype(np.float16)).to(DEV)
+    assert B.rrq_attention_workspace_bytes(hq, hkv, d, t_len, 2, 3) <= 4 << 20
+    host = [t.cpu().numpy() for t in (q, kc, kn, vc, vn)]
+    ref, p = oatt.decode_attention(*host, t_len, hkv, d, 2, 3, 42, 43, scale=0.125, return_weights=True)
+    bound = weighted_bound(p, host[3], host[4], t_len, hkv, d, 3, 43)
+    for _ in range(2):
+        out = torch.full((hq, d), float("nan"), dtype=torch.float32, device=DEV)
+        assert _noalloc(q, kc, kn, vc, vn, hkv, out, 0.125, d, 2, 3) == B.RRQ_OK
+        torch.cuda.synchronize()
+        err = np.linalg.norm(out.cpu().numpy().astype(np.float64) - ref, axis=1)
+        assert np.all(err <= bound), float(np.max(err / bound))
 
 
 def test_noalloc_attention_refuses_requests_beyond_its_scratch():
