@@ -270,7 +270,7 @@ namespace {
 bool attention_fused(int d, int k_bits, int v_bits) { return d == 128 && k_bits == 4 && v_bits == 4; }
 size_t attention_ws(int hq, int hkv, int d, int k_bits, int v_bits, int64_t T) {
   return attention_fused(d, k_bits, v_bits) ? rrq::attention_workspace_bytes(hq, hkv, T)
-                                            : rrq::attention_general_workspace_bytes(hq, hkv, d, T);
+                                            : rrq::attention_general_workspace_bytes(hq, hkv, d, v_bits, T);
 }
 // Validation shared by the two attention entries: RRQ_OK, or the status to return.
 int attention_check(const void* q, int hq, const uint8_t* k_codes, const float* k_norms,

@@ -62,9 +62,9 @@ struct AttnGenArgs {
   QuantParams pk, pv;
 };
 bool attention_general_supported(int d, int k_bits, int hq, int hkv);
-int attention_general_splits(int hkv, int group, int d, int64_t T);
+int attention_general_splits(int hkv, int group, int d, int v_bits, int64_t T);
 // counters (256-byte padded), partial states, then hq × T fp32 scores
-size_t attention_general_workspace_bytes(int hq, int hkv, int d, int64_t T);
+size_t attention_general_workspace_bytes(int hq, int hkv, int d, int v_bits, int64_t T);
 // Asynchronous on `stream`: the score launch, then the value launch.  The
 // workspace's counters are zero before the call and after it.
 cudaError_t launch_attention_general(AttnGenArgs a, void* workspace, cudaStream_t stream);

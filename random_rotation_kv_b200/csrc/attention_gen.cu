@@ -15,11 +15,14 @@
 // tiles on the packed K codes, every d and bit width), written to the
 // workspace.  Then one CTA per (kv head, token range): the range's per-head
 // maximum of the scores; each warp walks its tokens in batches of 32 (lane j
-// computes token j's weights e^{s − m}·ν for the group's heads), lane l owning
-// coordinates [l·d/32, (l + 1)·d/32) of every row — it reads the 32-bit words
-// that hold its b·d/32 code bits (a batch's 32 rows in flight at once), takes each
-// level from the lane that holds it (one shuffle) and each weight from the
-// token's lane, and adds w·c into its fp32 sums; warps meet through shared-memory atomics, the CTA writes its state
+// computes token j's weights e^{s − m}·ν for the group's heads and puts them in
+// the warp's shared-memory buffer), lane l owning coordinates [l·d/32,
+// (l + 1)·d/32) of every row — it reads the 32-bit words that hold its b·d/32
+// code bits (the loads of 32 rows, 16 for wide 3-bit rows, issued before any is
+// used, no branch between them), takes each level from the lane that holds it
+// (one shuffle) and each row's weights from the buffer (one broadcast read), and
+// adds w·c into its fp32 sums; the bit width is a template parameter, so every
+// shift is a constant.  Warps meet through shared-memory atomics, the CTA writes its state
 // (m, Σ e^{s−m}, d sums per head) to the workspace and counts itself in its kv
 // head's counter; the CTA that counts last merges the ranges, applies D·H (a
 // shared-memory Walsh–Hadamard transform per head), writes the output and sets
@@ -35,28 +38,31 @@ namespace {
 
 constexpr int kGWarps = 8;
 constexpr int kGThreads = kGWarps * 32;
-constexpr int kGMaxSplits = 296;  // token ranges per kv head: at most two CTAs per SM in all
+constexpr int kGMaxSplits = 444;  // token ranges per kv head: at most three CTAs per SM in all
 
-// The lane's b·CPL code bits of row `row` (bit i of the row = bit i mod 8 of byte
-// i / 8, coordinate j at bits [j·b, (j + 1)·b)), as the low bits of a 64-bit word.
-template <int CPL>
-__device__ __forceinline__ uint64_t lane_bits(const uint8_t* __restrict__ row, int lane, int b) {
-  const int start = lane * CPL * b;            // first bit of the lane
-  const int w0 = start >> 5, off = start & 31;  // its 32-bit word and the offset in it
-  const int nbits = CPL * b;                    // ≤ 64
-  const uint32_t* rw = reinterpret_cast<const uint32_t*>(row);
-  uint64_t v = __ldg(rw + w0);
-  if (off + nbits > 32) v |= uint64_t(__ldg(rw + w0 + 1)) << 32;
-  v >>= off;
-  if (off + nbits > 64) v |= uint64_t(__ldg(rw + w0 + 2)) << (64 - off);
-  return v;
-}
+// Words of a V row that lane `lane` reads: its B·CPL code bits start at bit
+// lane·B·CPL of the row (bit i of the row = bit i mod 8 of byte i / 8,
+// coordinate j at bits [j·B, (j + 1)·B)).  kWin words hold them once shifted
+// down by `off`; a 3-bit lane's bits may start inside a word and end inside the
+// next, so it reads one word more, the word index kept inside the row (a word
+// past the lane's bits only fills bits above them).
+// Rows whose loads are in flight together: 32, or 16 where the words of 32 rows
+// and the G × CPL sums would not fit the 128 registers of two CTAs per SM.
+template <int G, int B, int CPL> struct VRow {
+  static constexpr int kRowWords = B * CPL;                 // 32-bit words of a row
+  static constexpr int kWin = (B * CPL + 31) / 32;          // words of the lane's bits
+  static constexpr int kNW = kWin + (B == 3 ? 1 : 0);       // words read per row
+  static constexpr int kRows = kNW == 1 && G * CPL <= 32 ? 32 : 16;
+};
 
-template <int G, int CPL>
+template <int G, int CPL, int B>
 __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGenArgs a) {
+  using R = VRow<G, B, CPL>;
   constexpr int D = 32 * CPL;
   __shared__ float s_acc[G * D];     // the CTA's sums, then the merged sums
+  __shared__ __align__(16) float s_w[kGWarps][32][G];  // a warp's batch of weights, token-major
   __shared__ float s_max[kGWarps][G];
+  __shared__ float s_f[kGMaxSplits * G];  // the merge's per-range maxima, then factors
   __shared__ float s_m[G], s_l[G];
   __shared__ int s_last;
   pdl_release();
@@ -65,7 +71,6 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
   const int g = blockIdx.x / a.splits, r = blockIdx.x % a.splits;
   const int64_t per = (a.T + a.splits - 1) / a.splits;
   const int64_t t0 = int64_t(r) * per, t1 = t0 + per < a.T ? t0 + per : a.T;
-  const int bv = a.pv.bits;
   const float* sc = a.scores + int64_t(g) * G * a.T;  // [G][T] of this kv head's heads
   for (int i = tid; i < G * D; i += kGThreads) s_acc[i] = 0.f;
   if (tid < G) s_l[tid] = 0.f;
@@ -92,9 +97,16 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
   for (int h = 0; h < G; ++h) mh[h] = s_m[h];
 
   // ---- Σ_t e^{s − m}·ν·c over the warp's tokens, coordinates [lane·CPL, +CPL)
-  const float lev = a.pv.levels[lane & 15];  // lane i < 2^b holds level i
-  const uint64_t mask = (uint64_t(1) << bv) - 1;
-  const int64_t rowbytes = int64_t(D) * bv / 8;
+  // Lane i holds level i mod 2^B, so a shuffle whose source lane has the code in
+  // its low B bits (whatever lies above them) fetches that code's level.
+  const float lev = a.pv.levels[lane & ((1 << B) - 1)];
+  const int bit0 = lane * B * CPL;
+  const int w0 = bit0 >> 5, off = bit0 & 31;
+  int wo[R::kNW];  // the lane's word offsets within a row
+#pragma unroll
+  for (int k = 0; k < R::kNW; ++k) wo[k] = (w0 + k < R::kRowWords ? w0 + k : R::kRowWords - 1);
+  const int stride = a.hkv * R::kRowWords;  // words from one token's row to the next
+  const uint32_t* vrows = reinterpret_cast<const uint32_t*>(a.v_codes) + int64_t(g) * R::kRowWords;
   float acc[G][CPL];
   float lsum[G];
 #pragma unroll
@@ -103,9 +115,10 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
 #pragma unroll
     for (int j = 0; j < CPL; ++j) acc[h][j] = 0.f;
   }
-  // batches of 32 tokens per warp: lane j takes token j's scores and norm (coalesced)
-  // and every lane its code bits of all 32 rows, all loads of a batch issued
-  // before any of them is used
+  // batches of 32 tokens per warp: lane j takes token j's scores and norm
+  // (coalesced) and puts its weights in the warp's buffer; every lane reads its
+  // words of the batch's rows, all loads of a group of rows issued before any of
+  // them is used.  Rows past the range's end repeat its last row with weight 0.
   for (int64_t tb = t0 + int64_t(warp) * 32; tb < t1; tb += int64_t(kGWarps) * 32) {
     const int nt = int(t1 - tb < 32 ? t1 - tb : 32);
     const bool mine = lane < nt;
@@ -114,10 +127,7 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
 #pragma unroll
     for (int h = 0; h < G; ++h) sv[h] = mine ? sc[int64_t(h) * a.T + t] : -INFINITY;
     const float nu = mine ? __ldg(a.v_norms + t * a.hkv + g) : 0.f;
-    uint64_t cw[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      cw[j] = j < nt ? lane_bits<CPL>(a.v_codes + ((tb + j) * a.hkv + g) * rowbytes, lane, bv) : 0;
+    const uint32_t* rows = vrows + tb * stride;
     float wl[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -126,18 +136,42 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
       wl[h] *= nu;
     }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j >= nt) break;
-      float w[G];
+    for (int h = 0; h < G; ++h) s_w[warp][lane][h] = wl[h];
+    __syncwarp();
 #pragma unroll
-      for (int h = 0; h < G; ++h) w[h] = __shfl_sync(kFull, wl[h], j);
+    for (int j0 = 0; j0 < 32; j0 += R::kRows) {
+      uint32_t cw[R::kRows][R::kNW];
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        const float lv = __shfl_sync(kFull, lev, int((cw[j] >> (c * bv)) & mask));
+      for (int j = 0; j < R::kRows; ++j) {
+        const int row = j0 + j < nt ? j0 + j : nt - 1;
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[h][c] = fmaf(w[h], lv, acc[h][c]);
+        for (int k = 0; k < R::kNW; ++k) cw[j][k] = __ldg(rows + row * stride + wo[k]);
+      }
+#pragma unroll
+      for (int j = 0; j < R::kRows; ++j) {
+        float w[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) w[h] = s_w[warp][j0 + j][h];
+        uint32_t u[R::kWin + 1];  // the lane's bits from bit 0 on
+#pragma unroll
+        for (int k = 0; k < R::kWin; ++k) {
+          if constexpr (B == 3) u[k] = __funnelshift_r(cw[j][k], cw[j][k + 1], off);
+          else if constexpr (R::kWin == 1) u[k] = cw[j][0] >> off;
+          else u[k] = cw[j][k];  // B·CPL ≥ 32: the lane's bits start at a word
+        }
+        u[R::kWin] = 0u;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          constexpr int kB = B;
+          const int bit = c * kB, k = bit >> 5, sh = bit & 31;
+          const uint32_t code = sh + kB > 32 ? __funnelshift_r(u[k], u[k + 1], sh) : u[k] >> sh;
+          const float lv = __shfl_sync(kFull, lev, int(code));  // lane = code mod 32
+#pragma unroll
+          for (int h = 0; h < G; ++h) acc[h][c] = fmaf(w[h], lv, acc[h][c]);
+        }
       }
     }
+    __syncwarp();  // the buffer is rewritten by the next batch
   }
   // the lanes' shares of the softmax sums
 #pragma unroll
@@ -163,30 +197,36 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
   if (!s_last) return;
   __threadfence();
 
-  // ---- the last range of kv head g: merge the ranges' states
-  const float* st0 = a.states + int64_t(g) * a.splits * G * (D + 2);
-  if (tid < G) {
+  // ---- the last range of kv head g: merge the ranges' states, in three short
+  // passes over shared memory and one over the states: every state's maxima,
+  // the heads' maxima (warp h reduces head h), the factors e^{m_q − m}; then each
+  // thread's sums (and the denominators) as batches of independent loads
+  const int S = a.splits;
+  const int64_t sstride = int64_t(G) * (D + 2);
+  const float* st0 = a.states + int64_t(g) * S * sstride;
+  for (int i = tid; i < S * G; i += kGThreads) s_f[i] = __ldcg(st0 + (i / G) * sstride + i % G);
+  __syncthreads();
+  if (warp < G) {
     float m = -INFINITY;
-    for (int q = 0; q < a.splits; ++q) m = fmaxf(m, __ldcg(st0 + int64_t(q) * G * (D + 2) + tid));
-    float l = 0.f;
-    for (int q = 0; q < a.splits; ++q) {
-      const float* sq = st0 + int64_t(q) * G * (D + 2);
-      const float mq = __ldcg(sq + tid);
-      if (mq != -INFINITY) l += __ldcg(sq + G + tid) * __expf(mq - m);
-    }
-    s_m[tid] = m;
-    s_l[tid] = l;
+    for (int q = lane; q < S; q += 32) m = fmaxf(m, s_f[q * G + warp]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+    if (lane == 0) s_m[warp] = m;
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += kGThreads) {
-    const int h = i / D;
+  for (int i = tid; i < S * G; i += kGThreads) {
+    const float mq = s_f[i];
+    s_f[i] = mq == -INFINITY ? 0.f : __expf(mq - s_m[i % G]);  // an empty range adds nothing
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * (D + 1); idx += kGThreads) {
+    const int h = idx / (D + 1), c = idx % (D + 1);
+    const float* src = st0 + (c < D ? 2 * G + h * D + c : G + h);
     float v = 0.f;
-    for (int q = 0; q < a.splits; ++q) {
-      const float* sq = st0 + int64_t(q) * G * (D + 2);
-      const float mq = __ldcg(sq + h);
-      if (mq != -INFINITY) v = fmaf(__ldcg(sq + 2 * G + i), __expf(mq - s_m[h]), v);
-    }
-    s_acc[i] = v;
+#pragma unroll 16
+    for (int q = 0; q < S; ++q) v = fmaf(s_f[q * G + h], __ldcg(src + q * sstride), v);
+    if (c < D) s_acc[h * D + c] = v;
+    else s_l[h] = v;
   }
   __syncthreads();
   // H (unnormalised, Sylvester order) per head, in place
@@ -209,53 +249,58 @@ __global__ void __launch_bounds__(kGThreads) attention_value_kernel(const AttnGe
   if (tid == 0) a.counters[g] = 0u;  // ready for the next call
 }
 
-template <int G>
-cudaError_t launch_value_g(const AttnGenArgs& a, cudaStream_t stream) {
-  const int grid = a.hkv * a.splits;
-  switch (a.d) {
-    case 64: return launch_pdl(attention_value_kernel<G, 2>, grid, kGThreads, 0, stream, a);
-    case 128: return launch_pdl(attention_value_kernel<G, 4>, grid, kGThreads, 0, stream, a);
-    case 256: return launch_pdl(attention_value_kernel<G, 8>, grid, kGThreads, 0, stream, a);
+using ValueKernel = void (*)(AttnGenArgs);
+
+// The value kernel for (G, d, V bits), or null where none is built.
+template <int G, int B> ValueKernel value_kernel_d(int d) {
+  switch (d) {
+    case 64: return attention_value_kernel<G, 2, B>;
+    case 128: return attention_value_kernel<G, 4, B>;
+    case 256: return attention_value_kernel<G, 8, B>;
     case 512:
-      if constexpr (G <= 4) return launch_pdl(attention_value_kernel<G, 16>, grid, kGThreads, 0, stream, a);
+      if constexpr (G <= 4) return attention_value_kernel<G, 16, B>;
       break;
   }
-  return cudaErrorNotSupported;
+  return nullptr;
+}
+template <int G> ValueKernel value_kernel_g(int d, int bits) {
+  switch (bits) {
+    case 1: return value_kernel_d<G, 1>(d);
+    case 2: return value_kernel_d<G, 2>(d);
+    case 3: return value_kernel_d<G, 3>(d);
+    case 4: return value_kernel_d<G, 4>(d);
+  }
+  return nullptr;
+}
+ValueKernel value_kernel(int group, int d, int bits) {
+  switch (group) {
+    case 1: return value_kernel_g<1>(d, bits);
+    case 2: return value_kernel_g<2>(d, bits);
+    case 4: return value_kernel_g<4>(d, bits);
+    case 8: return value_kernel_g<8>(d, bits);
+  }
+  return nullptr;
 }
 
-// CTAs of the value kernel for (group, d) that one SM holds at once
-int value_ctas_per_sm(int group, int d) {
-  const void* k = nullptr;
-  auto pick = [&](auto g) {
-    constexpr int G = decltype(g)::value;
-    switch (d) {
-      case 64: k = reinterpret_cast<const void*>(attention_value_kernel<G, 2>); break;
-      case 128: k = reinterpret_cast<const void*>(attention_value_kernel<G, 4>); break;
-      case 256: k = reinterpret_cast<const void*>(attention_value_kernel<G, 8>); break;
-      case 512:
-        if constexpr (G <= 4) k = reinterpret_cast<const void*>(attention_value_kernel<G, 16>);
-        break;
-    }
-  };
-  switch (group) {
-    case 1: pick(std::integral_constant<int, 1>()); break;
-    case 2: pick(std::integral_constant<int, 2>()); break;
-    case 4: pick(std::integral_constant<int, 4>()); break;
-    case 8: pick(std::integral_constant<int, 8>()); break;
-  }
+// CTAs of the value kernel for (group, d, V bits) that one SM holds at once, at most three
+int value_ctas_per_sm(int group, int d, int v_bits) {
+  const ValueKernel k = value_kernel(group, d, v_bits);
   int n = 1;
-  if (k == nullptr || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kGThreads, 0) != cudaSuccess || n < 1)
+  if (k == nullptr ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reinterpret_cast<const void*>(k), kGThreads, 0) !=
+          cudaSuccess ||
+      n < 1)
     n = 1;
-  return n > 2 ? 2 : n;
+  return n > 3 ? 3 : n;
 }
 
 }  // namespace
 
-int attention_general_splits(int hkv, int group, int d, int64_t T) {
+int attention_general_splits(int hkv, int group, int d, int v_bits, int64_t T) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // as many CTAs as the SMs hold at once (at most two each), so the grid is one wave
-  int64_t s = int64_t(value_ctas_per_sm(group, d)) * sms / hkv;
+  // as many CTAs as the SMs hold at once (at most three each), so the grid is one wave
+  int64_t s = int64_t(value_ctas_per_sm(group, d, v_bits)) * sms / hkv;
   if (s > kGMaxSplits) s = kGMaxSplits;
   const int64_t most = (T + 4 * kGWarps - 1) / (4 * kGWarps);  // at least 4 tokens per warp
   if (s > most) s = most;
@@ -272,15 +317,15 @@ bool attention_general_supported(int d, int k_bits, int hq, int hkv) {
 
 // counters (padded to 256 bytes) | states hkv × splits × G × (d + 2) floats
 // (padded to 256 bytes) | scores hq × T floats
-size_t attention_general_workspace_bytes(int hq, int hkv, int d, int64_t T) {
-  const int s = attention_general_splits(hkv, hkv > 0 ? hq / hkv : 1, d, T);
+size_t attention_general_workspace_bytes(int hq, int hkv, int d, int v_bits, int64_t T) {
+  const int s = attention_general_splits(hkv, hkv > 0 ? hq / hkv : 1, d, v_bits, T);
   const size_t counters = (size_t(hkv) * 4 + 255) / 256 * 256;
   const size_t states = (size_t(hq) * s * (d + 2) * 4 + 255) / 256 * 256;
   return counters + states + size_t(hq) * size_t(T) * 4;
 }
 
 cudaError_t launch_attention_general(AttnGenArgs a, void* workspace, cudaStream_t stream) {
-  a.splits = attention_general_splits(a.hkv, a.group, a.d, a.T);
+  a.splits = attention_general_splits(a.hkv, a.group, a.d, a.pv.bits, a.T);
   const size_t counters = (size_t(a.hkv) * 4 + 255) / 256 * 256;
   const size_t states = (size_t(a.hq) * a.splits * (a.d + 2) * 4 + 255) / 256 * 256;
   a.counters = static_cast<unsigned*>(workspace);
@@ -289,13 +334,9 @@ cudaError_t launch_attention_general(AttnGenArgs a, void* workspace, cudaStream_
   cudaError_t e = launch_qk_scores(a.q, a.hq, a.k_codes, a.k_norms, a.T, a.hkv, a.d, a.pk, a.scale, a.scores,
                                    stream);
   if (e != cudaSuccess) return e;
-  switch (a.group) {
-    case 1: return launch_value_g<1>(a, stream);
-    case 2: return launch_value_g<2>(a, stream);
-    case 4: return launch_value_g<4>(a, stream);
-    case 8: return launch_value_g<8>(a, stream);
-  }
-  return cudaErrorInvalidValue;
+  const ValueKernel k = value_kernel(a.group, a.d, a.pv.bits);
+  if (k == nullptr) return cudaErrorNotSupported;
+  return launch_pdl(k, a.hkv * a.splits, kGThreads, 0, stream, a);
 }
 
 }  // namespace rrq

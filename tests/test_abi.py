@@ -179,9 +179,10 @@ def test_attention_splits_fill_the_sms_in_one_wave(hq, hkv):
 def test_general_attention_workspace(hq, hkv, d):
     """Shapes other than d = 128 with 4-bit K and V: counters (256-byte padded), the
     ranges' partial states (hq × ranges × (d + 2) floats, 256-byte padded), then the
-    scores (hq × T floats); as many CTAs as the SMs hold at once (one or two each, by
-    the value kernel's occupancy: one when no device is visible), at most 296 ranges
-    per kv head, at least 32 tokens per range, at least one range."""
+    scores (hq × T floats); as many CTAs as the SMs hold at once (one to three each, by
+    the occupancy of the value kernel for that d and V bit width: one when no device is
+    visible), at most 444 ranges per kv head, at least 32 tokens per range, at least
+    one range."""
     import torch
     lib = B.lib()
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
@@ -189,8 +190,8 @@ def test_general_attention_workspace(hq, hkv, d):
     for t_len in (1, 100, 4096, 1 << 17):
         ws = lib.rrq_attention_workspace_bytes(hq, hkv, d, 2, 3, t_len)
         sizes = []
-        for per_sm in (1, 2):
-            s = max(1, min(per_sm * sms // hkv, 296, (t_len + 31) // 32))
+        for per_sm in (1, 2, 3):
+            s = max(1, min(per_sm * sms // hkv, 444, (t_len + 31) // 32))
             sizes.append(counters + (hq * s * (d + 2) * 4 + 255) // 256 * 256 + hq * t_len * 4)
         assert ws in sizes, (ws, sizes)
         if not torch.cuda.is_available():
