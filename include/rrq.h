@@ -304,10 +304,12 @@ int rrq_attention_decode_noalloc(const void* q, int hq, const uint8_t* k_codes,
 /*
  * rrq_attention_workspace_bytes — the workspace rrq_attention_decode needs for
  * (hq, hkv, d, k_bits, v_bits, T) on the current device (it depends on the SM
- * count), or 0 for an invalid shape.  d = 128 with 4-bit K and V needs the
- * counters and partial states only (well under 1 MB for 32 query heads); every
- * other shape adds hq × T floats of scores.  No CUDA work beyond reading the
- * device's attributes.
+ * count and, for the shapes other than d = 128 with 4-bit K and V, on how many
+ * CTAs of the value kernel for that d and V width one SM holds), or 0 for an
+ * invalid shape.  d = 128 with 4-bit K and V needs the counters and partial
+ * states only (well under 1 MB for 32 query heads); every other shape adds
+ * hq × T floats of scores.  No CUDA work beyond reading the device's attributes
+ * and the kernels' occupancy.
  */
 size_t rrq_attention_workspace_bytes(int hq, int hkv, int d, int k_bits, int v_bits, int64_t T);
 
