@@ -187,8 +187,8 @@ def test_general_attention_workspace(hq, hkv, d):
     lib = B.lib()
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
     counters = (hkv * 4 + 255) // 256 * 256
-    for t_len in (1, 100, 4096, 1 << 17):
-        ws = lib.rrq_attention_workspace_bytes(hq, hkv, d, 2, 3, t_len)
+    for t_len, v_bits in ((1, 3), (100, 1), (4096, 2), (1 << 17, 3), (1 << 17, 4)):
+        ws = lib.rrq_attention_workspace_bytes(hq, hkv, d, 2, v_bits, t_len)
         sizes = []
         for per_sm in (1, 2, 3):
             s = max(1, min(per_sm * sms // hkv, 444, (t_len + 31) // 32))
