@@ -28,7 +28,6 @@
 // shared-memory Walsh–Hadamard transform per head), writes the output and sets
 // the counter back to zero.  No CTA waits for another.  Everything is fp32.
 #include <cmath>
-#include <type_traits>
 
 #include "attention.h"
 #include "rrq_device.cuh"
